@@ -1,0 +1,385 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- a number printed on the pages, a library routine, a closed form, an
+invariant or an exact brute-force computation -- so that a dropped term, a
+wrong sign or index, or a transposed operand in the oracle fails one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+G = 128
+
+
+# ----------------------------------------------------------------- IEEE types
+def test_half_decode_exhaustive_vs_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros keep their sign
+    assert math.copysign(1.0, oracle.half_to_double(0x8000)) == -1.0
+
+
+def test_half_encode_rne_vs_numpy():
+    g = synth.rng(1)
+    vals = np.concatenate([
+        g.standard_normal(20000) * 10.0 ** g.integers(-9, 6, 20000),
+        g.uniform(-70000, 70000, 2000),
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e9, -1e9, 2.0 ** -24, 2.0 ** -25,
+         2.0 ** -25 * 1.0000001, 3 * 2.0 ** -26, 2.0 ** -14, 2.0 ** -14 * (1 - 2.0 ** -12)],
+    ])
+    # exact midpoints between consecutive representable halves (ties -> even)
+    mids = []
+    for b in range(0x0000, 0x7BFF, 97):
+        lo = np.uint16(b).view(np.float16).astype(np.float64)
+        hi = np.uint16(b + 1).view(np.float16).astype(np.float64)
+        mids += [(lo + hi) / 2, -(lo + hi) / 2]
+    vals = np.concatenate([vals, mids])
+    ref = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.double_to_half(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_decode_exhaustive_vs_torch():
+    torch = pytest.importorskip("torch")
+    bits = np.arange(65536, dtype=np.int64)
+    t = torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([oracle.bf16_to_double(int(b)) for b in bits])
+    nan = np.isnan(t)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], t[~nan])
+
+
+def test_bf16_encode_rne_vs_torch():
+    torch = pytest.importorskip("torch")
+    g = synth.rng(2)
+    vals = g.standard_normal(20000) * 10.0 ** g.integers(-30, 30, 20000)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([oracle.double_to_bf16(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------ page facts
+def _facts(golden_dir):
+    with open(os.path.join(golden_dir, "page_facts.json")) as f:
+        return json.load(f)
+
+
+def test_bits_per_weight_page_facts(golden_dir):
+    facts = _facts(golden_dir)
+    assert oracle.effective_bits("q1g128") == facts["binary_bits_per_weight"]["value"]
+    # 2-bit slots and 5 trits per byte (+ the FP16 scale)
+    assert oracle.effective_bits("t2g128") == 2.0 + 16 / 128
+    assert oracle.effective_bits("t5p8") == 26 * 8 / 128 + 16 / 128
+    # the ~1.71 figure is the information content log2(3) plus the scale share;
+    # 5-per-byte storage sits between it and the 2-bit slots
+    entropy = math.log2(3) + 16 / 128
+    assert round(entropy, 2) == facts["ternary_effective_bits"]["value"]
+    assert entropy < oracle.effective_bits("t5p8") < oracle.effective_bits("t2g128")
+
+
+def test_trit_packing_bounds(golden_dir):
+    facts = _facts(golden_dir)
+    tb = facts["trits_per_byte"]
+    assert 3 ** tb["trits"] <= 2 ** tb["bits"] < 3 ** (tb["trits"] + 1)
+    assert tb["bits"] / tb["trits"] == tb["bits_per_trit"]
+    t27 = facts["trits_per_27_bits"]
+    assert 3 ** t27["trits"] <= 2 ** t27["bits"]
+    assert round(t27["bits"] / t27["trits"], 3) == t27["bits_per_trit"]
+    # a 128-trit group in 5-per-byte storage: 25 full bytes + one byte of 3
+    assert oracle.codes_bytes("t5p8", 1, 128) == 26 == math.ceil(128 / tb["trits"])
+
+
+def test_table2_byte_count_identity(golden_dir):
+    t2 = _facts(golden_dir)["table2_bytes"]
+    params = t2["fp16_safetensors"] // 2
+    assert params * 2 == t2["fp16_safetensors"]
+    # params = rows x 128: codes + scales of the binary format
+    rows = params // 128
+    assert rows * 128 == params
+    total = oracle.codes_bytes("q1g128", rows, 128) + oracle.scales_bytes(rows, 128)
+    assert total == t2["gguf_q1_0_g128"]
+
+
+def test_sign_convention(golden_dir):
+    sc = _facts(golden_dir)["binary_sign_convention"]
+    row = np.zeros(16, dtype=np.uint8)
+    row[0] = 0b10  # weight 0 -> bit 0, weight 1 -> bit 1
+    assert oracle.weight_code("q1g128", row, 0) == sc["bit0"]
+    assert oracle.weight_code("q1g128", row, 1) == sc["bit1"]
+
+
+# --------------------------------------------------------------- packing
+def test_pack_binary_signs_and_zero():
+    w = np.zeros((1, G), dtype=np.float32)
+    w[0, :4] = [1.0, -1.0, 0.0, -0.0]
+    w[0, 4:] = np.linspace(-2, 2, G - 4, dtype=np.float32)
+    codes, scales = oracle.pack("q1g128", w)
+    q = oracle.unpack("q1g128", codes, 1, G)[0]
+    assert list(q[:4]) == [1, -1, 1, 1]  # zero (either sign) maps to +1
+    assert np.array_equal(q[4:], np.where(w[0, 4:] >= 0, 1, -1))
+    # LSB-first bit order inside each byte
+    assert codes[0] & 1 == 1 and (codes[0] >> 1) & 1 == 0
+
+
+def test_scale_is_fp16_of_mean_abs_and_l2_optimal():
+    g = synth.rng(3)
+    w = synth.weights_normal(g, 8, 4 * G)
+    codes, scales = oracle.pack("q1g128", w)
+    s = scales.view(np.float16).astype(np.float64).reshape(8, 4)
+    wg = w.astype(np.float64).reshape(8, 4, G)
+    mean_abs = np.abs(wg).mean(axis=2)
+    assert np.array_equal(scales.reshape(8, 4), mean_abs.astype(np.float16).view(np.uint16))
+    # closed form: for fixed signs, argmin_a sum (w - a sign(w))^2 = mean |w|
+    sgn = np.where(wg >= 0, 1.0, -1.0)
+    def sse(a):
+        return ((wg - a[..., None] * sgn) ** 2).sum(axis=2)
+    for d in (1e-4, -1e-4):
+        assert np.all(sse(mean_abs) < sse(mean_abs + d))
+    assert np.all(np.abs(s - mean_abs) <= np.abs(mean_abs) * 2.0 ** -11 + 2.0 ** -25)
+
+
+def test_ternary_threshold_is_clamped_round_half_even():
+    s_bits = np.array([[np.float16(0.03125).view(np.uint16)]], dtype=np.uint16)
+    s = 0.03125
+    vals = np.array([0, s / 2, -s / 2, np.nextafter(np.float32(s / 2), np.float32(1)),
+                     -np.nextafter(np.float32(s / 2), np.float32(1)), s, -s, 1.5 * s, 3 * s,
+                     -7 * s, 1e-9, -1e-9], dtype=np.float32)
+    w = np.zeros((1, G), dtype=np.float32)
+    w[0, :vals.size] = vals
+    for fmt in ("t2g128", "t5p8"):
+        codes, scales = oracle.pack(fmt, w, scales_in=s_bits)
+        q = oracle.unpack(fmt, codes, 1, G)[0, :vals.size]
+        ref = np.clip(np.rint(vals.astype(np.float64) / s), -1, 1).astype(np.int8)
+        assert np.array_equal(q, ref), fmt
+
+
+def test_ternary_mean_abs_scale_matches_binary_rule():
+    g = synth.rng(4)
+    w = synth.weights_normal(g, 4, 2 * G)
+    _, s1 = oracle.pack("q1g128", w)
+    for fmt in ("t2g128", "t5p8"):
+        _, st = oracle.pack(fmt, w)
+        assert np.array_equal(s1, st)
+
+
+@pytest.mark.parametrize("fmt", ["t2g128", "t5p8"])
+def test_ternary_given_scale_roundtrip(fmt):
+    g = synth.rng(5)
+    n, k = 7, 3 * G
+    t = synth.trits(g, n, k)
+    s = synth.scales_uniform(g, n, k // G)
+    w = t.astype(np.float32) * np.repeat(synth.fp16_bits_to_float32(s), G, axis=1)
+    codes, scales = oracle.pack(fmt, w, scales_in=s)
+    assert np.array_equal(scales, s.reshape(-1))
+    assert np.array_equal(oracle.unpack(fmt, codes, n, k), t)
+
+
+def test_t2_code_layout_and_invalid_pattern():
+    # trits -1, 0, +1, 0 -> codes 0, 1, 2, 1 at bits 0,2,4,6
+    w = np.zeros((1, G), dtype=np.float32)
+    w[0, :4] = [-1, 0, 1, 0]
+    codes, _ = oracle.pack("t2g128", w, scales_in=np.array([[0x3C00]], dtype=np.uint16))
+    assert codes[0] == (0 | 1 << 2 | 2 << 4 | 1 << 6)
+    assert oracle.codes_bytes("t2g128", 1, G) == 32
+    bad = codes.copy()
+    bad[0] |= 3  # the unused fourth pattern
+    with pytest.raises(oracle.OracleError):
+        oracle.unpack("t2g128", bad, 1, G)
+
+
+def test_t5p8_every_byte_value_decodes_as_base3():
+    row = np.zeros(26, dtype=np.uint8)
+    for v in range(256):
+        row[0] = v
+        got = [oracle.weight_code("t5p8", row, i) for i in range(5)]
+        if v >= 243:
+            assert all(c == -2 for c in got)
+            continue
+        digits = [int(ch) for ch in np.base_repr(v, 3).zfill(5)[::-1]]  # least significant first
+        assert got == [d - 1 for d in digits]
+    for v in range(256):  # tail byte of a group holds three trits
+        row[25] = v
+        got = [oracle.weight_code("t5p8", row, 125 + i) for i in range(3)]
+        if v >= 27:
+            assert all(c == -2 for c in got)
+        else:
+            assert got == [int(ch) - 1 for ch in np.base_repr(v, 3).zfill(3)[::-1]]
+
+
+def test_pack_errors():
+    w = np.ones((2, G), dtype=np.float32)
+    assert oracle.pack_status("q1g128", np.ones((2, 100), dtype=np.float32))[0] == oracle.ERR_SHAPE
+    wn = w.copy(); wn[1, 5] = np.nan
+    assert oracle.pack_status("q1g128", wn)[0] == oracle.ERR_NONFINITE
+    wi = w.copy(); wi[0, 0] = np.inf
+    assert oracle.pack_status("t2g128", wi)[0] == oracle.ERR_NONFINITE
+    big = np.full((1, G), 70000.0, dtype=np.float32)
+    assert oracle.pack_status("q1g128", big)[0] == oracle.ERR_SCALE_RANGE
+    ok_big = np.full((1, G), 65504.0, dtype=np.float32)
+    assert oracle.pack_status("q1g128", ok_big)[0] == oracle.OK
+    neg = np.array([[0xBC00]], dtype=np.uint16)
+    assert oracle.pack_status("t2g128", np.ones((1, G), np.float32), neg)[0] == oracle.ERR_SCALE_RANGE
+    assert oracle.pack_status("t5p8", np.zeros((0, G), np.float32))[0] == oracle.OK
+
+
+# --------------------------------------------------------------- products
+def _exact_dot(t_row, s_row, x_row):
+    """Exact rational sum_g s_g sum_k t_k x_k from the ORIGINAL trits/signs."""
+    acc = Fraction(0)
+    for gi in range(len(s_row)):
+        s = Fraction(float(np.uint16(s_row[gi]).view(np.float16)))
+        p = Fraction(0)
+        for i in range(G):
+            kk = gi * G + i
+            xv = Fraction(float(x_row[kk]))
+            p += int(t_row[kk]) * xv
+        acc += s * p
+    return acc
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+def test_brute_force_tiny_exact(fmt):
+    import torch
+    g = synth.rng(6)
+    n, k, b = 5, 2 * G, 3
+    if fmt == "q1g128":
+        t = np.where(g.random((n, k)) < 0.5, -1, 1).astype(np.int8)
+    else:
+        t = synth.trits(g, n, k)
+    s = synth.scales_uniform(g, n, k // G)
+    w = t.astype(np.float32) * np.repeat(synth.fp16_bits_to_float32(s), G, axis=1)
+    codes, scales = oracle.pack(fmt, w, scales_in=s)
+    x = synth.x_bf16(g, b, k)
+    xf = torch.from_numpy(x.astype(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    y, bound = oracle.matmul(fmt, codes, scales, n, k, x)
+    for bi in range(b):
+        for r in range(n):
+            ex = _exact_dot(t[r], s[r], xf[bi])
+            assert abs(Fraction(y[bi, r]) - ex) <= abs(ex) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 80)
+            sab = sum(abs(Fraction(float(np.uint16(s[r, kk // G]).view(np.float16))) * Fraction(float(xf[bi, kk])))
+                      for kk in range(k))
+            assert abs(Fraction(bound[bi, r]) - sab) <= sab * Fraction(1, 2 ** 50)
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+def test_matmul_vs_numpy_matmul(fmt):
+    import torch
+    g = synth.rng(7)
+    n, k, b = 64, 8 * G, 4
+    w = synth.weights_normal(g, n, k)
+    codes, scales = oracle.pack(fmt, w)
+    x = synth.x_bf16(g, b, k)
+    xf = torch.from_numpy(x.astype(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    wd = oracle.dequant(fmt, codes, scales, n, k)
+    ref = xf @ wd.T  # library primitive
+    y, bound = oracle.matmul(fmt, codes, scales, n, k, x)
+    assert np.allclose(y, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    s_rep = np.repeat(scales.view(np.float16).astype(np.float64).reshape(n, -1), G, axis=1)
+    assert np.allclose(bound, np.abs(xf) @ s_rep.T, rtol=1e-13, atol=0)
+
+
+def test_closed_form_all_ones_x_binary():
+    g = synth.rng(8)
+    n, k = 6, 3 * G
+    codes = synth.code_bytes_uniform(g, oracle.codes_bytes("q1g128", n, k))
+    scales = synth.scales_uniform(g, n, k // G).reshape(-1)
+    x = np.full((1, k), 0x3F80, dtype=np.uint16)  # BF16 1.0
+    y, _ = oracle.matmul("q1g128", codes, scales, n, k, x)
+    cb = codes.reshape(n, k // 8)
+    for r in range(n):
+        exp = 0.0
+        for gi in range(k // G):
+            pop = sum(bin(int(v)).count("1") for v in cb[r, gi * 16:(gi + 1) * 16])
+            exp += float(np.uint16(scales[r * (k // G) + gi]).view(np.float16)) * (2 * pop - G)
+        assert y[0, r] == exp
+
+
+@pytest.mark.parametrize("fmt", ["t2g128", "t5p8"])
+def test_closed_form_all_ones_x_ternary(fmt):
+    g = synth.rng(9)
+    n, k = 5, 2 * G
+    t = synth.trits(g, n, k)
+    s = synth.scales_uniform(g, n, k // G)
+    w = t.astype(np.float32) * np.repeat(synth.fp16_bits_to_float32(s), G, axis=1)
+    codes, scales = oracle.pack(fmt, w, scales_in=s)
+    x = np.full((1, k), 0x3F80, dtype=np.uint16)
+    y, _ = oracle.matmul(fmt, codes, scales, n, k, x)
+    tg = t.reshape(n, k // G, G)
+    exp = ((tg == 1).sum(axis=2) - (tg == -1).sum(axis=2)) * s.view(np.float16).astype(np.float64)
+    assert np.array_equal(y[0], exp.sum(axis=1))
+
+
+@pytest.mark.parametrize("fmt", ["t2g128", "t5p8"])
+def test_all_zero_trits_give_exact_zero(fmt):
+    n, k = 3, 2 * G
+    w = np.zeros((n, k), dtype=np.float32)
+    s = np.full((n, k // G), 0x3C00, dtype=np.uint16)
+    codes, scales = oracle.pack(fmt, w, scales_in=s)
+    x = synth.x_bf16(synth.rng(10), 2, k)
+    y, _ = oracle.matmul(fmt, codes, scales, n, k, x)
+    assert np.all(y == 0.0)
+
+
+def test_flipping_every_bit_negates_binary():
+    g = synth.rng(11)
+    n, k = 9, 4 * G
+    codes = synth.code_bytes_uniform(g, oracle.codes_bytes("q1g128", n, k))
+    scales = synth.scales_uniform(g, n, k // G).reshape(-1)
+    x = synth.x_bf16(g, 2, k)
+    y, _ = oracle.matmul("q1g128", codes, scales, n, k, x)
+    y2, _ = oracle.matmul("q1g128", codes ^ 0xFF, scales, n, k, x)
+    assert np.array_equal(y2, -y)
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+def test_one_hot_x_returns_effective_weight_column(fmt):
+    g = synth.rng(12)
+    n, k = 7, 2 * G
+    w = synth.weights_normal(g, n, k)
+    codes, scales = oracle.pack(fmt, w)
+    wd = oracle.dequant(fmt, codes, scales, n, k)
+    for col in (0, 1, 127, 128, 255):
+        x = np.zeros((1, k), dtype=np.uint16)
+        x[0, col] = 0x3F80
+        y, _ = oracle.matmul(fmt, codes, scales, n, k, x)
+        assert np.array_equal(y[0], wd[:, col])
+        # and the column is s * q with the page's sign meaning
+        s = scales.view(np.float16).astype(np.float64).reshape(n, -1)[:, col // G]
+        q = oracle.unpack(fmt, codes, n, k)[:, col]
+        assert np.array_equal(wd[:, col], s * q)
+
+
+def test_small_integer_exact_product():
+    # power-of-two scales and small-integer activations: the product is an exact integer
+    g = synth.rng(13)
+    n, k = 4, 2 * G
+    t = synth.trits(g, n, k)
+    s = np.full((n, k // G), np.float16(2.0).view(np.uint16), dtype=np.uint16)
+    w = t.astype(np.float32) * 2.0
+    codes, scales = oracle.pack("t2g128", w, scales_in=s)
+    xi = g.integers(-8, 9, size=(1, k))
+    x = synth.float32_to_bf16_bits(xi.astype(np.float32))
+    y, _ = oracle.matmul("t2g128", codes, scales, n, k, x)
+    assert np.array_equal(y[0], 2.0 * (t.astype(np.int64) @ xi[0]).astype(np.float64))
+
+
+def test_rows_variant_matches_full():
+    g = synth.rng(14)
+    n, k = 50, 2 * G
+    w = synth.weights_normal(g, n, k)
+    codes, scales = oracle.pack("t5p8", w)
+    x = synth.x_bf16(g, 3, k)
+    y, b = oracle.matmul("t5p8", codes, scales, n, k, x)
+    rows = np.array([49, 0, 17, 17, 3])
+    yr, br = oracle.matmul_rows("t5p8", codes, scales, n, k, x, rows)
+    assert np.array_equal(yr, y[:, rows]) and np.array_equal(br, b[:, rows])
