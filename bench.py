@@ -1,0 +1,382 @@
+"""Benchmark of the weight-streaming g128 GEMV on B200.
+
+Default workload (one step = one decode weight pass, batch 1): the Qwen3-8B
+shapes -- 36 layers x (q 4096x4096, k 1024x4096, v 1024x4096, o 4096x4096,
+gate 12288x4096, up 12288x4096, down 4096x12288) + LM head 151936x4096 -- every
+layer with its own binary g128 weights (codes+scales 1.06 GB per pass, larger
+than the 126 MB L2, so no flush is needed between steps).  Weights are packed
+on the GPU from N(0, 0.02) floats; x ~ N(0,1) BF16.
+
+Prints ONE JSON line (rank 0).  ``value`` = effective weight GB/s (codes +
+scales bytes streamed per step / device time per step, summed over ranks);
+``e2e`` = the same through the public API with the activations copied from
+pinned host memory and every output copied back inside the timed region.
+``--impl reference`` times the CPU oracle (the plain FP64 definition) on a
+bounded sample of the same workload.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; N > 1 under torchrun,
+one independent replica per GPU (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FMT_NAMES = {"q1g128": 1, "t2g128": 2, "t5p8": 3}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--fmt", choices=list(FMT_NAMES), default="q1g128")
+    p.add_argument("--batch", type=int, default=1)
+    p.add_argument("--layers", type=int, default=36)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def layer_shapes():
+    import synth
+    return list(synth.QWEN3_8B_LAYER.items())
+
+
+def workload_name(fmt, batch, layers):
+    return (f"qwen3-8b-shapes {fmt} GEMV batch {batch}: {layers} x (q 4096x4096, k/v 1024x4096, "
+            f"o 4096x4096, gate/up 12288x4096, down 4096x12288) + LM head 151936x4096, "
+            f"distinct weights per layer")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        loaded = [v for v in sm if smax and v > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ reference
+def run_reference(args):
+    """The CPU oracle as it stands, on a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    import synth
+    fmt = args.fmt
+    n, k = synth.QWEN3_8B_LAYER["q"]
+    g = synth.rng(synth.SEED_BASE + 1)
+    codes = synth.code_bytes_uniform(g, oracle.codes_bytes(fmt, n, k)) if fmt == "q1g128" else None
+    if codes is None:
+        t = synth.trits(g, n, k)
+        s = synth.scales_uniform(g, n, k // 128)
+        w = t.astype(np.float32) * np.repeat(synth.fp16_bits_to_float32(s), 128, axis=1)
+        codes, scales = oracle.pack(fmt, w, scales_in=s)
+    else:
+        scales = synth.scales_uniform(g, n, k // 128).reshape(-1)
+    x = synth.x_bf16(g, args.batch, k)
+    wbytes = codes.nbytes + scales.nbytes
+    for _ in range(args.warmup):
+        oracle.matmul(fmt, codes, scales, n, k, x)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.matmul(fmt, codes, scales, n, k, x)
+        times.append(time.perf_counter() - t0)
+    ms = 1000.0 * sum(times) / len(times)
+    value = wbytes / (ms / 1000.0) / 1e9
+    sample = f"one q matrix 4096x4096 ({fmt}, batch {args.batch}) per step"
+    line = {
+        "impl": "reference", "metric": "effective weight GB/s (g128 GEMV weight stream)",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(fmt, args.batch, args.layers), "fmt": fmt,
+                   "batch": args.batch, "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(fmt, mats, x_by_k, batch):
+    """Oracle on a bounded sample (the LM head plus the first layer), host cores."""
+    import numpy as np
+    import torch
+    import oracle
+    sample = [mats[-1]] + mats[:7]  # LM head + the first layer's seven matrices
+    host = []
+    for (name, n, k, codes, scales, _) in sample:
+        host.append((name, n, k, codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16),
+                     x_by_k[k][:batch].view(torch.int16).cpu().numpy().view(np.uint16)))
+    total_bytes, t0 = 0, time.perf_counter()
+    for (name, n, k, c, s, x) in host:
+        oracle.matmul(fmt, c, s, n, k, x)
+        total_bytes += c.nbytes + s.nbytes
+    dt = time.perf_counter() - t0
+    return {"value": round(total_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"LM head 151936x4096 + one layer's 7 matrices ({fmt}, batch {batch}), "
+                      f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------- ours
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    fmt, batch = args.fmt, args.batch
+    f = FMT_NAMES[fmt]
+    gen = synth.device_generator(synth.SEED_BASE + 1 + 1000 * rank, device=dev)
+
+    # ---- weights: distinct per layer, packed on the GPU
+    mats = []  # (name, n, k, codes, scales, y)
+    shapes = []
+    for layer in range(args.layers):
+        for name, (n, k) in layer_shapes():
+            shapes.append((f"L{layer}.{name}", n, k))
+    shapes.append(("lm_head",) + synth.QWEN3_8B_LM_HEAD)
+    for (name, n, k) in shapes:
+        if fmt == "q1g128":
+            w = synth.device_weights_normal(gen, n, k, device=dev)
+            codes, scales = bq.bq_pack(fmt, w)
+        else:
+            t = synth.device_trits(gen, n, k, device=dev)
+            s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
+            w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
+            codes, scales = bq.bq_pack(fmt, w, scales_in=s)
+        del w
+        y = torch.empty((batch, n), dtype=torch.bfloat16, device=dev)
+        mats.append((name, n, k, codes, scales, y))
+    torch.cuda.synchronize()
+    x_by_k = {k: synth.device_x_bf16(gen, batch, k, device=dev) for k in sorted({k for _, _, k in shapes})}
+    ws_need = max(bq.bq_gemv_workspace_bytes(f, n, k, batch) for _, n, k in shapes)
+    workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
+    weight_bytes = sum(c.numel() + 2 * s.numel() for (_, _, _, c, s, _) in mats)
+    algo_bytes = weight_bytes + sum(2 * k * batch + 2 * n * batch for (_, n, k, _, _, _) in mats)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        for i, (name, n, k, codes, scales, y) in enumerate(mats):
+            if events is not None:
+                events[i][0].record(stream)
+            bq.bq_gemv(f, codes, scales, n, k, x_by_k[k], y=y, workspace=workspace, stream=stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    assert bq.bq_check() == bq.BQ_OK
+
+    # ---- device-timed region (per-launch events for the roofline)
+    launch_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in mats] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s_i in range(args.steps):
+        step(launch_ev[s_i])
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    assert bq.bq_check() == bq.BQ_OK
+    per_launch = []
+    for s_i in range(args.steps):
+        for i in range(len(mats)):
+            per_launch.append(launch_ev[s_i][i][0].elapsed_time(launch_ev[s_i][i][1]))
+    kernel_ms_per_step = sum(per_launch) / args.steps
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        ks = sorted(x_by_k)
+        x_host = {k: torch.empty_like(x_by_k[k], device="cpu").pin_memory() for k in ks}
+        for k in ks:
+            x_host[k].copy_(x_by_k[k])
+        y_host = [torch.empty_like(m[5], device="cpu").pin_memory() for m in mats]
+        h2d = d2h = 0
+
+        def e2e_step():
+            nonlocal h2d, d2h
+            h2d_b = d2h_b = 0
+            for i, (name, n, k, codes, scales, y) in enumerate(mats):
+                x_by_k[k].copy_(x_host[k], non_blocking=True)
+                h2d_b += x_host[k].numel() * 2
+                bq.bq_gemv(f, codes, scales, n, k, x_by_k[k], y=y, workspace=workspace, stream=stream)
+                y_host[i].copy_(y, non_blocking=True)
+                d2h_b += y.numel() * 2
+            h2d, d2h = h2d_b, d2h_b
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        e2e = {"ms_per_step": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    # ---- max over ranks
+    ms_per_step = elapsed_ms / args.steps
+    if dist is not None:
+        t = torch.tensor([ms_per_step, e2e["ms_per_step"] if e2e else 0.0], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step, e2e_ms_max = float(t[0]), float(t[1])
+        if e2e:
+            e2e["ms_per_step"] = e2e_ms_max
+
+    peak, peak_src = measured_peaks()
+    total_weight_bytes = weight_bytes * world
+    value = total_weight_bytes / (ms_per_step / 1000.0) / 1e9
+    achieved = algo_bytes / (kernel_ms_per_step / 1000.0) / 1e9
+    traffic_path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    traffic = None
+    if os.path.exists(traffic_path):
+        with open(traffic_path) as fh:
+            tr = json.load(fh)
+        if tr.get("fmt") == fmt and tr.get("batch") == batch and tr.get("kernel_rev") == bq.bq_version():
+            traffic = tr.get("bytes_per_step")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(fmt, mats, x_by_k, batch)
+
+    if rank == 0:
+        line = {
+            "metric": "effective weight GB/s (g128 GEMV weight stream)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": workload_name(fmt, batch, args.layers), "fmt": fmt, "batch": batch,
+                       "weight_bytes_per_step": weight_bytes, "launches_per_step": len(mats),
+                       "l2": "inputs larger than L2 (weights per step > 126 MB), no flush",
+                       "parallelism": f"replicas x{world}"},
+            "hbm_roofline_pct": round(100.0 * value / world / peak, 2),
+            "tokens_per_s_equiv": round(1000.0 / ms_per_step, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                         "kernel": "bq GEMV, all launches of a step",
+                         "algorithmic_bytes_per_step": algo_bytes,
+                         "kernel_ms_per_step": round(kernel_ms_per_step, 4)},
+            "clocks": clocks,
+            "gpu_launches": len(mats) * args.steps,
+        }
+        if e2e:
+            line["e2e"] = {"value": round(total_weight_bytes / (e2e["ms_per_step"] / 1000.0) / 1e9, 2),
+                           "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                           "d2h_bytes_per_step": e2e["d2h"]}
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,162 @@
+/*
+ * bq.h -- C ABI of the binary / ternary g128 weight library for NVIDIA B200
+ * (sm_100a).
+ *
+ * What it computes.  End-to-end low-bit weights as described on the pages
+ *   "Bonsai-27B-mlx-1bit ... Binary g128 权重表示" (section "Binary g128权重表示原理"),
+ *   "Ternary Bonsai" (section "什么是Ternary Bonsai技术"),
+ *   "把 27B 模型压到 4GB 跑在手机上" (section 2.4, trit storage), and
+ *   "1-bit Bonsai 8B" notes (section 2 "内存带宽是真正的瓶颈", section 4.1 Q1_0_g128,
+ *   Table 3 tg128 / pp512):
+ * every weight is a code q in {-1,+1} (binary) or {-1,0,+1} (ternary), every
+ * 128 consecutive weights of a row share one FP16 scale s, and the effective
+ * weight is s*q.  Products decode the codes inside the kernel; no FP16 copy of
+ * W is ever written to memory.
+ *
+ * Shapes and layouts (all row-major, no padding between rows):
+ *   W        N x K, K % 128 == 0, G = K/128 groups per row.
+ *   scales   uint16 FP16 bit patterns [N][G]; scales[r][g] covers weights
+ *            r, 128g .. 128g+127.
+ *   codes    BQ_Q1G128  : [N][K/8]  bytes; weight k at bit (k&7) of byte k>>3,
+ *                         bit 1 -> +1, bit 0 -> -1.          1.125 bits/weight
+ *            BQ_T2G128  : [N][K/4]  bytes; code c = q+1 in bits 2(k&3)..+1 of
+ *                         byte k>>2; c == 3 is not a valid code. 2.125 bits/weight
+ *            BQ_T5P8G128: [N][26*G] bytes; in group g, byte j < 25 holds
+ *                         v = sum_{i<5} (q_{128g+5j+i}+1) 3^i, byte 25 holds the
+ *                         last three codes the same way.      1.75 bits/weight
+ *   x        BF16 bit patterns [B][K] (GEMV) or [T][K] (GEMM), contiguous.
+ *   y        [B][N] (GEMV, BF16 or F32) or [T][N] (GEMM, BF16).
+ *
+ * Ownership.  Every pointer argument of the compute calls is a DEVICE pointer
+ * owned by the caller.  The library allocates no memory and keeps no pointer
+ * after a call returns.  Workspaces are caller-allocated device buffers of at
+ * least the size the matching *_workspace_bytes call reports.
+ *
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ * default stream).  bq_gemv and bq_gemm only enqueue work and return; they do
+ * not synchronise.  The packers synchronise `stream` before returning because
+ * their status (non-finite input, scale overflow) is produced on the device.
+ *
+ * Errors.  Argument errors are detected on the host before anything is
+ * launched and returned synchronously; nothing is written.  A launch failure
+ * returns BQ_ERR_CUDA.  Asynchronous faults and device-side time-outs of
+ * bounded waits surface through bq_check().  Invalid codes (a 2-bit code of 3,
+ * a base-3 byte >= 243) give unspecified output values, never a fault.
+ *
+ * Precision.  Activations are read as BF16, products accumulate in FP32 with
+ * one scale multiply per group; every output satisfies
+ *   |y - y_exact| <= 2e-3 * sum_k |s_{g(k)} x_k|
+ * plus the final rounding to the output type (for BF16 output at most
+ * 2^-8 |y|).
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_NULL = 1,        /* a required pointer is NULL */
+    BQ_ERR_SHAPE = 2,       /* K % 128 != 0, a negative size, batch out of range */
+    BQ_ERR_ALIGN = 3,       /* a pointer is not aligned as documented */
+    BQ_ERR_NONFINITE = 4,   /* packer input holds NaN or +-Inf */
+    BQ_ERR_SCALE_RANGE = 5, /* a scale would exceed FP16, or a given scale is negative / non-finite */
+    BQ_ERR_FORMAT = 6,      /* unknown format or output dtype */
+    BQ_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch error, sticky fault) */
+    BQ_ERR_TIMEOUT = 8,     /* a bounded device wait gave up (reported by bq_check) */
+    BQ_ERR_WORKSPACE = 9    /* workspace NULL or smaller than *_workspace_bytes */
+} bq_status;
+
+typedef enum { BQ_Q1G128 = 1, BQ_T2G128 = 2, BQ_T5P8G128 = 3 } bq_format;
+typedef enum { BQ_BF16 = 0, BQ_F32 = 1 } bq_dtype;
+
+#define BQ_GROUP 128
+#define BQ_MAX_BATCH 16
+
+/* ------------------------------------------------------------------ sizes */
+/* Bytes of the code array for an N x K matrix; -1 for an invalid format or
+ * shape (negative size or K % 128 != 0). */
+int64_t bq_codes_bytes(int fmt, int64_t n, int64_t k);
+/* Bytes of the FP16 scale array, N * (K/128) * 2; -1 for an invalid shape. */
+int64_t bq_scales_bytes(int64_t n, int64_t k);
+/* Storage bits per weight including the scale: 1.125, 2.125, 1.75; -1 if invalid. */
+double bq_effective_bits(int fmt);
+
+/* ---------------------------------------------------------------- packers */
+/* Float weights -> codes + FP16 scales (one thread per 128-weight group).
+ * Reading of the pages, which do not state the rule for trained weights:
+ *   s = FP16 round-to-nearest-even of (sum of |w| over the group, summed in
+ *       order in FP64) / 128, unless `scales_in` gives the scales;
+ *   binary : q = +1 if w >= 0 (both zeros give +1), else -1;
+ *   ternary: q = 0 if |w| <= s/2, else sign(w)  (= clamp(round-half-even(w/s))).
+ * w        device float32 [N][K], 16-byte aligned.
+ * scales_in device FP16 [N][G] or NULL; each must be finite and non-negative.
+ * codes    device [bq_codes_bytes] bytes; scales device FP16 [N][G].
+ * Returns BQ_ERR_NONFINITE / BQ_ERR_SCALE_RANGE if any group fails (then the
+ * outputs are unspecified).  Synchronises `stream`.  The result is bit-exact
+ * with the reference definition. */
+bq_status bq_pack_q1g128(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                         uint8_t* codes, uint16_t* scales, void* stream);
+bq_status bq_pack_t2g128(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                         uint8_t* codes, uint16_t* scales, void* stream);
+bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                       uint8_t* codes, uint16_t* scales, void* stream);
+
+/* ------------------------------------------------------------------- GEMV */
+/* Workspace bytes bq_gemv needs for this call shape (0 when none is needed);
+ * -1 for an invalid format or shape. */
+int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
+
+/* y[b][r] = sum_g s[r][g] * sum_{k in g} q[r][k] * x[b][k],   b < batch <= 16.
+ * The weight-streaming decode product ("1-bit Bonsai 8B" section 2: token
+ * generation is bound by streaming the weights; section 4.1: codes decoded
+ * inline in the matmul).
+ * codes/scales as above; x BF16 [batch][K]; y [batch][N] of y_dtype.  The
+ * base of every array (codes, scales, x, y) must be 16-byte aligned.
+ * workspace: device buffer of >= bq_gemv_workspace_bytes bytes (may be NULL
+ * when that is 0), 256-byte aligned; its contents on entry do not matter.
+ * Asynchronous on `stream`. */
+bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                  const uint16_t* x, int batch, void* y, int y_dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------- GEMM */
+/* Workspace bytes bq_gemm needs for T tokens (0 if none); -1 if invalid. */
+int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t);
+
+/* Prefill: Y[t][r] = sum_k X[t][k] * s[r][g(k)] q[r][k] for t < T, BF16 out
+ * ("1-bit Bonsai 8B" summary section 3 and Table 3 pp512: prompt processing is
+ * a dense contraction).  For T <= 16 this is bq_gemv with batch = T.  Larger T
+ * runs a tensor-core (tcgen05) kernel that dequantises W tiles on chip to FP16
+ * s*q (exact) and multiplies by X converted to FP16 with a per-token
+ * power-of-two pre-scale (exact for every BF16 value within 2^-32 of the
+ * token's largest magnitude), accumulating in FP32.
+ * X BF16 [T][K] 16-byte aligned; Y BF16 [T][N] 16-byte aligned; workspace as
+ * bq_gemm_workspace_bytes, 256-byte aligned.  Asynchronous on `stream`. */
+bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                  const uint16_t* x, int64_t t, uint16_t* y,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ errors */
+/* Synchronises `stream`, then reports a pending CUDA error (BQ_ERR_CUDA) or a
+ * device wait that timed out since the last check (BQ_ERR_TIMEOUT, and the
+ * flag is cleared).  BQ_OK otherwise. */
+bq_status bq_check(void* stream);
+/* Test hook for the time-out path: run one kernel that waits on a flag that
+ * nothing sets, with a limit of `spin_limit` polls; it gives up, records
+ * BQ_ERR_TIMEOUT and returns.  Never hangs. */
+bq_status bq_debug_wait_timeout(int64_t spin_limit, void* stream);
+/* Static, NUL-terminated description of a status code. */
+const char* bq_status_string(int status);
+/* Library version as 10000*major + 100*minor + patch. */
+int bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BQ_H */

@@ -53,14 +53,17 @@ def float32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
 
 
 def weights_normal(g: np.random.Generator, n: int, k: int, std: float = 0.02) -> np.ndarray:
-    return g.normal(0.0, std, size=(n, k)).astype(np.float32)
+    w = g.standard_normal(size=(n, k), dtype=np.float32)
+    w *= np.float32(std)
+    return w
 
 
-def trits(g: np.random.Generator, n: int, k: int, p_neg=0.35, p_zero=0.30) -> np.ndarray:
-    u = g.random(size=(n, k))
+def trits(g: np.random.Generator, n: int, k: int) -> np.ndarray:
+    """P(-1) = P(+1) = 7/20 = 0.35, P(0) = 6/20 = 0.30."""
+    u = g.integers(0, 20, size=(n, k), dtype=np.uint8)
     t = np.ones((n, k), dtype=np.int8)
-    t[u < p_neg + p_zero] = 0
-    t[u < p_neg] = -1
+    t[u < 13] = 0
+    t[u < 7] = -1
     return t
 
 
@@ -70,7 +73,7 @@ def scales_uniform(g: np.random.Generator, n: int, groups: int, lo=0.005, hi=0.0
 
 
 def x_bf16(g: np.random.Generator, batch: int, k: int) -> np.ndarray:
-    return float32_to_bf16_bits(g.standard_normal(size=(batch, k)).astype(np.float32))
+    return float32_to_bf16_bits(g.standard_normal(size=(batch, k), dtype=np.float32))
 
 
 def code_bytes_uniform(g: np.random.Generator, nbytes: int) -> np.ndarray:
@@ -80,3 +83,44 @@ def code_bytes_uniform(g: np.random.Generator, nbytes: int) -> np.ndarray:
 def fp16_bits_to_float32(h: np.ndarray) -> np.ndarray:
     """Storage decoding used to build w = t * s for given-scale packing."""
     return np.asarray(h, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+# ------------------------------------------------------------ on the device
+# Full-size workloads (up to 1.3e9 weights) are drawn on the GPU with a seeded
+# torch generator; the oracle reads back whatever rows it checks.
+def device_generator(seed: int, device="cuda"):
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return gen
+
+
+def device_weights_normal(gen, n: int, k: int, std: float = 0.02, device="cuda"):
+    import torch
+    return torch.randn((n, k), generator=gen, device=device, dtype=torch.float32) * std
+
+
+def device_trits(gen, n: int, k: int, device="cuda"):
+    import torch
+    u = torch.randint(0, 20, (n, k), generator=gen, device=device, dtype=torch.int16)
+    t = torch.ones((n, k), device=device, dtype=torch.int8)
+    t[u < 13] = 0
+    t[u < 7] = -1
+    return t
+
+
+def device_scales_uniform(gen, n: int, groups: int, lo=0.005, hi=0.05, device="cuda"):
+    """FP16 bit patterns (int16 tensor) of uniform draws in [lo, hi]."""
+    import torch
+    u = torch.rand((n, groups), generator=gen, device=device, dtype=torch.float32)
+    return (lo + (hi - lo) * u).to(torch.float16).view(torch.int16)
+
+
+def device_x_bf16(gen, batch: int, k: int, device="cuda"):
+    import torch
+    return torch.randn((batch, k), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def device_code_bytes(gen, nbytes: int, device="cuda"):
+    import torch
+    return torch.randint(0, 256, (nbytes,), generator=gen, device=device, dtype=torch.int16).to(torch.uint8)

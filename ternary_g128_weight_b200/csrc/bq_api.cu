@@ -1,0 +1,212 @@
+// C ABI entry points: argument validation on the host, dispatch to the
+// kernels, device status words and their read-back.  Nothing here computes
+// on the data path.
+#include <mutex>
+
+#include "bq_internal.cuh"
+
+namespace bq {
+
+namespace {
+
+__device__ int g_device_status = 0;
+__device__ unsigned long long g_pack_first_error = ~0ull;
+
+std::mutex g_pack_mutex;
+
+inline bool fmt_ok(int fmt) { return fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128; }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+__global__ void wait_never_set_kernel(int64_t spin_limit, const volatile int* flag, int* status) {
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    for (int64_t i = 0; i < spin_limit; ++i) {
+        if (*flag != 0) return;
+        __nanosleep(32);
+    }
+    record_status(status, BQ_ERR_TIMEOUT);
+}
+
+__device__ int g_never_set_flag = 0;
+
+bq_status validate_matrix(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k) {
+    if (!fmt_ok(fmt)) return BQ_ERR_FORMAT;
+    if (n < 0 || k < 0 || k % kGroup != 0) return BQ_ERR_SHAPE;
+    if (n > 0 && k > 0) {
+        if (!codes || !scales) return BQ_ERR_NULL;
+        if (!aligned(codes, 16) || !aligned(scales, 16)) return BQ_ERR_ALIGN;
+    }
+    return BQ_OK;
+}
+
+bq_status pack_common(int fmt, const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                      uint8_t* codes, uint16_t* scales, void* stream) {
+    if (!fmt_ok(fmt)) return BQ_ERR_FORMAT;
+    if (n < 0 || k < 0 || k % kGroup != 0) return BQ_ERR_SHAPE;
+    if (n == 0 || k == 0) return BQ_OK;
+    if (!w || !codes || !scales) return BQ_ERR_NULL;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 16) ||
+        (scales_in && !aligned(scales_in, 16)))
+        return BQ_ERR_ALIGN;
+    std::lock_guard<std::mutex> lock(g_pack_mutex);
+    cudaStream_t s = as_stream(stream);
+    const unsigned long long none = ~0ull;
+    if (cudaMemcpyToSymbolAsync(g_pack_first_error, &none, sizeof(none), 0,
+                                cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    unsigned long long* first_ptr = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&first_ptr), g_pack_first_error) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (launch_pack(fmt, w, n, k, scales_in, codes, scales, first_ptr, s) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    unsigned long long first = 0;
+    if (cudaMemcpyFromSymbolAsync(&first, g_pack_first_error, sizeof(first), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BQ_ERR_CUDA;
+    if (first != ~0ull) return static_cast<bq_status>(first & 0xFF);
+    return BQ_OK;
+}
+
+}  // namespace
+
+int* device_status_ptr() {
+    int* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_status) != cudaSuccess) return nullptr;
+    return p;
+}
+
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" {
+
+int64_t bq_codes_bytes(int fmt, int64_t n, int64_t k) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup) return -1;
+    if (fmt == BQ_Q1G128) return n * (k / 8);
+    if (fmt == BQ_T2G128) return n * (k / 4);
+    return n * (k / kGroup) * 26;
+}
+
+int64_t bq_scales_bytes(int64_t n, int64_t k) {
+    if (n < 0 || k < 0 || k % kGroup) return -1;
+    return n * (k / kGroup) * 2;
+}
+
+double bq_effective_bits(int fmt) {
+    if (!fmt_ok(fmt)) return -1.0;
+    return 8.0 * (double)(bq_codes_bytes(fmt, 1, kGroup) + 2) / (double)kGroup;
+}
+
+bq_status bq_pack_q1g128(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                         uint8_t* codes, uint16_t* scales, void* stream) {
+    return pack_common(BQ_Q1G128, w, n, k, scales_in, codes, scales, stream);
+}
+bq_status bq_pack_t2g128(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                         uint8_t* codes, uint16_t* scales, void* stream) {
+    return pack_common(BQ_T2G128, w, n, k, scales_in, codes, scales, stream);
+}
+bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                       uint8_t* codes, uint16_t* scales, void* stream) {
+    return pack_common(BQ_T5P8G128, w, n, k, scales_in, codes, scales, stream);
+}
+
+int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
+    return 0;
+}
+
+bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                  const uint16_t* x, int batch, void* y, int y_dtype, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    bq_status st = validate_matrix(fmt, codes, scales, n, k);
+    if (st != BQ_OK) return st;
+    if (batch < 1 || batch > BQ_MAX_BATCH) return BQ_ERR_SHAPE;
+    if (y_dtype != BQ_BF16 && y_dtype != BQ_F32) return BQ_ERR_FORMAT;
+    if (n == 0) return BQ_OK;
+    if (!y || (k > 0 && !x)) return BQ_ERR_NULL;
+    if (!aligned(y, 16) || (x && !aligned(x, 16))) return BQ_ERR_ALIGN;
+    const int64_t need = bq_gemv_workspace_bytes(fmt, n, k, batch);
+    if (need > 0 && (!workspace || workspace_bytes < (size_t)need)) return BQ_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return BQ_ERR_ALIGN;
+    if (k == 0) {
+        const size_t bytes = (size_t)batch * n * (y_dtype == BQ_F32 ? 4 : 2);
+        return cudaMemsetAsync(y, 0, bytes, as_stream(stream)) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    }
+    if (launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, as_stream(stream)) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    return BQ_OK;
+}
+
+int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
+    return 0;
+}
+
+bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                  const uint16_t* x, int64_t t, uint16_t* y, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+    bq_status st = validate_matrix(fmt, codes, scales, n, k);
+    if (st != BQ_OK) return st;
+    if (t < 0) return BQ_ERR_SHAPE;
+    if (n == 0 || t == 0) return BQ_OK;
+    if (!y || (k > 0 && !x)) return BQ_ERR_NULL;
+    if (!aligned(y, 16) || (x && !aligned(x, 16))) return BQ_ERR_ALIGN;
+    const int64_t need = bq_gemm_workspace_bytes(fmt, n, k, t);
+    if (need > 0 && (!workspace || workspace_bytes < (size_t)need)) return BQ_ERR_WORKSPACE;
+    if (workspace && !aligned(workspace, 256)) return BQ_ERR_ALIGN;
+    cudaStream_t s = as_stream(stream);
+    if (k == 0)
+        return cudaMemsetAsync(y, 0, (size_t)t * n * 2, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    for (int64_t t0 = 0; t0 < t; t0 += BQ_MAX_BATCH) {
+        const int b = (int)((t - t0) < BQ_MAX_BATCH ? (t - t0) : BQ_MAX_BATCH);
+        if (launch_gemv_simt(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, s) != cudaSuccess)
+            return BQ_ERR_CUDA;
+    }
+    return BQ_OK;
+}
+
+bq_status bq_check(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BQ_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpyFromSymbol(&st, g_device_status, sizeof(st)) != cudaSuccess) return BQ_ERR_CUDA;
+    if (st != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return BQ_ERR_CUDA;
+        return static_cast<bq_status>(st);
+    }
+    return BQ_OK;
+}
+
+bq_status bq_debug_wait_timeout(int64_t spin_limit, void* stream) {
+    if (spin_limit < 0) return BQ_ERR_SHAPE;
+    int* flag = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&flag), g_never_set_flag) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    int* status = device_status_ptr();
+    if (!status) return BQ_ERR_CUDA;
+    wait_never_set_kernel<<<1, 32, 0, as_stream(stream)>>>(spin_limit, flag, status);
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+const char* bq_status_string(int status) {
+    switch (status) {
+        case BQ_OK: return "ok";
+        case BQ_ERR_NULL: return "null pointer";
+        case BQ_ERR_SHAPE: return "invalid shape (K % 128 != 0, negative size or batch out of range)";
+        case BQ_ERR_ALIGN: return "pointer not aligned as required";
+        case BQ_ERR_NONFINITE: return "non-finite weight (NaN or Inf)";
+        case BQ_ERR_SCALE_RANGE: return "scale out of FP16 range, negative or non-finite";
+        case BQ_ERR_FORMAT: return "unknown format or output dtype";
+        case BQ_ERR_CUDA: return "CUDA runtime error";
+        case BQ_ERR_TIMEOUT: return "device wait timed out";
+        case BQ_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int bq_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bq.h"
+
+namespace bq {
+
+constexpr int kGroup = 128;
+
+// Device-side status words live in bq_api.cu; kernels receive their
+// addresses as arguments.
+//   status      : first error of a bounded device wait that gave up.
+//   pack_first  : first failing group of a packer call, encoded
+//                 (group index << 8) | status, so that the error reported is the
+//                 one of the lowest (row, group) as in the sequential
+//                 definition; ~0 means none.
+__device__ __forceinline__ void record_status(int* status, int st) {
+    atomicCAS(status, 0, st);
+}
+
+__device__ __forceinline__ void record_pack_error(unsigned long long* first, int64_t group_index, int st) {
+    atomicMin(first, ((unsigned long long)group_index << 8) | (unsigned)st);
+}
+
+// Address of the device status word of the current device.
+int* device_status_ptr();
+
+// BF16 bit pattern -> float (exact).
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+// Low / high BF16 of a packed pair -> float.
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Host-side launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_pack(int fmt, const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
+                        uint8_t* codes, uint16_t* scales, unsigned long long* first_error,
+                        cudaStream_t s);
+cudaError_t launch_gemv_simt(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n,
+                             int64_t k, const uint16_t* x, int batch, void* y, int y_dtype,
+                             cudaStream_t s);
+cudaError_t launch_wait_timeout(int64_t spin_limit, cudaStream_t s);
+
+}  // namespace bq

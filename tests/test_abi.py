@@ -1,0 +1,112 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every symbol include/bq.h declares, its host helpers agree with the oracle,
+and argument errors are returned before anything touches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import ternary_g128_weight_b200 as bq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(bq_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ternary_g128_weight_b200 import build
+    build.build()
+    return bq.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    decl = declared_symbols()
+    assert {"bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8", "bq_gemv", "bq_gemm"} <= decl
+    for name in decl:
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+    assert set(bq.EXPORTED) == decl
+
+
+def test_enums_match_oracle():
+    assert (bq.BQ_Q1G128, bq.BQ_T2G128, bq.BQ_T5P8G128) == (oracle.Q1G128, oracle.T2G128, oracle.T5P8G128)
+    assert (bq.BQ_OK, bq.BQ_ERR_NULL, bq.BQ_ERR_SHAPE, bq.BQ_ERR_ALIGN, bq.BQ_ERR_NONFINITE,
+            bq.BQ_ERR_SCALE_RANGE, bq.BQ_ERR_FORMAT) == (
+        oracle.OK, oracle.ERR_NULL, oracle.ERR_SHAPE, oracle.ERR_ALIGN, oracle.ERR_NONFINITE,
+        oracle.ERR_SCALE_RANGE, oracle.ERR_FORMAT)
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+@pytest.mark.parametrize("n,k", [(0, 128), (1, 128), (7, 1024), (151936, 4096), (3, 100), (-1, 128)])
+def test_sizes_match_oracle(lib, fmt, n, k):
+    assert bq.bq_codes_bytes(fmt, n, k) == oracle.codes_bytes(fmt, n, k)
+    assert bq.bq_scales_bytes(n, k) == oracle.scales_bytes(n, k)
+    assert bq.bq_effective_bits(fmt) == oracle.effective_bits(fmt)
+
+
+def test_status_strings_and_version(lib):
+    for s in range(10):
+        assert len(bq.status_string(s)) > 0
+    assert bq.status_string(99) == "unknown status"
+    assert bq.bq_version() >= 100
+
+
+def _gemv(lib, fmt=1, codes=16, scales=16, n=4, k=128, x=16, batch=1, y=16, ydt=0, ws=None, wsb=0):
+    vp = ctypes.c_void_p
+    return lib.bq_gemv(fmt, vp(codes) if codes else None, vp(scales) if scales else None, n, k,
+                       vp(x) if x else None, batch, vp(y) if y else None, ydt,
+                       vp(ws) if ws else None, wsb, None)
+
+
+def test_argument_errors_need_no_device(lib):
+    # host validation happens before any CUDA call, so these run without a GPU
+    assert _gemv(lib, fmt=9) == bq.BQ_ERR_FORMAT
+    assert _gemv(lib, k=100) == bq.BQ_ERR_SHAPE
+    assert _gemv(lib, n=-1) == bq.BQ_ERR_SHAPE
+    assert _gemv(lib, batch=0) == bq.BQ_ERR_SHAPE
+    assert _gemv(lib, batch=17) == bq.BQ_ERR_SHAPE
+    assert _gemv(lib, codes=0) == bq.BQ_ERR_NULL
+    assert _gemv(lib, x=0) == bq.BQ_ERR_NULL
+    assert _gemv(lib, y=0) == bq.BQ_ERR_NULL
+    assert _gemv(lib, codes=24) == bq.BQ_ERR_ALIGN
+    assert _gemv(lib, x=8) == bq.BQ_ERR_ALIGN
+    assert _gemv(lib, ydt=5) == bq.BQ_ERR_FORMAT
+    vp = ctypes.c_void_p
+    assert lib.bq_gemm(1, vp(16), vp(16), 4, 130, vp(16), 5, vp(16), None, 0, None) == bq.BQ_ERR_SHAPE
+    assert lib.bq_gemm(1, vp(16), vp(16), 4, 128, vp(16), -1, vp(16), None, 0, None) == bq.BQ_ERR_SHAPE
+    assert lib.bq_gemm(4, vp(16), vp(16), 4, 128, vp(16), 5, vp(16), None, 0, None) == bq.BQ_ERR_FORMAT
+    for name in ("bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8"):
+        f = getattr(lib, name)
+        assert f(vp(16), 4, 127, None, vp(16), vp(16), None) == bq.BQ_ERR_SHAPE
+        assert f(None, 4, 128, None, vp(16), vp(16), None) == bq.BQ_ERR_NULL
+        assert f(vp(20), 4, 128, None, vp(16), vp(16), None) == bq.BQ_ERR_ALIGN
+        assert f(vp(16), 0, 128, None, None, None, None) == bq.BQ_OK  # empty: nothing to do
+    assert lib.bq_gemv_workspace_bytes(1, 4, 100, 1) == -1
+    assert lib.bq_gemv_workspace_bytes(1, 4, 128, 17) == -1
+    assert lib.bq_gemv_workspace_bytes(1, 4096, 4096, 1) >= 0
+    assert lib.bq_gemm_workspace_bytes(2, 4096, 4096, 512) >= 0
+    assert lib.bq_debug_wait_timeout(-1, None) == bq.BQ_ERR_SHAPE
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import importlib
+    mod = importlib.import_module("ternary_g128_weight_b200")
+    saved = mod._lib
+    try:
+        mod._lib = None
+        with pytest.raises(RuntimeError, match="no CPU fallback"):
+            mod.load(str(tmp_path / "missing.so"))
+    finally:
+        mod._lib = saved
