@@ -114,7 +114,7 @@ bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* sca
 
 int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
-    return 0;
+    return gemv_tc_workspace_bytes(fmt, n, k, batch);
 }
 
 bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -134,14 +134,27 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
         const size_t bytes = (size_t)batch * n * (y_dtype == BQ_F32 ? 4 : 2);
         return cudaMemsetAsync(y, 0, bytes, as_stream(stream)) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     }
-    if (launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, as_stream(stream)) != cudaSuccess)
-        return BQ_ERR_CUDA;
-    return BQ_OK;
+    cudaError_t e;
+    if (need > 0 && gemv_tc_eligible(fmt, n, k, batch))
+        e = launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, as_stream(stream));
+    else
+        e = launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, as_stream(stream));
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+// Token chunk the GEMM hands to the GEMV kernels while no tensor-core GEMM
+// covers the shape: 4 (tensor-core decode path) or 16 (CUDA-core path).
+static int gemm_chunk(int fmt, int64_t n, int64_t k, int64_t t) {
+    const int c = (int)(t < 4 ? t : 4);
+    return (c > 0 && gemv_tc_eligible(fmt, n, k, c)) ? 4 : BQ_MAX_BATCH;
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
-    return 0;
+    if (t == 0) return 0;
+    const int chunk = gemm_chunk(fmt, n, k, t);
+    const int b = (int)(t < chunk ? t : chunk);
+    return gemv_tc_workspace_bytes(fmt, n, k, b);
 }
 
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -159,10 +172,15 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     cudaStream_t s = as_stream(stream);
     if (k == 0)
         return cudaMemsetAsync(y, 0, (size_t)t * n * 2, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
-    for (int64_t t0 = 0; t0 < t; t0 += BQ_MAX_BATCH) {
-        const int b = (int)((t - t0) < BQ_MAX_BATCH ? (t - t0) : BQ_MAX_BATCH);
-        if (launch_gemv_simt(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, s) != cudaSuccess)
-            return BQ_ERR_CUDA;
+    const int chunk = gemm_chunk(fmt, n, k, t);
+    for (int64_t t0 = 0; t0 < t; t0 += chunk) {
+        const int b = (int)((t - t0) < chunk ? (t - t0) : chunk);
+        cudaError_t e;
+        if (need > 0 && gemv_tc_eligible(fmt, n, k, b))
+            e = launch_gemv_tc(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, workspace, s);
+        else
+            e = launch_gemv_simt(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, s);
+        if (e != cudaSuccess) return BQ_ERR_CUDA;
     }
     return BQ_OK;
 }

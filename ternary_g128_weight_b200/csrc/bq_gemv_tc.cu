@@ -1,0 +1,512 @@
+// Weight-streaming GEMV with tensor-core accumulation of the decoded codes
+// (binary g128 and 2-bit-slot ternary g128, batch 1..4).
+//
+// Why the tensor core: at batch 1 the binary format must be consumed at
+// ~126 weights per clock per SM to stream HBM at 80% of its bandwidth, while
+// the integer/logic pipe retires 64 operations per clock per SM; any CUDA-core
+// decode that spends half an operation per weight cannot get there (the
+// "1-bit Bonsai 8B" notes, section 4.4, observe the same shift of inline
+// dequantisation towards compute).  So the codes are expanded with a handful of
+// LOP3s into int8 operands and the multiply-accumulate runs on mma.sync:
+//
+//   binary  : byte j of (w & (0x01010101 << p)) is 2^p * bit(8j+p) of the code
+//             word w -- eight masks turn one 32-bit word into eight operand
+//             registers with no shift.  The activation operand of that k-slot
+//             carries Q_k / 2^p, so the product is bit * Q_k exactly.
+//   2-bit   : byte j of ((w >> 2i) & 0x03030303) is the code c = q+1 of trit
+//             4j+i; the activation operand carries Q_k.
+//
+// Q_k is the activation in fixed point: per (batch row b, group g) a power of
+// two 2^E maps the group's largest |x| into [2^29, 2^30); Q = round(x 2^E)
+// (binary: rounded to a multiple of 2^7 so that Q / 2^p stays an integer).
+// Q is split into four signed base-256 digits, one MMA column each, and the
+// int32 column sums are recombined in FP32.  Per group and row:
+//   binary : y += s * (2 * 2^-E * sum_k bit_k Q_k - 2^-E * sum_k Q_k)
+//   ternary: y += s * (    2^-E * sum_k c_k   Q_k - 2^-E * sum_k Q_k)
+// (sum of s * q * x with q = 2 bit - 1, resp. q = c - 1; "Bonsai-27B ...
+// Binary g128" section on the representation: 0 -> -scale, 1 -> +scale).  The
+// only rounding before the FP32 recombination is that of x to Q: at most
+// 2^6 units of 2^-E per element, i.e. 2^-23 of the group's largest |x|.
+//
+// Data movement: per pipeline stage (1024 weights of K for 128 rows) a
+// producer warp issues a TMA tile load of the codes (128-byte swizzle), one of
+// the FP16 scales and a bulk copy of the prepared activation operands into
+// shared memory; four compute warps read conflict-free from there.  K is split
+// across CTAs when the matrix has too few rows to fill the GPU; the last CTA of
+// a row block adds the partial sums in a fixed order (deterministic).
+#include <cuda.h>
+
+#include "bq_internal.cuh"
+#include "bq_ptx.cuh"
+
+namespace bq {
+namespace tc {
+
+constexpr int kGroupsPerStage = 8;
+constexpr int kRowsPerCta = 128;
+constexpr int kComputeWarps = 4;
+constexpr int kRowTiles = 2;  // 16-row MMA tiles per compute warp
+constexpr int kThreads = (kComputeWarps + 1) * 32;
+constexpr int kBfragBytesPerGroup = 4 * 32 * 8;  // 4 MMAs x 32 lanes x (b0, b1)
+constexpr int kTableBytesPerGroup = 4 * 16;      // 4 lanes-in-quad x float4
+constexpr int kXTileBytes = kGroupsPerStage * (kBfragBytesPerGroup + kTableBytesPerGroup);  // 8704
+constexpr uint32_t kWaitPolls = 1u << 23;
+
+template <int FMT>
+struct Fmt;
+template <>
+struct Fmt<BQ_Q1G128> {
+    static constexpr int kRowBytesPerStage = 128;  // 8 groups x 16 bytes
+    static constexpr int kCoefShift = 1;           // y uses 2 * sum(bit * x) - sum(x)
+};
+template <>
+struct Fmt<BQ_T2G128> {
+    static constexpr int kRowBytesPerStage = 256;  // 8 groups x 32 bytes
+    static constexpr int kCoefShift = 0;           // y uses sum(c * x) - sum(x)
+};
+
+template <int FMT, int NT>
+struct Layout {
+    static constexpr int kCodesBytes = kRowsPerCta * Fmt<FMT>::kRowBytesPerStage;
+    static constexpr int kScalesBytes = kRowsPerCta * kGroupsPerStage * 2;
+    static constexpr int kXBytes = NT * kXTileBytes;
+    static constexpr int kStageBytes = (kCodesBytes + kScalesBytes + kXBytes + 1023) / 1024 * 1024;
+    static constexpr int kStages = (FMT == BQ_Q1G128 && NT == 1) ? 4 : 3;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 2 * kStages * 8;
+};
+
+struct Params {
+    const uint8_t* xdata;     // prepared activation operands, [stage][NT][kXTileBytes]
+    float* partial;           // [splits][batch][n] when splits > 1
+    unsigned int* counters;   // [row_blocks], zeroed by the prep kernel
+    void* y;
+    int y_dtype;
+    int batch;
+    int64_t n;
+    int stages_total;
+    int splits;
+    int* status;
+};
+
+__device__ __forceinline__ void named_barrier_compute() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
+}
+
+// ----------------------------------------------------------------- prep
+// One CTA per stage (8 groups).  Writes, for each n-tile (two batch rows x four
+// digits), the B fragments of the 32 MMAs of the stage in lane order and the
+// per-(group, lane-in-quad) recombination table {2^a, 2^b, sum term, 0}.
+template <int FMT, int NT>
+__global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int64_t k, int batch,
+                                                   uint8_t* __restrict__ xdata, unsigned int* counters,
+                                                   int row_blocks) {
+    __shared__ int8_t dig[2 * NT][kGroupsPerStage * 128][4];
+    const int st = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (st == 0)
+        for (int i = threadIdx.x; i < row_blocks; i += blockDim.x) counters[i] = 0u;
+    uint8_t* out = xdata + (size_t)st * NT * kXTileBytes;
+
+    const int G = warp;  // 8 warps <-> 8 groups of the stage
+    const int64_t kbase = ((int64_t)st * kGroupsPerStage + G) * 128;
+    for (int bb = 0; bb < 2 * NT; ++bb) {
+        float xv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (bb < batch) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(x + bb * k + kbase + lane * 4);
+            xv[0] = bf16_lo(raw.x); xv[1] = bf16_hi(raw.x); xv[2] = bf16_lo(raw.y); xv[3] = bf16_hi(raw.y);
+        }
+        float m = fmaxf(fmaxf(fabsf(xv[0]), fabsf(xv[1])), fmaxf(fabsf(xv[2]), fabsf(xv[3])));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const int E = (m > 0.f) ? 29 - ilogbf(m) : 0;
+        long long sumq = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int kk = lane * 4 + i;  // position in the group
+            int q, b;
+            if (FMT == BQ_Q1G128) {
+                q = __float2int_rn(ldexpf(xv[i], E - 7)) * 128;
+                b = q >> (kk & 7);  // exact: q is a multiple of 2^7
+            } else {
+                q = __float2int_rn(ldexpf(xv[i], E));
+                b = q;
+            }
+            sumq += q;
+            const int d0 = (int8_t)(b & 0xFF);
+            b = (b - d0) >> 8;
+            const int d1 = (int8_t)(b & 0xFF);
+            b = (b - d1) >> 8;
+            const int d2 = (int8_t)(b & 0xFF);
+            const int d3 = (b - d2) >> 8;
+            int8_t* dst = dig[bb][G * 128 + kk];
+            dst[0] = (int8_t)d0; dst[1] = (int8_t)d1; dst[2] = (int8_t)d2; dst[3] = (int8_t)d3;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sumq += __shfl_xor_sync(0xffffffffu, sumq, off);
+        if (lane < 2) {
+            const int h = lane;  // digit pair (0,1) or (2,3)
+            const int t = 2 * (bb & 1) + h;
+            const int nt = bb >> 1;
+            const int e = Fmt<FMT>::kCoefShift - E + 16 * h;
+            const int a = max(-60, min(60, e));
+            float4 tab;
+            tab.x = ldexpf(1.0f, a);
+            tab.y = ldexpf(1.0f, e - a);
+            tab.z = (h == 0) ? (float)ldexp((double)sumq, -E) : 0.0f;
+            tab.w = 0.0f;
+            *reinterpret_cast<float4*>(out + nt * kXTileBytes + kGroupsPerStage * kBfragBytesPerGroup +
+                                       (G * 4 + t) * 16) = tab;
+        }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < NT * kGroupsPerStage * 4 * 32; idx += blockDim.x) {
+        const int ln = idx & 31, q = (idx >> 5) & 3, g8 = (idx >> 7) & 7, nt = idx >> 10;
+        const int gq = ln >> 2, t = ln & 3;
+        const int bb = nt * 2 + (gq >> 2), dg = gq & 3;
+        uint32_t b0 = 0, b1 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int k0, k1;
+            if (FMT == BQ_Q1G128) {
+                k0 = 32 * t + 8 * j + 2 * q;
+                k1 = k0 + 1;
+            } else {
+                k0 = 16 * t + 4 * j + q;
+                k1 = 16 * (t + 4) + 4 * j + q;
+            }
+            b0 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k0][dg] << (8 * j);
+            b1 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k1][dg] << (8 * j);
+        }
+        *reinterpret_cast<uint2*>(out + nt * kXTileBytes + ((g8 * 4 + q) * 32 + ln) * 8) = make_uint2(b0, b1);
+    }
+}
+
+// ----------------------------------------------------------------- main
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
+                                                              const __grid_constant__ CUtensorMap tm_scales,
+                                                              const Params p) {
+    using L = Layout<FMT, NT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
+    uint64_t* empty = full + L::kStages;
+    __shared__ int s_last;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rb = blockIdx.x, sp = blockIdx.y;
+    const int st0 = (int)((int64_t)sp * p.stages_total / p.splits);
+    const int st1 = (int)((int64_t)(sp + 1) * p.stages_total / p.splits);
+    const int nst = st1 - st0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::kStages; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], kComputeWarps);
+        }
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&tm_codes);
+            ptx::prefetch_tensormap(&tm_scales);
+            int issued = 0;
+            for (int it = 0; it < nst; ++it) {
+                const int slot = it % L::kStages;
+                if (it >= L::kStages &&
+                    !ptx::mbar_wait_bounded(&empty[slot], ((it / L::kStages) - 1) & 1, kWaitPolls)) {
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+                    break;
+                }
+                uint8_t* sb = smem + slot * L::kStageBytes;
+                const int st = st0 + it;
+                ptx::mbar_arrive_expect_tx(&full[slot], L::kCodesBytes + L::kScalesBytes + L::kXBytes);
+#pragma unroll
+                for (int box = 0; box < Fmt<FMT>::kRowBytesPerStage / 128; ++box)
+                    ptx::tma_load_2d(sb + box * (kRowsPerCta * 128), &tm_codes,
+                                     st * Fmt<FMT>::kRowBytesPerStage + box * 128, rb * kRowsPerCta, &full[slot]);
+                ptx::tma_load_2d(sb + L::kCodesBytes, &tm_scales, st * kGroupsPerStage, rb * kRowsPerCta,
+                                 &full[slot]);
+                ptx::bulk_load(sb + L::kCodesBytes + L::kScalesBytes, p.xdata + (size_t)st * L::kXBytes,
+                               L::kXBytes, &full[slot]);
+                issued = it + 1;
+            }
+            // make sure every copy this CTA issued has landed before it may exit
+            for (int it = (issued > L::kStages ? issued - L::kStages : 0); it < issued; ++it)
+                if (!ptx::mbar_wait_bounded(&full[it % L::kStages], (it / L::kStages) & 1, kWaitPolls))
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- compute warps
+    const int g = lane >> 2, t = lane & 3;
+    float yacc[kRowTiles][NT][2];
+#pragma unroll
+    for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
+
+    for (int it = 0; it < nst; ++it) {
+        const int slot = it % L::kStages;
+        if (!ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
+            record_status(p.status, BQ_ERR_TIMEOUT);
+            break;
+        }
+        const uint32_t sb = ptx::smem_u32(smem + slot * L::kStageBytes);
+        const uint32_t codes_s = sb, scales_s = sb + L::kCodesBytes, x_s = sb + L::kCodesBytes + L::kScalesBytes;
+#pragma unroll 1
+        for (int G = 0; G < kGroupsPerStage; ++G) {
+            uint2 bf[NT][4];
+            float4 tab[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    bf[nt][q] = ptx::lds64(x_s + nt * kXTileBytes + ((G * 4 + q) * 32 + lane) * 8);
+                tab[nt] = ptx::lds128f(x_s + nt * kXTileBytes + kGroupsPerStage * kBfragBytesPerGroup +
+                                       (G * 4 + t) * 16);
+            }
+#pragma unroll
+            for (int j = 0; j < kRowTiles; ++j) {
+                const int r0 = warp * (16 * kRowTiles) + j * 16 + g;
+                const float s0 = half_bits_to_float(ptx::lds16(scales_s + r0 * 16 + 2 * G));
+                const float s1 = half_bits_to_float(ptx::lds16(scales_s + (r0 + 8) * 16 + 2 * G));
+                int acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+                if (FMT == BQ_Q1G128) {
+                    const uint32_t off = ((uint32_t)(G ^ g) << 4) + 4 * t;
+                    const uint32_t w0 = ptx::lds32(codes_s + r0 * 128 + off);
+                    const uint32_t w1 = ptx::lds32(codes_s + (r0 + 8) * 128 + off);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
+                        const uint32_t a0 = w0 & m0, a1 = w1 & m0, a2 = w0 & m1, a3 = w1 & m1;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
+                    }
+                } else {
+                    const uint32_t box = codes_s + (G >> 2) * (kRowsPerCta * 128);
+                    const uint32_t c0 = 2 * (G & 3), c1 = c0 + 1;
+                    const uint32_t offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
+                    const uint32_t w0a = ptx::lds32(box + r0 * 128 + offa);
+                    const uint32_t w0b = ptx::lds32(box + r0 * 128 + offb);
+                    const uint32_t w1a = ptx::lds32(box + (r0 + 8) * 128 + offa);
+                    const uint32_t w1b = ptx::lds32(box + (r0 + 8) * 128 + offb);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
+                        const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const float v0 = fmaf(256.0f, (float)acc[nt][1], (float)acc[nt][0]);
+                    const float v1 = fmaf(256.0f, (float)acc[nt][3], (float)acc[nt][2]);
+                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    yacc[j][nt][0] = fmaf(s0, u0, yacc[j][nt][0]);
+                    yacc[j][nt][1] = fmaf(s1, u1, yacc[j][nt][1]);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[slot]);
+    }
+
+    // ---------------------------------------------------- epilogue
+    // lanes t and t^1 hold the low and high digit pairs of the same (row, batch row)
+#pragma unroll
+    for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) yacc[j][nt][r] += __shfl_xor_sync(0xffffffffu, yacc[j][nt][r], 1);
+
+    const bool writer = (t & 1) == 0;
+    if (p.splits == 1) {
+        if (writer) {
+#pragma unroll
+            for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int bb = nt * 2 + (t >> 1);
+                        const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
+                        if (bb < p.batch && row < p.n) {
+                            if (p.y_dtype == BQ_F32)
+                                static_cast<float*>(p.y)[bb * p.n + row] = yacc[j][nt][r];
+                            else
+                                static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[j][nt][r]);
+                        }
+                    }
+        }
+        return;
+    }
+    // split K: publish this CTA's partial sums; the last CTA of the row block adds them in order
+    if (writer) {
+#pragma unroll
+        for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int bb = nt * 2 + (t >> 1);
+                    const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
+                    if (bb < p.batch && row < p.n) p.partial[((int64_t)sp * p.batch + bb) * p.n + row] = yacc[j][nt][r];
+                }
+    }
+    __threadfence();
+    named_barrier_compute();
+    if (threadIdx.x == 0) {
+        const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
+        s_last = (prev == (unsigned int)(p.splits - 1));
+    }
+    named_barrier_compute();
+    if (!s_last) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < kRowsPerCta * p.batch; i += kComputeWarps * 32) {
+        const int bb = i / kRowsPerCta;
+        const int64_t row = (int64_t)rb * kRowsPerCta + (i % kRowsPerCta);
+        if (row >= p.n) continue;
+        float acc = 0.0f;
+        for (int s = 0; s < p.splits; ++s) acc += __ldcg(&p.partial[((int64_t)s * p.batch + bb) * p.n + row]);
+        if (p.y_dtype == BQ_F32)
+            static_cast<float*>(p.y)[bb * p.n + row] = acc;
+        else
+            static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(acc);
+    }
+    if (threadIdx.x == 0) p.counters[rb] = 0u;
+}
+
+// ----------------------------------------------------------------- host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+struct Plan {
+    int nt = 0, stages_total = 0, row_blocks = 0, splits = 0;
+    size_t xdata_bytes = 0, counters_off = 0, partial_off = 0, total = 0;
+};
+
+bool eligible(int fmt, int64_t n, int64_t k, int batch) {
+    return (fmt == BQ_Q1G128 || fmt == BQ_T2G128) && batch >= 1 && batch <= 4 && k > 0 && k % 1024 == 0 &&
+           n > 0 && n <= (int64_t)INT32_MAX && k / 8 <= (int64_t)INT32_MAX / 4;
+}
+
+Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
+    Plan pl;
+    pl.nt = (batch + 1) / 2;
+    pl.stages_total = (int)(k / 1024);
+    pl.row_blocks = (int)((n + kRowsPerCta - 1) / kRowsPerCta);
+    const int ctas_per_sm = (fmt == BQ_Q1G128) ? 2 : 1;
+    const int target = 148 * ctas_per_sm;
+    int splits = (target + pl.row_blocks - 1) / pl.row_blocks;
+    splits = splits < 1 ? 1 : splits;
+    splits = splits > pl.stages_total ? pl.stages_total : splits;
+    pl.splits = splits;
+    pl.xdata_bytes = (size_t)pl.stages_total * pl.nt * kXTileBytes;
+    pl.counters_off = (pl.xdata_bytes + 255) / 256 * 256;
+    pl.partial_off = (pl.counters_off + (size_t)pl.row_blocks * 4 + 255) / 256 * 256;
+    pl.total = pl.partial_off + (splits > 1 ? (size_t)splits * batch * n * 4 : 0);
+    return pl;
+}
+
+template <int FMT, int NT>
+cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
+                         int batch, void* y, int y_dtype, uint8_t* ws, const Plan& pl, cudaStream_t s) {
+    using L = Layout<FMT, NT>;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_tc_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : k / 4;
+    const int64_t G = k / 128;
+    CUtensorMap tm_codes, tm_scales;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n};
+        cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+        cuuint32_t box[2] = {128, (cuuint32_t)kRowsPerCta};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)n};
+        cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
+        cuuint32_t box[2] = {(cuuint32_t)kGroupsPerStage, (cuuint32_t)kRowsPerCta};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(&tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    Params prm;
+    prm.xdata = ws;
+    prm.counters = reinterpret_cast<unsigned int*>(ws + pl.counters_off);
+    prm.partial = reinterpret_cast<float*>(ws + pl.partial_off);
+    prm.y = y;
+    prm.y_dtype = y_dtype;
+    prm.batch = batch;
+    prm.n = n;
+    prm.stages_total = pl.stages_total;
+    prm.splits = pl.splits;
+    prm.status = device_status_ptr();
+    if (!prm.status) return cudaErrorUnknown;
+    prep_kernel<FMT, NT><<<pl.stages_total, 256, 0, s>>>(x, k, batch, ws, prm.counters, pl.row_blocks);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    gemv_tc_kernel<FMT, NT><<<dim3(pl.row_blocks, pl.splits), kThreads, L::kSmemBytes, s>>>(tm_codes, tm_scales, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+
+int64_t gemv_tc_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
+    if (!tc::eligible(fmt, n, k, batch)) return 0;
+    return (int64_t)tc::make_plan(fmt, n, k, batch).total;
+}
+
+bool gemv_tc_eligible(int fmt, int64_t n, int64_t k, int batch) { return tc::eligible(fmt, n, k, batch); }
+
+cudaError_t launch_gemv_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                           const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s) {
+    const tc::Plan pl = tc::make_plan(fmt, n, k, batch);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (fmt == BQ_Q1G128) {
+        if (pl.nt == 1) return tc::launch_typed<BQ_Q1G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, ws, pl, s);
+        return tc::launch_typed<BQ_Q1G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, ws, pl, s);
+    }
+    if (pl.nt == 1) return tc::launch_typed<BQ_T2G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, ws, pl, s);
+    return tc::launch_typed<BQ_T2G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, ws, pl, s);
+}
+
+}  // namespace bq

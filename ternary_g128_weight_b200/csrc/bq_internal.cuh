@@ -55,4 +55,10 @@ cudaError_t launch_gemv_simt(int fmt, const uint8_t* codes, const uint16_t* scal
                              cudaStream_t s);
 cudaError_t launch_wait_timeout(int64_t spin_limit, cudaStream_t s);
 
+// Tensor-core decode GEMV (binary and 2-bit ternary, batch <= 4, K % 1024 == 0).
+bool gemv_tc_eligible(int fmt, int64_t n, int64_t k, int batch);
+int64_t gemv_tc_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
+cudaError_t launch_gemv_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                           const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s);
+
 }  // namespace bq
