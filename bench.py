@@ -48,15 +48,25 @@ def parse():
     return p.parse_args()
 
 
-def layer_shapes():
+def step_shapes(layers):
+    """One decode weight pass: per layer q|k|v (one launch, rows concatenated),
+    o, gate|up (one launch), down; then the LM head."""
     import synth
-    return list(synth.QWEN3_8B_LAYER.items())
+    L = synth.QWEN3_8B_LAYER
+    qkv = (L["q"][0] + L["k"][0] + L["v"][0], L["q"][1])
+    gate_up = (L["gate"][0] + L["up"][0], L["gate"][1])
+    shapes = []
+    for layer in range(layers):
+        shapes += [(f"L{layer}.qkv",) + qkv, (f"L{layer}.o",) + L["o"],
+                   (f"L{layer}.gate_up",) + gate_up, (f"L{layer}.down",) + L["down"]]
+    shapes.append(("lm_head",) + synth.QWEN3_8B_LM_HEAD)
+    return shapes
 
 
 def workload_name(fmt, batch, layers):
-    return (f"qwen3-8b-shapes {fmt} GEMV batch {batch}: {layers} x (q 4096x4096, k/v 1024x4096, "
-            f"o 4096x4096, gate/up 12288x4096, down 4096x12288) + LM head 151936x4096, "
-            f"distinct weights per layer")
+    return (f"qwen3-8b-shapes {fmt} GEMV batch {batch}: {layers} x (q|k|v 6144x4096 [q 4096, k 1024, "
+            f"v 1024 rows], o 4096x4096, gate|up 24576x4096 [2 x 12288 rows], down 4096x12288) + LM head "
+            f"151936x4096, distinct weights per layer, one CUDA graph per step")
 
 
 # --------------------------------------------------------------------- clocks
@@ -169,24 +179,24 @@ def run_reference(args):
     return 0
 
 
-def cpu_baseline(fmt, mats, x_by_k, batch):
+def cpu_baseline(fmt, mats, batch):
     """Oracle on a bounded sample (the LM head plus the first layer), host cores."""
     import numpy as np
     import torch
     import oracle
-    sample = [mats[-1]] + mats[:7]  # LM head + the first layer's seven matrices
+    sample = [mats[-1]] + mats[:4]  # LM head + the first layer's four launches
     host = []
-    for (name, n, k, codes, scales, _) in sample:
-        host.append((name, n, k, codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16),
-                     x_by_k[k][:batch].view(torch.int16).cpu().numpy().view(np.uint16)))
+    for m in sample:
+        host.append((m["n"], m["k"], m["codes"].cpu().numpy(), m["scales"].cpu().numpy().view(np.uint16),
+                     m["x"].view(torch.int16).cpu().numpy().view(np.uint16)))
     total_bytes, t0 = 0, time.perf_counter()
-    for (name, n, k, c, s, x) in host:
+    for (n, k, c, s, x) in host:
         oracle.matmul(fmt, c, s, n, k, x)
         total_bytes += c.nbytes + s.nbytes
     dt = time.perf_counter() - t0
     return {"value": round(total_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
             "kind": "oracle",
-            "sample": f"LM head 151936x4096 + one layer's 7 matrices ({fmt}, batch {batch}), "
+            "sample": f"LM head 151936x4096 + one layer's q|k|v, o, gate|up, down ({fmt}, batch {batch}), "
                       f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s"}
 
 
@@ -211,21 +221,28 @@ def main():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     fmt, batch = args.fmt, args.batch
     f = FMT_NAMES[fmt]
     gen = synth.device_generator(synth.SEED_BASE + 1 + 1000 * rank, device=dev)
+    shapes = step_shapes(args.layers)
 
-    # ---- weights: distinct per layer, packed on the GPU
-    mats = []  # (name, n, k, codes, scales, y)
-    shapes = []
-    for layer in range(args.layers):
-        for name, (n, k) in layer_shapes():
-            shapes.append((f"L{layer}.{name}", n, k))
-    shapes.append(("lm_head",) + synth.QWEN3_8B_LM_HEAD)
-    for (name, n, k) in shapes:
+    # ---- activations and outputs: one contiguous buffer each (one copy per step for e2e)
+    def offsets(sizes):
+        offs, tot = [], 0
+        for sz in sizes:
+            offs.append(tot)
+            tot += (sz + 127) // 128 * 128
+        return offs, tot
+    x_offs, x_tot = offsets([batch * k for _, _, k in shapes])
+    y_offs, y_tot = offsets([batch * n for _, n, _ in shapes])
+    X_all = synth.device_x_bf16(gen, 1, x_tot, device=dev).view(-1)
+    Y_all = torch.zeros(y_tot, dtype=torch.bfloat16, device=dev)
+
+    # ---- weights: distinct per launch, packed on the GPU
+    mats = []
+    for i, (name, n, k) in enumerate(shapes):
         if fmt == "q1g128":
             w = synth.device_weights_normal(gen, n, k, device=dev)
             codes, scales = bq.bq_pack(fmt, w)
@@ -235,23 +252,33 @@ def main():
             w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
             codes, scales = bq.bq_pack(fmt, w, scales_in=s)
         del w
-        y = torch.empty((batch, n), dtype=torch.bfloat16, device=dev)
-        mats.append((name, n, k, codes, scales, y))
+        mats.append({"name": name, "n": n, "k": k, "codes": codes, "scales": scales,
+                     "x": X_all[x_offs[i]:x_offs[i] + batch * k].view(batch, k),
+                     "y": Y_all[y_offs[i]:y_offs[i] + batch * n].view(batch, n)})
     torch.cuda.synchronize()
-    x_by_k = {k: synth.device_x_bf16(gen, batch, k, device=dev) for k in sorted({k for _, _, k in shapes})}
-    ws_need = max(bq.bq_gemv_workspace_bytes(f, n, k, batch) for _, n, k in shapes)
+    ws_need = max(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) for m in mats)
     workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
-    weight_bytes = sum(c.numel() + 2 * s.numel() for (_, _, _, c, s, _) in mats)
-    algo_bytes = weight_bytes + sum(2 * k * batch + 2 * n * batch for (_, n, k, _, _, _) in mats)
-    stream = torch.cuda.current_stream()
+    weight_bytes = sum(m["codes"].numel() + 2 * m["scales"].numel() for m in mats)
+    algo_bytes = weight_bytes + sum(2 * m["k"] * batch + 2 * m["n"] * batch for m in mats)
+    launches_per_step = sum(2 if bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) > 0 else 1 for m in mats)
 
-    def step(events=None):
-        for i, (name, n, k, codes, scales, y) in enumerate(mats):
-            if events is not None:
-                events[i][0].record(stream)
-            bq.bq_gemv(f, codes, scales, n, k, x_by_k[k], y=y, workspace=workspace, stream=stream)
-            if events is not None:
-                events[i][1].record(stream)
+    def step():
+        for m in mats:
+            bq.bq_gemv(f, m["codes"], m["scales"], m["n"], m["k"], m["x"], y=m["y"], workspace=workspace)
+
+    # warm up eagerly (lazy initialisation), then capture one step in a CUDA graph
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert bq.bq_check() == bq.BQ_OK
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stream = torch.cuda.current_stream()
 
     def barrier():
         if dist is not None:
@@ -259,51 +286,56 @@ def main():
         torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
-        step()
+        graph.replay()
+    barrier()
     assert bq.bq_check() == bq.BQ_OK
 
-    # ---- device-timed region (per-launch events for the roofline)
-    launch_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in mats] for _ in range(args.steps)]
+    # ---- device-timed region
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
     barrier()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for s_i in range(args.steps):
-        step(launch_ev[s_i])
+    for _ in range(args.steps):
+        graph.replay()
     t_end.record(stream)
     barrier()
     clocks = sampler.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
     assert bq.bq_check() == bq.BQ_OK
-    per_launch = []
-    for s_i in range(args.steps):
-        for i in range(len(mats)):
-            per_launch.append(launch_ev[s_i][i][0].elapsed_time(launch_ev[s_i][i][1]))
-    kernel_ms_per_step = sum(per_launch) / args.steps
 
-    # ---- end-to-end through the public API with host buffers
+    # ---- LM head alone (largest launch): per-launch time with events around it
+    head = mats[-1]
+    hg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(hg):
+        bq.bq_gemv(f, head["codes"], head["scales"], head["n"], head["k"], head["x"], y=head["y"],
+                   workspace=workspace)
+    hg.replay()
+    torch.cuda.synchronize()
+    h_times = []
+    for _ in range(max(3, args.steps)):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        graph.replay()  # evicts the head's weights from L2 (1 GB streamed)
+        e0.record(stream)
+        hg.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        h_times.append(e0.elapsed_time(e1))
+    head_bytes = head["codes"].numel() + 2 * head["scales"].numel() + 2 * head["k"] * batch + 2 * head["n"] * batch
+    head_ms = statistics.median(h_times)
+
+    # ---- end-to-end through the public API: pinned host inputs in, outputs out
     e2e = None
     if not args.no_e2e:
-        ks = sorted(x_by_k)
-        x_host = {k: torch.empty_like(x_by_k[k], device="cpu").pin_memory() for k in ks}
-        for k in ks:
-            x_host[k].copy_(x_by_k[k])
-        y_host = [torch.empty_like(m[5], device="cpu").pin_memory() for m in mats]
-        h2d = d2h = 0
+        x_host = torch.empty_like(X_all, device="cpu").pin_memory()
+        x_host.copy_(X_all)
+        y_host = torch.empty_like(Y_all, device="cpu").pin_memory()
 
         def e2e_step():
-            nonlocal h2d, d2h
-            h2d_b = d2h_b = 0
-            for i, (name, n, k, codes, scales, y) in enumerate(mats):
-                x_by_k[k].copy_(x_host[k], non_blocking=True)
-                h2d_b += x_host[k].numel() * 2
-                bq.bq_gemv(f, codes, scales, n, k, x_by_k[k], y=y, workspace=workspace, stream=stream)
-                y_host[i].copy_(y, non_blocking=True)
-                d2h_b += y.numel() * 2
-            h2d, d2h = h2d_b, d2h_b
+            X_all.copy_(x_host, non_blocking=True)
+            graph.replay()
+            y_host.copy_(Y_all, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -314,24 +346,23 @@ def main():
             e2e_step()
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        e2e = {"ms_per_step": e2e_ms, "h2d": h2d, "d2h": d2h}
+        e2e = {"ms_per_step": e0.elapsed_time(e1) / args.steps,
+               "h2d": sum(2 * batch * m["k"] for m in mats), "d2h": sum(2 * batch * m["n"] for m in mats)}
 
     # ---- max over ranks
     ms_per_step = elapsed_ms / args.steps
     if dist is not None:
         t = torch.tensor([ms_per_step, e2e["ms_per_step"] if e2e else 0.0], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, e2e_ms_max = float(t[0]), float(t[1])
+        ms_per_step = float(t[0])
         if e2e:
-            e2e["ms_per_step"] = e2e_ms_max
+            e2e["ms_per_step"] = float(t[1])
 
     peak, peak_src = measured_peaks()
-    total_weight_bytes = weight_bytes * world
-    value = total_weight_bytes / (ms_per_step / 1000.0) / 1e9
-    achieved = algo_bytes / (kernel_ms_per_step / 1000.0) / 1e9
-    traffic_path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    value = weight_bytes * world / (ms_per_step / 1000.0) / 1e9
+    achieved = algo_bytes / (ms_per_step / 1000.0) / 1e9
     traffic = None
+    traffic_path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if os.path.exists(traffic_path):
         with open(traffic_path) as fh:
             tr = json.load(fh)
@@ -340,7 +371,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(fmt, mats, x_by_k, batch)
+        cpu = cpu_baseline(fmt, mats, batch)
 
     if rank == 0:
         line = {
@@ -350,28 +381,31 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": workload_name(fmt, batch, args.layers), "fmt": fmt, "batch": batch,
-                       "weight_bytes_per_step": weight_bytes, "launches_per_step": len(mats),
-                       "l2": "inputs larger than L2 (weights per step > 126 MB), no flush",
+                       "weight_bytes_per_step": weight_bytes, "gemv_calls_per_step": len(mats),
+                       "l2": "inputs larger than L2 (1.06 GB of weights per step at q1g128), no flush",
                        "parallelism": f"replicas x{world}"},
             "hbm_roofline_pct": round(100.0 * value / world / peak, 2),
             "tokens_per_s_equiv": round(1000.0 / ms_per_step, 2),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "bq GEMV, all launches of a step",
-                         "algorithmic_bytes_per_step": algo_bytes,
-                         "kernel_ms_per_step": round(kernel_ms_per_step, 4)},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
+                         "kernel": "bq GEMV (prep + decode kernels), every launch of a step back to back",
+                         "algorithmic_bytes_per_step": algo_bytes},
+            "lm_head_launch": {"us": round(head_ms * 1000, 2), "bytes": head_bytes,
+                               "GB_s": round(head_bytes / (head_ms / 1000.0) / 1e9, 2),
+                               "frac": round(head_bytes / (head_ms / 1000.0) / 1e9 / peak, 4)},
             "clocks": clocks,
-            "gpu_launches": len(mats) * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
         }
         if e2e:
-            line["e2e"] = {"value": round(total_weight_bytes / (e2e["ms_per_step"] / 1000.0) / 1e9, 2),
+            line["e2e"] = {"value": round(weight_bytes * world / (e2e["ms_per_step"] / 1000.0) / 1e9, 2),
                            "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
                            "d2h_bytes_per_step": e2e["d2h"]}
         if cpu:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
 
+    del graph, hg
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

@@ -31,9 +31,13 @@
 // Data movement: per pipeline stage (1024 weights of K for 128 rows) a
 // producer warp issues a TMA tile load of the codes (128-byte swizzle), one of
 // the FP16 scales and a bulk copy of the prepared activation operands into
-// shared memory; four compute warps read conflict-free from there.  K is split
-// across CTAs when the matrix has too few rows to fill the GPU; the last CTA of
-// a row block adds the partial sums in a fixed order (deterministic).
+// shared memory; four compute warps read conflict-free from there.  The grid
+// is persistent (a fixed number of CTAs per SM) and splits the sequence of
+// (row block, stage) items evenly ("stream-K"), so there is no tail wave; a row
+// block shared by two CTAs is finished by the last of them, which adds the
+// partial sums in CTA order (deterministic).  Launches use programmatic
+// dependent launch: a call's weight stream starts while the previous kernel in
+// the stream is still draining.
 #include <cuda.h>
 
 #include "bq_internal.cuh"
@@ -77,14 +81,14 @@ struct Layout {
 
 struct Params {
     const uint8_t* xdata;     // prepared activation operands, [stage][NT][kXTileBytes]
-    float* partial;           // [splits][batch][n] when splits > 1
+    float* partial;           // [grid][2][batch][kRowsPerCta] partial sums of split row blocks
     unsigned int* counters;   // [row_blocks], zeroed by the prep kernel
     void* y;
     int y_dtype;
     int batch;
     int64_t n;
     int stages_total;
-    int splits;
+    int row_blocks;
     int* status;
 };
 
@@ -103,6 +107,10 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
     __shared__ int8_t dig[2 * NT][kGroupsPerStage * 128][4];
     const int st = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Let the GEMV kernel launch and prefetch weights now; x and the workspace
+    // are touched only after the previous kernel in the stream has finished.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     if (st == 0)
         for (int i = threadIdx.x; i < row_blocks; i += blockDim.x) counters[i] = 0u;
     uint8_t* out = xdata + (size_t)st * NT * kXTileBytes;
@@ -182,6 +190,14 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
 }
 
 // ----------------------------------------------------------------- main
+// Persistent stream-K kernel.  The work is the sequence of items
+// (row block, stage) in row-block-major order; CTA c takes items
+// [c*T/C, (c+1)*T/C).  A row block whose stages all fall inside one CTA is
+// written directly; a row block split between CTAs is combined by the CTA that
+// finishes it last, adding the partial sums in CTA order (deterministic).
+__host__ __device__ __forceinline__ int64_t item_begin(int64_t c, int64_t T, int64_t C) { return c * T / C; }
+__device__ __forceinline__ int64_t cta_of_item(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
+
 template <int FMT, int NT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_scales,
@@ -194,10 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
     __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rb = blockIdx.x, sp = blockIdx.y;
-    const int st0 = (int)((int64_t)sp * p.stages_total / p.splits);
-    const int st1 = (int)((int64_t)(sp + 1) * p.stages_total / p.splits);
-    const int nst = st1 - st0;
+    const int64_t S = p.stages_total, T = (int64_t)p.row_blocks * S, C = gridDim.x, c = blockIdx.x;
+    const int64_t it0 = item_begin(c, T, C), it1 = item_begin(c + 1, T, C);
+    const int nit = (int)(it1 - it0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::kStages; ++i) {
@@ -207,22 +222,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
         ptx::fence_barrier_init();
     }
     __syncthreads();
+    // The next grid in the stream may start its prologue (and its own weight
+    // prefetch) as soon as SMs free up; it waits for this grid before it reads
+    // anything this grid writes.
+    ptx::pdl_launch_dependents();
 
     if (warp == kComputeWarps) {
         // ------------------------------------------------ producer
         if (lane == 0) {
             ptx::prefetch_tensormap(&tm_codes);
             ptx::prefetch_tensormap(&tm_scales);
-            int issued = 0;
-            for (int it = 0; it < nst; ++it) {
+            auto issue_weights = [&](int it) {
                 const int slot = it % L::kStages;
-                if (it >= L::kStages &&
-                    !ptx::mbar_wait_bounded(&empty[slot], ((it / L::kStages) - 1) & 1, kWaitPolls)) {
-                    record_status(p.status, BQ_ERR_TIMEOUT);
-                    break;
-                }
                 uint8_t* sb = smem + slot * L::kStageBytes;
-                const int st = st0 + it;
+                const int64_t item = it0 + it;
+                const int rb = (int)(item / S), st = (int)(item % S);
                 ptx::mbar_arrive_expect_tx(&full[slot], L::kCodesBytes + L::kScalesBytes + L::kXBytes);
 #pragma unroll
                 for (int box = 0; box < Fmt<FMT>::kRowBytesPerStage / 128; ++box)
@@ -230,11 +244,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
                                      st * Fmt<FMT>::kRowBytesPerStage + box * 128, rb * kRowsPerCta, &full[slot]);
                 ptx::tma_load_2d(sb + L::kCodesBytes, &tm_scales, st * kGroupsPerStage, rb * kRowsPerCta,
                                  &full[slot]);
+            };
+            auto issue_x = [&](int it) {
+                const int slot = it % L::kStages;
+                uint8_t* sb = smem + slot * L::kStageBytes;
+                const int st = (int)((it0 + it) % S);
                 ptx::bulk_load(sb + L::kCodesBytes + L::kScalesBytes, p.xdata + (size_t)st * L::kXBytes,
                                L::kXBytes, &full[slot]);
+            };
+            // The weights do not depend on the previous kernel: start streaming
+            // them before waiting for it; the activation operands come after.
+            const int pre = nit < L::kStages ? nit : L::kStages;
+            for (int it = 0; it < pre; ++it) issue_weights(it);
+            ptx::pdl_wait();
+            for (int it = 0; it < pre; ++it) issue_x(it);
+            int issued = pre;
+            for (int it = pre; it < nit; ++it) {
+                const int slot = it % L::kStages;
+                if (!ptx::mbar_wait_bounded(&empty[slot], ((it / L::kStages) - 1) & 1, kWaitPolls)) {
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+                    break;
+                }
+                issue_weights(it);
+                issue_x(it);
                 issued = it + 1;
             }
-            // make sure every copy this CTA issued has landed before it may exit
+            // every copy this CTA issued must land before it may exit
             for (int it = (issued > L::kStages ? issued - L::kStages : 0); it < issued; ++it)
                 if (!ptx::mbar_wait_bounded(&full[it % L::kStages], (it / L::kStages) & 1, kWaitPolls))
                     record_status(p.status, BQ_ERR_TIMEOUT);
@@ -244,148 +279,168 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
 
     // ---------------------------------------------------- compute warps
     const int g = lane >> 2, t = lane & 3;
+    const bool writer = (t & 1) == 0;
     float yacc[kRowTiles][NT][2];
 #pragma unroll
     for (int j = 0; j < kRowTiles; ++j)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
 
-    for (int it = 0; it < nst; ++it) {
+    bool alive = true;
+    for (int it = 0; it < nit; ++it) {
         const int slot = it % L::kStages;
-        if (!ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
+        const int64_t item = it0 + it;
+        const int rb = (int)(item / S), st = (int)(item % S);
+        if (alive && !ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
             record_status(p.status, BQ_ERR_TIMEOUT);
-            break;
+            alive = false;
         }
-        const uint32_t sb = ptx::smem_u32(smem + slot * L::kStageBytes);
-        const uint32_t codes_s = sb, scales_s = sb + L::kCodesBytes, x_s = sb + L::kCodesBytes + L::kScalesBytes;
-#pragma unroll 1
-        for (int G = 0; G < kGroupsPerStage; ++G) {
-            uint2 bf[NT][4];
-            float4 tab[NT];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    bf[nt][q] = ptx::lds64(x_s + nt * kXTileBytes + ((G * 4 + q) * 32 + lane) * 8);
-                tab[nt] = ptx::lds128f(x_s + nt * kXTileBytes + kGroupsPerStage * kBfragBytesPerGroup +
-                                       (G * 4 + t) * 16);
-            }
-#pragma unroll
-            for (int j = 0; j < kRowTiles; ++j) {
-                const int r0 = warp * (16 * kRowTiles) + j * 16 + g;
-                const float s0 = half_bits_to_float(ptx::lds16(scales_s + r0 * 16 + 2 * G));
-                const float s1 = half_bits_to_float(ptx::lds16(scales_s + (r0 + 8) * 16 + 2 * G));
-                int acc[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
-                if (FMT == BQ_Q1G128) {
-                    const uint32_t off = ((uint32_t)(G ^ g) << 4) + 4 * t;
-                    const uint32_t w0 = ptx::lds32(codes_s + r0 * 128 + off);
-                    const uint32_t w1 = ptx::lds32(codes_s + (r0 + 8) * 128 + off);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
-                        const uint32_t a0 = w0 & m0, a1 = w1 & m0, a2 = w0 & m1, a3 = w1 & m1;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
-                    }
-                } else {
-                    const uint32_t box = codes_s + (G >> 2) * (kRowsPerCta * 128);
-                    const uint32_t c0 = 2 * (G & 3), c1 = c0 + 1;
-                    const uint32_t offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
-                    const uint32_t w0a = ptx::lds32(box + r0 * 128 + offa);
-                    const uint32_t w0b = ptx::lds32(box + r0 * 128 + offb);
-                    const uint32_t w1a = ptx::lds32(box + (r0 + 8) * 128 + offa);
-                    const uint32_t w1b = ptx::lds32(box + (r0 + 8) * 128 + offb);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
-                        const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
-                        const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
-                        const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
-                    }
-                }
+        if (alive) {
+            const uint8_t* stage = smem + slot * L::kStageBytes;
+            const uint8_t* codes_s = stage;
+            const uint16_t* scales_s = reinterpret_cast<const uint16_t*>(stage + L::kCodesBytes);
+            const uint8_t* x_s = stage + L::kCodesBytes + L::kScalesBytes;
+#pragma unroll 2
+            for (int G = 0; G < kGroupsPerStage; ++G) {
+                uint2 bf[NT][4];
+                float4 tab[NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const float v0 = fmaf(256.0f, (float)acc[nt][1], (float)acc[nt][0]);
-                    const float v1 = fmaf(256.0f, (float)acc[nt][3], (float)acc[nt][2]);
-                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                    yacc[j][nt][0] = fmaf(s0, u0, yacc[j][nt][0]);
-                    yacc[j][nt][1] = fmaf(s1, u1, yacc[j][nt][1]);
+                    const uint8_t* xt = x_s + nt * kXTileBytes;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        bf[nt][q] = *reinterpret_cast<const uint2*>(xt + ((G * 4 + q) * 32 + lane) * 8);
+                    tab[nt] = *reinterpret_cast<const float4*>(xt + kGroupsPerStage * kBfragBytesPerGroup + (G * 4 + t) * 16);
                 }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[slot]);
-    }
-
-    // ---------------------------------------------------- epilogue
-    // lanes t and t^1 hold the low and high digit pairs of the same (row, batch row)
 #pragma unroll
-    for (int j = 0; j < kRowTiles; ++j)
+                for (int j = 0; j < kRowTiles; ++j) {
+                    const int r0 = warp * (16 * kRowTiles) + j * 16 + g;
+                    int acc[NT][2][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int r = 0; r < 2; ++r) yacc[j][nt][r] += __shfl_xor_sync(0xffffffffu, yacc[j][nt][r], 1);
-
-    const bool writer = (t & 1) == 0;
-    if (p.splits == 1) {
-        if (writer) {
+                        for (int h = 0; h < 2; ++h) acc[nt][h][0] = acc[nt][h][1] = acc[nt][h][2] = acc[nt][h][3] = 0;
+                    if (FMT == BQ_Q1G128) {
+                        const int off = ((G ^ g) << 4) + 4 * t;
+                        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_s + r0 * 128 + off);
+                        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_s + (r0 + 8) * 128 + off);
 #pragma unroll
-            for (int j = 0; j < kRowTiles; ++j)
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                            for (int nt = 0; nt < NT; ++nt)
+                                ptx::mma_u8s8(acc[nt][q >> 1], w0 & m0, w1 & m0, w0 & m1, w1 & m1, bf[nt][q].x, bf[nt][q].y);
+                        }
+                    } else {
+                        const uint8_t* box = codes_s + (G >> 2) * (kRowsPerCta * 128);
+                        const int c0 = 2 * (G & 3), c1 = c0 + 1;
+                        const int offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
+                        const uint32_t w0a = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offa);
+                        const uint32_t w0b = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offb);
+                        const uint32_t w1a = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offa);
+                        const uint32_t w1b = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offb);
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int bb = nt * 2 + (t >> 1);
-                        const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
-                        if (bb < p.batch && row < p.n) {
-                            if (p.y_dtype == BQ_F32)
-                                static_cast<float*>(p.y)[bb * p.n + row] = yacc[j][nt][r];
-                            else
-                                static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[j][nt][r]);
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
+                            const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
+                            const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
+                            const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                ptx::mma_u8s8(acc[nt][q >> 1], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
                         }
                     }
+                    const float s0 = half_bits_to_float(scales_s[r0 * kGroupsPerStage + G]);
+                    const float s1 = half_bits_to_float(scales_s[(r0 + 8) * kGroupsPerStage + G]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const float v0 = fmaf(256.0f, (float)(acc[nt][0][1] + acc[nt][1][1]), (float)(acc[nt][0][0] + acc[nt][1][0]));
+                        const float v1 = fmaf(256.0f, (float)(acc[nt][0][3] + acc[nt][1][3]), (float)(acc[nt][0][2] + acc[nt][1][2]));
+                        const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                        const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                        yacc[j][nt][0] = fmaf(s0, u0, yacc[j][nt][0]);
+                        yacc[j][nt][1] = fmaf(s1, u1, yacc[j][nt][1]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&empty[slot]);
         }
-        return;
-    }
-    // split K: publish this CTA's partial sums; the last CTA of the row block adds them in order
-    if (writer) {
+        // ---------------------------------------- row block finished here?
+        if (st != S - 1 && it != nit - 1) continue;
 #pragma unroll
         for (int j = 0; j < kRowTiles; ++j)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int bb = nt * 2 + (t >> 1);
-                    const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
-                    if (bb < p.batch && row < p.n) p.partial[((int64_t)sp * p.batch + bb) * p.n + row] = yacc[j][nt][r];
+                for (int r = 0; r < 2; ++r) yacc[j][nt][r] += __shfl_xor_sync(0xffffffffu, yacc[j][nt][r], 1);
+        const int64_t rb_first = (int64_t)rb * S, rb_last = rb_first + S - 1;
+        const bool whole = rb_first >= it0 && rb_last < it1;
+        if (whole) {
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int bb = nt * 2 + (t >> 1);
+                            const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
+                            if (bb < p.batch && row < p.n) {
+                                if (p.y_dtype == BQ_F32)
+                                    static_cast<float*>(p.y)[bb * p.n + row] = yacc[j][nt][r];
+                                else
+                                    static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[j][nt][r]);
+                            }
+                        }
+            }
+        } else {
+            const int slot_p = (item_begin(c, T, C) / S == rb) ? 0 : 1;
+            float* mine = p.partial + ((c * 2 + slot_p) * p.batch) * kRowsPerCta;
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int bb = nt * 2 + (t >> 1);
+                            if (bb < p.batch)
+                                mine[bb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r] = yacc[j][nt][r];
+                        }
+            }
+            __threadfence();
+            named_barrier_compute();
+            const int64_t c_first = cta_of_item(rb_first, T, C), c_last = cta_of_item(rb_last, T, C);
+            if (threadIdx.x == 0) {
+                const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
+                s_last = (prev == (unsigned int)(c_last - c_first));
+            }
+            named_barrier_compute();
+            if (s_last) {
+                __threadfence();
+                for (int i = threadIdx.x; i < kRowsPerCta * p.batch; i += kComputeWarps * 32) {
+                    const int bb = i / kRowsPerCta, rin = i % kRowsPerCta;
+                    const int64_t row = (int64_t)rb * kRowsPerCta + rin;
+                    if (row >= p.n) continue;
+                    float acc = 0.0f;
+                    for (int64_t cc = c_first; cc <= c_last; ++cc) {
+                        const int sl = (item_begin(cc, T, C) / S == rb) ? 0 : 1;
+                        acc += __ldcg(p.partial + ((cc * 2 + sl) * p.batch + bb) * kRowsPerCta + rin);
+                    }
+                    if (p.y_dtype == BQ_F32)
+                        static_cast<float*>(p.y)[bb * p.n + row] = acc;
+                    else
+                        static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(acc);
                 }
+                if (threadIdx.x == 0) p.counters[rb] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
     }
-    __threadfence();
-    named_barrier_compute();
-    if (threadIdx.x == 0) {
-        const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
-        s_last = (prev == (unsigned int)(p.splits - 1));
-    }
-    named_barrier_compute();
-    if (!s_last) return;
-    __threadfence();
-    for (int i = threadIdx.x; i < kRowsPerCta * p.batch; i += kComputeWarps * 32) {
-        const int bb = i / kRowsPerCta;
-        const int64_t row = (int64_t)rb * kRowsPerCta + (i % kRowsPerCta);
-        if (row >= p.n) continue;
-        float acc = 0.0f;
-        for (int s = 0; s < p.splits; ++s) acc += __ldcg(&p.partial[((int64_t)s * p.batch + bb) * p.n + row]);
-        if (p.y_dtype == BQ_F32)
-            static_cast<float*>(p.y)[bb * p.n + row] = acc;
-        else
-            static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(acc);
-    }
-    if (threadIdx.x == 0) p.counters[rb] = 0u;
 }
 
 // ----------------------------------------------------------------- host
@@ -406,7 +461,7 @@ EncodeTiledFn encode_fn() {
 }
 
 struct Plan {
-    int nt = 0, stages_total = 0, row_blocks = 0, splits = 0;
+    int nt = 0, stages_total = 0, row_blocks = 0, grid = 0;
     size_t xdata_bytes = 0, counters_off = 0, partial_off = 0, total = 0;
 };
 
@@ -415,21 +470,30 @@ bool eligible(int fmt, int64_t n, int64_t k, int batch) {
            n > 0 && n <= (int64_t)INT32_MAX && k / 8 <= (int64_t)INT32_MAX / 4;
 }
 
+int sm_count() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
 Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     Plan pl;
     pl.nt = (batch + 1) / 2;
     pl.stages_total = (int)(k / 1024);
     pl.row_blocks = (int)((n + kRowsPerCta - 1) / kRowsPerCta);
     const int ctas_per_sm = (fmt == BQ_Q1G128) ? 2 : 1;
-    const int target = 148 * ctas_per_sm;
-    int splits = (target + pl.row_blocks - 1) / pl.row_blocks;
-    splits = splits < 1 ? 1 : splits;
-    splits = splits > pl.stages_total ? pl.stages_total : splits;
-    pl.splits = splits;
+    const int64_t items = (int64_t)pl.row_blocks * pl.stages_total;
+    const int64_t cap = (int64_t)sm_count() * ctas_per_sm;
+    pl.grid = (int)(items < cap ? items : cap);
     pl.xdata_bytes = (size_t)pl.stages_total * pl.nt * kXTileBytes;
     pl.counters_off = (pl.xdata_bytes + 255) / 256 * 256;
     pl.partial_off = (pl.counters_off + (size_t)pl.row_blocks * 4 + 255) / 256 * 256;
-    pl.total = pl.partial_off + (splits > 1 ? (size_t)splits * batch * n * 4 : 0);
+    pl.total = pl.partial_off + (size_t)pl.grid * 2 * batch * kRowsPerCta * 4;
     return pl;
 }
 
@@ -478,13 +542,29 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     prm.batch = batch;
     prm.n = n;
     prm.stages_total = pl.stages_total;
-    prm.splits = pl.splits;
+    prm.row_blocks = pl.row_blocks;
     prm.status = device_status_ptr();
     if (!prm.status) return cudaErrorUnknown;
-    prep_kernel<FMT, NT><<<pl.stages_total, 256, 0, s>>>(x, k, batch, ws, prm.counters, pl.row_blocks);
-    cudaError_t e = cudaGetLastError();
+    // Both kernels are launched as programmatic dependents of whatever precedes
+    // them in the stream; each waits (griddepcontrol.wait) before touching data
+    // the predecessor may still produce or read.
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.stages_total);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prep_kernel<FMT, NT>, x, k, batch, ws, prm.counters, pl.row_blocks);
     if (e != cudaSuccess) return e;
-    gemv_tc_kernel<FMT, NT><<<dim3(pl.row_blocks, pl.splits), kThreads, L::kSmemBytes, s>>>(tm_codes, tm_scales, prm);
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::kSmemBytes;
+    e = cudaLaunchKernelEx(&cfg, gemv_tc_kernel<FMT, NT>, tm_codes, tm_scales, prm);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
