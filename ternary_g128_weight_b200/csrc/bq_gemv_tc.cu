@@ -48,8 +48,8 @@ namespace tc {
 
 constexpr int kGroupsPerStage = 8;
 constexpr int kRowsPerCta = 128;
-constexpr int kComputeWarps = 4;
-constexpr int kRowTiles = 2;  // 16-row MMA tiles per compute warp
+constexpr int kComputeWarps = 8;
+constexpr int kRowTiles = 1;  // 16-row MMA tiles per compute warp
 constexpr int kThreads = (kComputeWarps + 1) * 32;
 constexpr int kBfragBytesPerGroup = 4 * 32 * 8;  // 4 MMAs x 32 lanes x (b0, b1)
 constexpr int kTableBytesPerGroup = 4 * 16;      // 4 lanes-in-quad x float4
@@ -75,7 +75,9 @@ struct Layout {
     static constexpr int kScalesBytes = kRowsPerCta * kGroupsPerStage * 2;
     static constexpr int kXBytes = NT * kXTileBytes;
     static constexpr int kStageBytes = (kCodesBytes + kScalesBytes + kXBytes + 1023) / 1024 * 1024;
-    static constexpr int kStages = (FMT == BQ_Q1G128 && NT == 1) ? 4 : 3;
+    // two CTAs per SM: 4 (binary, batch <= 2), 3 (binary, batch <= 4) or 2 (2-bit) stages
+    static constexpr int kStages = (FMT == BQ_Q1G128) ? (NT == 1 ? 4 : 3) : 2;
+    static_assert(kComputeWarps * 16 * kRowTiles == kRowsPerCta, "row tiling");
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 2 * kStages * 8;
 };
 
@@ -185,7 +187,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
             b0 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k0][dg] << (8 * j);
             b1 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k1][dg] << (8 * j);
         }
-        *reinterpret_cast<uint2*>(out + nt * kXTileBytes + ((g8 * 4 + q) * 32 + ln) * 8) = make_uint2(b0, b1);
+        // lane-contiguous 16 bytes hold (b0, b1) of MMAs 2j and 2j+1 of the group
+        *reinterpret_cast<uint2*>(out + nt * kXTileBytes + ((g8 * 2 + (q >> 1)) * 32 + ln) * 16 + (q & 1) * 8) =
+            make_uint2(b0, b1);
     }
 }
 
@@ -199,7 +203,7 @@ __host__ __device__ __forceinline__ int64_t item_begin(int64_t c, int64_t T, int
 __device__ __forceinline__ int64_t cta_of_item(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
 
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
+__global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_scales,
                                                               const Params p) {
     using L = Layout<FMT, NT>;
@@ -300,67 +304,74 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
             const uint8_t* codes_s = stage;
             const uint16_t* scales_s = reinterpret_cast<const uint16_t*>(stage + L::kCodesBytes);
             const uint8_t* x_s = stage + L::kCodesBytes + L::kScalesBytes;
-#pragma unroll 2
+            const int r0 = warp * 16 + g;  // this thread's rows: r0 and r0 + 8
+            // the 8 group scales of both rows (FP16 pairs)
+            const uint4 sv0 = *reinterpret_cast<const uint4*>(scales_s + r0 * kGroupsPerStage);
+            const uint4 sv1 = *reinterpret_cast<const uint4*>(scales_s + (r0 + 8) * kGroupsPerStage);
+            const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w};
+            const uint32_t s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
+#pragma unroll
             for (int G = 0; G < kGroupsPerStage; ++G) {
-                uint2 bf[NT][4];
+                uint4 bf[NT][2];
                 float4 tab[NT];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const uint8_t* xt = x_s + nt * kXTileBytes;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        bf[nt][q] = *reinterpret_cast<const uint2*>(xt + ((G * 4 + q) * 32 + lane) * 8);
+                    for (int h = 0; h < 2; ++h)
+                        bf[nt][h] = *reinterpret_cast<const uint4*>(xt + ((G * 2 + h) * 32 + lane) * 16);
                     tab[nt] = *reinterpret_cast<const float4*>(xt + kGroupsPerStage * kBfragBytesPerGroup + (G * 4 + t) * 16);
                 }
+                int acc[NT][4];
 #pragma unroll
-                for (int j = 0; j < kRowTiles; ++j) {
-                    const int r0 = warp * (16 * kRowTiles) + j * 16 + g;
-                    int acc[NT][2][4];
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+                if (FMT == BQ_Q1G128) {
+                    const int off = ((G ^ g) << 4) + 4 * t;
+                    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_s + r0 * 128 + off);
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_s + (r0 + 8) * 128 + off);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) acc[nt][h][0] = acc[nt][h][1] = acc[nt][h][2] = acc[nt][h][3] = 0;
-                    if (FMT == BQ_Q1G128) {
-                        const int off = ((G ^ g) << 4) + 4 * t;
-                        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_s + r0 * 128 + off);
-                        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_s + (r0 + 8) * 128 + off);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                ptx::mma_u8s8(acc[nt][q >> 1], w0 & m0, w1 & m0, w0 & m1, w1 & m1, bf[nt][q].x, bf[nt][q].y);
-                        }
-                    } else {
-                        const uint8_t* box = codes_s + (G >> 2) * (kRowsPerCta * 128);
-                        const int c0 = 2 * (G & 3), c1 = c0 + 1;
-                        const int offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
-                        const uint32_t w0a = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offa);
-                        const uint32_t w0b = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offb);
-                        const uint32_t w1a = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offa);
-                        const uint32_t w1b = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offb);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
-                            const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
-                            const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
-                            const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                ptx::mma_u8s8(acc[nt][q >> 1], a0, a1, a2, a3, bf[nt][q].x, bf[nt][q].y);
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            ptx::mma_u8s8(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1);
                         }
                     }
-                    const float s0 = half_bits_to_float(scales_s[r0 * kGroupsPerStage + G]);
-                    const float s1 = half_bits_to_float(scales_s[(r0 + 8) * kGroupsPerStage + G]);
+                } else {
+                    const uint8_t* box = codes_s + (G >> 2) * (kRowsPerCta * 128);
+                    const int c0 = 2 * (G & 3), c1 = c0 + 1;
+                    const int offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
+                    const uint32_t w0a = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offa);
+                    const uint32_t w0b = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offb);
+                    const uint32_t w1a = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offa);
+                    const uint32_t w1b = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offb);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const float v0 = fmaf(256.0f, (float)(acc[nt][0][1] + acc[nt][1][1]), (float)(acc[nt][0][0] + acc[nt][1][0]));
-                        const float v1 = fmaf(256.0f, (float)(acc[nt][0][3] + acc[nt][1][3]), (float)(acc[nt][0][2] + acc[nt][1][2]));
-                        const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                        const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                        yacc[j][nt][0] = fmaf(s0, u0, yacc[j][nt][0]);
-                        yacc[j][nt][1] = fmaf(s1, u1, yacc[j][nt][1]);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
+                        const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, b0, b1);
+                        }
                     }
+                }
+                const float s0 = half_bits_to_float((uint16_t)(s0w[G >> 1] >> (16 * (G & 1))));
+                const float s1 = half_bits_to_float((uint16_t)(s1w[G >> 1] >> (16 * (G & 1))));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    // D0 + 256 D1 is exact in int32 (|D| < 2^21)
+                    const float v0 = (float)(acc[nt][0] + 256 * acc[nt][1]);
+                    const float v1 = (float)(acc[nt][2] + 256 * acc[nt][3]);
+                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    yacc[0][nt][0] = fmaf(s0, u0, yacc[0][nt][0]);
+                    yacc[0][nt][1] = fmaf(s1, u1, yacc[0][nt][1]);
                 }
             }
             __syncwarp();
@@ -486,7 +497,7 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.nt = (batch + 1) / 2;
     pl.stages_total = (int)(k / 1024);
     pl.row_blocks = (int)((n + kRowsPerCta - 1) / kRowsPerCta);
-    const int ctas_per_sm = (fmt == BQ_Q1G128) ? 2 : 1;
+    const int ctas_per_sm = 2;
     const int64_t items = (int64_t)pl.row_blocks * pl.stages_total;
     const int64_t cap = (int64_t)sm_count() * ctas_per_sm;
     pl.grid = (int)(items < cap ? items : cap);
