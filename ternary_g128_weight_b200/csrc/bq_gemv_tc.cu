@@ -27,15 +27,19 @@
 // q = c - 1.  The only rounding before FP32 is that of x to Q: at most 2^-23
 // of the group's largest |x| per element.
 //
-// CTA roles (2 CTAs per SM, 128 rows each):
-//   warps 0-3 : one row per thread (= TMEM lane): read the row's codes from
-//               shared memory, expand them into 32 TMEM columns per group
-//               (tcgen05.st), and, four groups later, read the group's int32
-//               sums back (tcgen05.ld) and fold them into y with the scale;
-//   warp 4    : TMA producer (codes with 128-byte swizzle, FP16 scales, and a
+// CTA roles (one CTA per SM, 128 rows, all 512 TMEM columns):
+//   warps 0-15: decode warps, four per TMEM lane quadrant; warp d handles the
+//               rows of quadrant d & 3 (one row per thread = TMEM lane) and
+//               groups d >> 2 and (d >> 2) + 4 of every stage: it expands the
+//               row's codes into the group's 32 TMEM columns (tcgen05.st) and,
+//               one stage later, reads the group's int32 sums back
+//               (tcgen05.ld) and folds them into y with the scale;
+//   warp 16   : TMA producer (codes with 128-byte swizzle, FP16 scales, and a
 //               bulk copy of the prepared activation operand per stage);
-//   warp 5    : allocates TMEM and issues the MMAs (M = 128, N = 8 or 16,
+//   warp 17   : allocates TMEM and issues the MMAs (M = 128, N = 8 or 16,
 //               K = 32 per instruction, A from TMEM, B from shared memory).
+// Each group has its own A (32 columns) and D (16 columns) slot, so the
+// decode of a stage never waits for the MMAs of the same stage.
 // The grid is persistent and splits the (row block, stage) items evenly
 // ("stream-K"); a row block shared by two CTAs is finished by the last one,
 // which adds the partial sums in CTA order (deterministic).  Launches use
@@ -51,13 +55,13 @@ namespace tc {
 
 constexpr int kGroupsPerStage = 8;
 constexpr int kRowsPerCta = 128;
-constexpr int kDecodeWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-constexpr int kRing = 4;         // groups in flight between decode and epilogue
-constexpr int kTmemCols = 256;   // A ring 4 x 32 columns + D ring 4 x 16 columns
-constexpr int kDCol0 = kRing * 32;
+constexpr int kSubs = 4;                         // decode warps per TMEM lane quadrant
+constexpr int kDecodeWarps = 4 * kSubs;          // warp d: quadrant d & 3, sub d >> 2
+constexpr int kProducerWarp = kDecodeWarps;
+constexpr int kMmaWarp = kDecodeWarps + 1;
+constexpr int kThreads = (kDecodeWarps + 2) * 32;
+constexpr int kTmemCols = 512;                   // A: 8 groups x 32 columns, D: 8 groups x 16 columns
+constexpr int kDCol0 = kGroupsPerStage * 32;
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <int FMT>
@@ -90,10 +94,11 @@ struct Layout {
     static constexpr int kScalesBytes = kRowsPerCta * kGroupsPerStage * 2;
     static constexpr int kXBytes = XTile<NT>::kBytes;
     static constexpr int kStageBytes = (kCodesBytes + kScalesBytes + kXBytes + 1023) / 1024 * 1024;
-    // two CTAs per SM
-    static constexpr int kStages = (FMT == BQ_Q1G128) ? (NT == 1 ? 4 : 3) : 2;
-    static constexpr int kBarriers = 2 * kStages + 2 * kRing + 1;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarriers * 8 + 16;
+    // one CTA per SM
+    static constexpr int kStages = (FMT == BQ_Q1G128) ? (NT == 1 ? 6 : 5) : (NT == 1 ? 4 : 3);
+    static constexpr int kBarriers = 2 * kStages + 2 * kGroupsPerStage + 1;
+    static constexpr int kCombineBytes = (kSubs - 1) * kRowsPerCta * 2 * NT * 4;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarriers * 8 + 16 + kCombineBytes;
 };
 
 struct Params {
@@ -109,9 +114,11 @@ struct Params {
     int* status;
 };
 
+// all decode warps / the sub-0 decode warps (the ones that write outputs)
 __device__ __forceinline__ void decode_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(kDecodeWarps * 32) : "memory");
 }
+__device__ __forceinline__ void writer_barrier() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 __host__ __device__ __forceinline__ int64_t item_begin(int64_t c, int64_t T, int64_t C) { return c * T / C; }
 __device__ __forceinline__ int64_t cta_of_item(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(128) prep_kernel(const uint16_t* __restrict__ 
 
 // ----------------------------------------------------------------- main
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
+__global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_scales,
                                                               const Params p) {
     using L = Layout<FMT, NT>;
@@ -210,9 +217,10 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
     uint64_t* empty = full + L::kStages;
     uint64_t* a_full = empty + L::kStages;
-    uint64_t* mma_done = a_full + kRing;
-    uint64_t* final_bar = mma_done + kRing;
+    uint64_t* mma_done = a_full + kGroupsPerStage;
+    uint64_t* final_bar = mma_done + kGroupsPerStage;
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(final_bar + 1);
+    float* combine = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tmem_base_smem) + 16);
     __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -225,8 +233,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             ptx::mbar_init(&full[i], 1);
             ptx::mbar_init(&empty[i], kDecodeWarps + 1);
         }
-        for (int i = 0; i < kRing; ++i) {
-            ptx::mbar_init(&a_full[i], kDecodeWarps);
+        for (int i = 0; i < kGroupsPerStage; ++i) {
+            ptx::mbar_init(&a_full[i], 4);  // the four quadrant warps of the group's sub
             ptx::mbar_init(&mma_done[i], 1);
         }
         ptx::mbar_init(final_bar, 1);
@@ -300,8 +308,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                 const uint32_t b_s = ptx::smem_u32(smem + slot * L::kStageBytes + L::kCodesBytes + L::kScalesBytes);
 #pragma unroll
                 for (int G = 0; G < kGroupsPerStage; ++G) {
-                    const int r = G & (kRing - 1);
-                    if (!ptx::mbar_wait_bounded(&a_full[r], G >> 2, kWaitPolls)) {
+                    if (!ptx::mbar_wait_bounded(&a_full[G], it & 1, kWaitPolls)) {
                         record_status(p.status, BQ_ERR_TIMEOUT);
                         ok = false;
                         break;
@@ -310,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const uint64_t bd = ptx::smem_desc_kmajor_noswizzle(b_s + (G * 4 + q) * 256 * NT, 128 * NT, 128);
-                        ptx::mma_i8_ts(tmem + kDCol0 + r * 8 * NT, tmem + r * 32 + q * 8, bd, idesc, q > 0 ? 1u : 0u);
+                        ptx::mma_i8_ts(tmem + kDCol0 + G * 16, tmem + G * 32 + q * 8, bd, idesc, q > 0 ? 1u : 0u);
                     }
-                    ptx::tc_commit(&mma_done[r]);
+                    ptx::tc_commit(&mma_done[G]);
                 }
                 if (ok) ptx::tc_commit(&empty[slot]);
             }
@@ -322,33 +329,33 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
         }
     } else {
         // ------------------------------------------------ decode + epilogue warps
-        const int row = warp * 32 + lane;  // row in the CTA tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int quad = warp & 3, sub = warp >> 2;
+        const int row = quad * 32 + lane;  // row in the CTA tile == TMEM lane
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         float y[NB];
-        float c1[kRing][NB], f2[kRing][NB], cx[kRing][NB];
+        float c1[2][NB], f2[2][NB], cx[2][NB];  // coefficients of groups sub and sub + 4
 #pragma unroll
         for (int b = 0; b < NB; ++b) y[b] = 0.0f;
         bool alive = true;
-        bool prev_stage_open = false;  // groups 4..7 of the previous stage await their epilogue
+        bool prev_stage_open = false;  // this warp's groups of the previous stage await their fold
 
-        auto epilogue = [&](int r) {
-            uint32_t d[8 * NT];
-            ptx::tc_fence_after();
+        auto epi_load = [&](int G, uint32_t (&d)[8 * NT]) {
 #pragma unroll
             for (int h = 0; h < NT; ++h) {
                 uint32_t t8[8];
-                ptx::tmem_ld_x8(tmem + lane_base + kDCol0 + r * 8 * NT + 8 * h, t8);
+                ptx::tmem_ld_x8(tmem + lane_base + kDCol0 + G * 16 + 8 * h, t8);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) d[8 * h + e] = t8[e];
             }
-            ptx::tc_wait_ld();
+        };
+        auto epi_fold = [&](int j, const uint32_t (&d)[8 * NT]) {
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
                 // columns 4b..4b+3 hold the four digit sums of batch slot b
                 const int lo = (int)d[4 * b] + 256 * (int)d[4 * b + 1];
                 const int hi = (int)d[4 * b + 2] + 256 * (int)d[4 * b + 3];
                 const float v = fmaf((float)hi, 65536.0f, (float)lo);
-                y[b] = fmaf(v * c1[r][b], f2[r][b], y[b]) - cx[r][b];
+                y[b] = fmaf(v * c1[j][b], f2[j][b], y[b]) - cx[j][b];
             }
         };
 
@@ -364,22 +371,23 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                 const uint8_t* stage = smem + slot * L::kStageBytes;
                 const uint16_t* scales_s = reinterpret_cast<const uint16_t*>(stage + L::kCodesBytes);
                 const uint8_t* tab_s = stage + L::kCodesBytes + L::kScalesBytes + XTile<NT>::kBBytes;
-                const uint4 sv = *reinterpret_cast<const uint4*>(scales_s + row * kGroupsPerStage);
-                const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-                for (int G = 0; G < kGroupsPerStage; ++G) {
-                    const int r = G & (kRing - 1);
-                    // the ring slot's previous group: wait for its MMAs; fold it into y
-                    const bool prev_exists = (G >= kRing) || it > 0;
-                    const bool prev_pending = (G >= kRing) || prev_stage_open;
-                    if (prev_exists && alive) {
-                        if (!ptx::mbar_wait_bounded(&mma_done[r], (G >> 2) ^ 1, kWaitPolls)) {
+                for (int j = 0; j < 2; ++j) {
+                    const int G = sub + 4 * j;
+                    // previous stage's group G: wait for its MMAs, start reading its sums
+                    uint32_t d[8 * NT];
+                    const bool fold = it > 0 && prev_stage_open;
+                    if (it > 0) {
+                        if (!ptx::mbar_wait_bounded(&mma_done[G], (it & 1) ^ 1, kWaitPolls)) {
                             record_status(p.status, BQ_ERR_TIMEOUT);
                             alive = false;
                         }
-                        if (prev_pending && alive) epilogue(r);
+                        if (fold && alive) {
+                            ptx::tc_fence_after();
+                            epi_load(G, d);
+                        }
                     }
-                    // decode this group into the slot's 32 TMEM columns
+                    // decode group G into its 32 TMEM columns
                     uint32_t a[32];
                     if (FMT == BQ_Q1G128) {
                         const uint4 w = *reinterpret_cast<const uint4*>(stage + row * 128 + ((G ^ (row & 7)) << 4));
@@ -399,20 +407,24 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 #pragma unroll
                             for (int i = 0; i < 4; ++i) a[4 * w8 + i] = (wv[w8] >> (2 * i)) & 0x03030303u;
                     }
-                    ptx::tmem_st_x32(tmem + lane_base + r * 32, a);
-                    // coefficients for this group's epilogue
-                    const float s = half_bits_to_float((uint16_t)(sw[G >> 1] >> (16 * (G & 1))));
+                    ptx::tmem_st_x32(tmem + lane_base + G * 32, a);
+                    if (fold && alive) {
+                        ptx::tc_wait_ld();
+                        epi_fold(j, d);
+                    }
+                    // coefficients of group G
+                    const float s = half_bits_to_float(scales_s[row * kGroupsPerStage + G]);
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
                         const float4 tab = *reinterpret_cast<const float4*>(tab_s + (G * NB + b) * 16);
-                        c1[r][b] = s * tab.x;
-                        f2[r][b] = tab.y;
-                        cx[r][b] = s * tab.z;
+                        c1[j][b] = s * tab.x;
+                        f2[j][b] = tab.y;
+                        cx[j][b] = s * tab.z;
                     }
                     ptx::tc_wait_st();
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&a_full[r]);
+                    if (lane == 0) ptx::mbar_arrive(&a_full[G]);
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&empty[slot]);
@@ -420,61 +432,79 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             prev_stage_open = true;
             // ---------------------------------------- row block finished here?
             if (st != S - 1 && it != nit - 1) continue;
-            // drain: groups 4..7 of this stage
 #pragma unroll
-            for (int r = 0; r < kRing; ++r) {
-                if (alive && !ptx::mbar_wait_bounded(&mma_done[r], 1, kWaitPolls)) {
+            for (int j = 0; j < 2; ++j) {
+                const int G = sub + 4 * j;
+                if (alive && !ptx::mbar_wait_bounded(&mma_done[G], it & 1, kWaitPolls)) {
                     record_status(p.status, BQ_ERR_TIMEOUT);
                     alive = false;
                 }
-                if (alive) epilogue(r);
+                if (alive) {
+                    uint32_t d[8 * NT];
+                    ptx::tc_fence_after();
+                    epi_load(G, d);
+                    ptx::tc_wait_ld();
+                    epi_fold(j, d);
+                }
             }
             prev_stage_open = false;
-            const int64_t rb_first = (int64_t)rb * S, rb_last = rb_first + S - 1;
-            const bool whole = rb_first >= it0 && rb_last < it1;
-            const int64_t grow = (int64_t)rb * kRowsPerCta + row;
-            if (whole) {
-                if (grow < p.n) {
+            // combine the four subs' partial sums of each row (fixed order)
+            if (sub > 0) {
+#pragma unroll
+                for (int b = 0; b < NB; ++b) combine[((sub - 1) * NB + b) * kRowsPerCta + row] = y[b];
+            }
+            decode_barrier();
+            if (sub == 0) {
+#pragma unroll
+                for (int k2 = 0; k2 < kSubs - 1; ++k2)
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) y[b] += combine[(k2 * NB + b) * kRowsPerCta + row];
+                const int64_t rb_first = (int64_t)rb * S, rb_last = rb_first + S - 1;
+                const bool whole = rb_first >= it0 && rb_last < it1;
+                const int64_t grow = (int64_t)rb * kRowsPerCta + row;
+                if (whole) {
+                    if (grow < p.n) {
+#pragma unroll
+                        for (int b = 0; b < NB; ++b)
+                            if (b < p.batch) {
+                                if (p.y_dtype == BQ_F32)
+                                    static_cast<float*>(p.y)[b * p.n + grow] = y[b];
+                                else
+                                    static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(y[b]);
+                            }
+                    }
+                } else {
+                    const int slot_p = (it0 / S == rb) ? 0 : 1;
+                    float* mine = p.partial + ((c * 2 + slot_p) * p.batch) * kRowsPerCta;
 #pragma unroll
                     for (int b = 0; b < NB; ++b)
-                        if (b < p.batch) {
-                            if (p.y_dtype == BQ_F32)
-                                static_cast<float*>(p.y)[b * p.n + grow] = y[b];
-                            else
-                                static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(y[b]);
-                        }
-                }
-            } else {
-                const int slot_p = (it0 / S == rb) ? 0 : 1;
-                float* mine = p.partial + ((c * 2 + slot_p) * p.batch) * kRowsPerCta;
-#pragma unroll
-                for (int b = 0; b < NB; ++b)
-                    if (b < p.batch) mine[b * kRowsPerCta + row] = y[b];
-                decode_barrier();
-                const int64_t c_first = cta_of_item(rb_first, T, C), c_last = cta_of_item(rb_last, T, C);
-                if (threadIdx.x == 0) {
-                    __threadfence();
-                    const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
-                    s_last = (prev == (unsigned int)(c_last - c_first));
-                    if (s_last) __threadfence();
-                }
-                decode_barrier();
-                if (s_last && grow < p.n) {
-                    for (int b = 0; b < p.batch; ++b) {
-                        float acc = 0.0f;
-                        for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                            const int sl = (item_begin(cc, T, C) / S == rb) ? 0 : 1;
-                            acc += __ldcg(p.partial + ((cc * 2 + sl) * p.batch + b) * kRowsPerCta + row);
-                        }
-                        if (p.y_dtype == BQ_F32)
-                            static_cast<float*>(p.y)[b * p.n + grow] = acc;
-                        else
-                            static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(acc);
+                        if (b < p.batch) mine[b * kRowsPerCta + row] = y[b];
+                    writer_barrier();
+                    const int64_t c_first = cta_of_item(rb_first, T, C), c_last = cta_of_item(rb_last, T, C);
+                    if (threadIdx.x == 0) {
+                        __threadfence();
+                        const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
+                        s_last = (prev == (unsigned int)(c_last - c_first));
+                        if (s_last) __threadfence();
                     }
+                    writer_barrier();
+                    if (s_last && grow < p.n) {
+                        for (int b = 0; b < p.batch; ++b) {
+                            float acc = 0.0f;
+                            for (int64_t cc = c_first; cc <= c_last; ++cc) {
+                                const int sl = (item_begin(cc, T, C) / S == rb) ? 0 : 1;
+                                acc += __ldcg(p.partial + ((cc * 2 + sl) * p.batch + b) * kRowsPerCta + row);
+                            }
+                            if (p.y_dtype == BQ_F32)
+                                static_cast<float*>(p.y)[b * p.n + grow] = acc;
+                            else
+                                static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(acc);
+                        }
+                    }
+                    if (s_last && threadIdx.x == 0) p.counters[rb] = 0u;
                 }
-                if (s_last && threadIdx.x == 0) p.counters[rb] = 0u;
-                decode_barrier();
             }
+            decode_barrier();  // combine buffer reusable
 #pragma unroll
             for (int b = 0; b < NB; ++b) y[b] = 0.0f;
         }
@@ -531,7 +561,7 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.stages_total = (int)(k / 1024);
     pl.row_blocks = (int)((n + kRowsPerCta - 1) / kRowsPerCta);
     const int64_t items = (int64_t)pl.row_blocks * pl.stages_total;
-    const int64_t cap = (int64_t)sm_count() * 2;
+    const int64_t cap = (int64_t)sm_count();
     pl.grid = (int)(items < cap ? items : cap);
     pl.xdata_bytes = (size_t)pl.stages_total * (pl.nt == 1 ? XTile<1>::kBytes : XTile<2>::kBytes);
     pl.counters_off = (pl.xdata_bytes + 255) / 256 * 256;
