@@ -1,50 +1,50 @@
-// Weight-streaming GEMV on the 5th-generation tensor cores (tcgen05): binary
-// g128 and 2-bit-slot ternary g128, batch 1..4, K % 1024 == 0.
+// Weight-streaming GEMV with tensor-core accumulation of the decoded codes
+// (binary g128 and 2-bit-slot ternary g128, batch 1..4, K % 1024 == 0).
 //
-// Why the tensor core at all: at batch 1 the binary format must be consumed at
+// Why the tensor core: at batch 1 the binary format must be consumed at
 // ~126 weights per clock per SM to stream HBM at 80% of its bandwidth, while
-// the integer/logic pipe retires 64 operations per clock per SM, so a decode
-// that spends one instruction per weight cannot keep up (the "1-bit Bonsai 8B"
-// notes, section 4.4, observe the same shift of inline dequantisation towards
-// compute).  Here the CUDA cores only expand bits with LOP3 (a quarter of an
-// instruction per weight) and the multiply-accumulate runs asynchronously on
-// the tensor core with the accumulators in tensor memory:
+// the integer/logic pipe retires 64 operations per clock per SM; any CUDA-core
+// decode that spends half an operation per weight cannot get there (the
+// "1-bit Bonsai 8B" notes, section 4.4, observe the same shift of inline
+// dequantisation towards compute).  So the codes are expanded with a handful of
+// LOP3s into int8 operands and the multiply-accumulate runs on the tensor core.
 //
-//   binary : byte j of (w & (0x01010101 << p)) is 2^p * bit(8j+p) of the
-//            32-bit code word w; eight masks turn one word into eight operand
-//            columns.  The activation operand of that k-slot is Q_k / 2^p.
-//   2-bit  : byte j of ((w >> 2i) & 0x03030303) is the code c = q+1 of trit
-//            4j+i of the word; the activation operand is Q_k.
+// Why the register-fed warp MMA (mma.sync) rather than tcgen05: with N = 8
+// activation columns the tcgen05 MMA (M = 128, K = 32, int8) has a floor of
+// ~46-56 cycles per instruction whatever N is (measured on B200), i.e. at most
+// ~89 A-operand bytes per clock per SM, below the 126 needed; the warp MMA
+// m16n8k32 retires 256 A bytes per clock per SM.  tcgen05 is used where the
+// contraction is dense (the prefill GEMM).
 //
-// Q is the activation in fixed point: per (batch row b, group g) a power of
+//   binary  : byte j of (w & (0x01010101 << p)) is 2^p * bit(8j+p) of the code
+//             word w -- eight masks turn one 32-bit word into eight operand
+//             registers with no shift.  The activation operand of that k-slot
+//             carries Q_k / 2^p, so the product is bit * Q_k exactly.
+//   2-bit   : byte j of ((w >> 2i) & 0x03030303) is the code c = q+1 of trit
+//             4j+i; the activation operand carries Q_k.
+//
+// Q_k is the activation in fixed point: per (batch row b, group g) a power of
 // two 2^E maps the group's largest |x| into [2^29, 2^30); Q = round(x 2^E)
-// (binary: rounded to a multiple of 2^7 so that Q / 2^p is an integer).  Q is
-// split into four signed base-256 digits, one MMA column each (N = 4 * batch
-// slots), and the four int32 column sums are recombined in FP32.  Per group g
-// and row: binary y += s (2^(1-E) sum_k bit_k Q_k - 2^-E sum_k Q_k); 2-bit
-// y += s (2^-E sum_k c_k Q_k - 2^-E sum_k Q_k); i.e. s * sum_k q_k x_k with
-// q = 2 bit - 1 ("Bonsai-27B ... Binary g128": 0 -> -scale, 1 -> +scale) or
-// q = c - 1.  The only rounding before FP32 is that of x to Q: at most 2^-23
-// of the group's largest |x| per element.
+// (binary: rounded to a multiple of 2^7 so that Q / 2^p stays an integer).
+// Q is split into four signed base-256 digits, one MMA column each, and the
+// int32 column sums are recombined in FP32.  Per group and row:
+//   binary : y += s * (2 * 2^-E * sum_k bit_k Q_k - 2^-E * sum_k Q_k)
+//   ternary: y += s * (    2^-E * sum_k c_k   Q_k - 2^-E * sum_k Q_k)
+// (sum of s * q * x with q = 2 bit - 1, resp. q = c - 1; "Bonsai-27B ...
+// Binary g128" section on the representation: 0 -> -scale, 1 -> +scale).  The
+// only rounding before the FP32 recombination is that of x to Q: at most
+// 2^6 units of 2^-E per element, i.e. 2^-23 of the group's largest |x|.
 //
-// CTA roles (one CTA per SM, 128 rows, all 512 TMEM columns):
-//   warps 0-15: decode warps, four per TMEM lane quadrant; warp d handles the
-//               rows of quadrant d & 3 (one row per thread = TMEM lane) and
-//               groups d >> 2 and (d >> 2) + 4 of every stage: it expands the
-//               row's codes into the group's 32 TMEM columns (tcgen05.st) and,
-//               one stage later, reads the group's int32 sums back
-//               (tcgen05.ld) and folds them into y with the scale;
-//   warp 16   : TMA producer (codes with 128-byte swizzle, FP16 scales, and a
-//               bulk copy of the prepared activation operand per stage);
-//   warp 17   : allocates TMEM and issues the MMAs (M = 128, N = 8 or 16,
-//               K = 32 per instruction, A from TMEM, B from shared memory).
-// Each group has its own A (32 columns) and D (16 columns) slot, so the
-// decode of a stage never waits for the MMAs of the same stage.
-// The grid is persistent and splits the (row block, stage) items evenly
-// ("stream-K"); a row block shared by two CTAs is finished by the last one,
-// which adds the partial sums in CTA order (deterministic).  Launches use
-// programmatic dependent launch so that a call's weight stream starts while
-// the previous kernel in the stream drains.
+// Data movement: per pipeline stage (1024 weights of K for 128 rows) a
+// producer warp issues a TMA tile load of the codes (128-byte swizzle), one of
+// the FP16 scales and a bulk copy of the prepared activation operands into
+// shared memory; eight compute warps read conflict-free from there.  The grid
+// is persistent (two CTAs per SM) and splits the sequence of (row block,
+// stage) items evenly ("stream-K"), so there is no tail wave; a row block
+// shared by two CTAs is finished by the last of them, which adds the partial
+// sums in CTA order (deterministic).  Launches use programmatic dependent
+// launch: a call's weight stream starts while the previous kernel in the
+// stream is still draining.
 #include <cuda.h>
 
 #include "bq_internal.cuh"
@@ -55,14 +55,13 @@ namespace tc {
 
 constexpr int kGroupsPerStage = 8;
 constexpr int kRowsPerCta = 128;
-constexpr int kSubs = 4;                         // decode warps per TMEM lane quadrant
-constexpr int kDecodeWarps = 4 * kSubs;          // warp d: quadrant d & 3, sub d >> 2
-constexpr int kProducerWarp = kDecodeWarps;
-constexpr int kMmaWarp = kDecodeWarps + 1;
-constexpr int kThreads = (kDecodeWarps + 2) * 32;
-constexpr int kTmemCols = 512;                   // A: 8 groups x 32 columns, D: 8 groups x 16 columns
-constexpr int kDCol0 = kGroupsPerStage * 32;
-constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr int kComputeWarps = 8;
+constexpr int kRowTiles = 1;  // 16-row MMA tiles per compute warp
+constexpr int kThreads = (kComputeWarps + 1) * 32;
+constexpr int kBfragBytesPerGroup = 4 * 32 * 8;  // 4 MMAs x 32 lanes x (b0, b1)
+constexpr int kTableBytesPerGroup = 4 * 16;      // 4 lanes-in-quad x float4
+constexpr int kXTileBytes = kGroupsPerStage * (kBfragBytesPerGroup + kTableBytesPerGroup);  // 8704
+constexpr uint32_t kWaitPolls = 1u << 23;
 
 template <int FMT>
 struct Fmt;
@@ -77,34 +76,22 @@ struct Fmt<BQ_T2G128> {
     static constexpr int kCoefShift = 0;           // y uses sum(c * x) - sum(x)
 };
 
-// Prepared activation operand of one stage: B in the canonical K-major
-// no-swizzle layout (per MMA: two 16-byte K chunks x NT groups of 8 rows), then
-// the per-(group, batch slot) table {2^a, 2^b, 2^-E sum Q, 0} with 2^(a+b) =
-// 2^(shift - E).
-template <int NT>
-struct XTile {
-    static constexpr int kBBytes = kGroupsPerStage * 4 * 256 * NT;
-    static constexpr int kTabBytes = kGroupsPerStage * 2 * NT * 16;
-    static constexpr int kBytes = kBBytes + kTabBytes;
-};
-
 template <int FMT, int NT>
 struct Layout {
     static constexpr int kCodesBytes = kRowsPerCta * Fmt<FMT>::kRowBytesPerStage;
     static constexpr int kScalesBytes = kRowsPerCta * kGroupsPerStage * 2;
-    static constexpr int kXBytes = XTile<NT>::kBytes;
+    static constexpr int kXBytes = NT * kXTileBytes;
     static constexpr int kStageBytes = (kCodesBytes + kScalesBytes + kXBytes + 1023) / 1024 * 1024;
-    // one CTA per SM
-    static constexpr int kStages = (FMT == BQ_Q1G128) ? (NT == 1 ? 6 : 5) : (NT == 1 ? 4 : 3);
-    static constexpr int kBarriers = 2 * kStages + 2 * kGroupsPerStage + 1;
-    static constexpr int kCombineBytes = (kSubs - 1) * kRowsPerCta * 2 * NT * 4;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarriers * 8 + 16 + kCombineBytes;
+    // two CTAs per SM: 4 (binary, batch <= 2), 3 (binary, batch <= 4) or 2 (2-bit) stages
+    static constexpr int kStages = (FMT == BQ_Q1G128) ? (NT == 1 ? 4 : 3) : 2;
+    static_assert(kComputeWarps * 16 * kRowTiles == kRowsPerCta, "row tiling");
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 2 * kStages * 8;
 };
 
 struct Params {
-    const uint8_t* xdata;    // prepared activation operands, [stage][XTile]
-    float* partial;          // [grid][2][batch][kRowsPerCta]
-    unsigned int* counters;  // [row_blocks], zeroed by the prep kernel
+    const uint8_t* xdata;     // prepared activation operands, [stage][NT][kXTileBytes]
+    float* partial;           // [grid][2][batch][kRowsPerCta] partial sums of split row blocks
+    unsigned int* counters;   // [row_blocks], zeroed by the prep kernel
     void* y;
     int y_dtype;
     int batch;
@@ -114,113 +101,123 @@ struct Params {
     int* status;
 };
 
-// all decode warps / the sub-0 decode warps (the ones that write outputs)
-__device__ __forceinline__ void decode_barrier() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecodeWarps * 32) : "memory");
-}
-__device__ __forceinline__ void writer_barrier() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
-
-__host__ __device__ __forceinline__ int64_t item_begin(int64_t c, int64_t T, int64_t C) { return c * T / C; }
-__device__ __forceinline__ int64_t cta_of_item(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
-
-// Position of weight kk (0..127) of a group in the MMA K order: MMA index and
-// byte (k-slot) inside that MMA's 32-byte K slice.
-template <int FMT>
-__host__ __device__ __forceinline__ void kslot_of(int kk, int& mma, int& kb) {
-    if (FMT == BQ_Q1G128) {  // word q = kk/32, bit 8j+p -> column 8q+p, byte j
-        mma = kk >> 5;
-        const int pp = kk & 7, j = (kk >> 3) & 3;
-        kb = 4 * pp + j;
-    } else {  // word w = kk/16 (MMA w/2), trit 4j+i -> column 4(w&1)+i, byte j
-        const int w = kk >> 4, i = kk & 3, j = (kk >> 2) & 3;
-        mma = w >> 1;
-        kb = 4 * (4 * (w & 1) + i) + j;
-    }
+__device__ __forceinline__ void named_barrier_compute() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory");
 }
 
 // ----------------------------------------------------------------- prep
-// One CTA per group (128 threads, one weight position each).  Writes the
-// group's B digits and table entries into its stage's XTile.
+// One CTA per stage (8 groups).  Writes, for each n-tile (two batch rows x four
+// digits), the B fragments of the 32 MMAs of the stage in lane order and the
+// per-(group, lane-in-quad) recombination table {2^a, 2^b, sum term, 0}.
 template <int FMT, int NT>
-__global__ void __launch_bounds__(128) prep_kernel(const uint16_t* __restrict__ x, int64_t k, int batch,
+__global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ x, int64_t k, int batch,
                                                    uint8_t* __restrict__ xdata, unsigned int* counters,
                                                    int row_blocks) {
-    __shared__ float s_max[4];
-    __shared__ long long s_sum[4];
+    __shared__ int8_t dig[2 * NT][kGroupsPerStage * 128][4];
+    const int st = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // Let the GEMV kernel launch and prefetch weights now; x and the workspace
+    // are touched only after the previous kernel in the stream has finished.
     ptx::pdl_launch_dependents();
     ptx::pdl_wait();
-    const int grp = blockIdx.x;
-    const int kk = threadIdx.x, warp = kk >> 5, lane = kk & 31;
-    if (grp == 0)
+    if (st == 0)
         for (int i = threadIdx.x; i < row_blocks; i += blockDim.x) counters[i] = 0u;
-    const int st = grp / kGroupsPerStage, G = grp % kGroupsPerStage;
-    uint8_t* tile = xdata + (size_t)st * XTile<NT>::kBytes;
-    int mma, kb;
-    kslot_of<FMT>(kk, mma, kb);
-    const int chunk = kb >> 4, byte = kb & 15;
-    uint8_t* bbase = tile + (size_t)(G * 4 + mma) * 256 * NT + chunk * NT * 128 + byte;
+    uint8_t* out = xdata + (size_t)st * NT * kXTileBytes;
+
+    const int G = warp;  // 8 warps <-> 8 groups of the stage
+    const int64_t kbase = ((int64_t)st * kGroupsPerStage + G) * 128;
     for (int bb = 0; bb < 2 * NT; ++bb) {
-        const float xv = (bb < batch) ? bf16_bits_to_float(x[bb * k + (int64_t)grp * 128 + kk]) : 0.0f;
-        float m = fabsf(xv);
+        float xv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (bb < batch) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(x + bb * k + kbase + lane * 4);
+            xv[0] = bf16_lo(raw.x); xv[1] = bf16_hi(raw.x); xv[2] = bf16_lo(raw.y); xv[3] = bf16_hi(raw.y);
+        }
+        float m = fmaxf(fmaxf(fabsf(xv[0]), fabsf(xv[1])), fmaxf(fabsf(xv[2]), fabsf(xv[3])));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (lane == 0) s_max[warp] = m;
-        __syncthreads();
-        m = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
         const int E = (m > 0.f) ? 29 - ilogbf(m) : 0;
-        int q, b;
-        if (FMT == BQ_Q1G128) {
-            q = __float2int_rn(ldexpf(xv, E - 7)) * 128;
-            b = q >> (kk & 7);  // exact: q is a multiple of 2^7
-        } else {
-            q = __float2int_rn(ldexpf(xv, E));
-            b = q;
-        }
-        // balanced base-256 digits: rows n = 4 (bb % 2) + digit of 8-row group bb / 2
-        uint8_t* dst = bbase + (bb >> 1) * 128 + (4 * (bb & 1)) * 16;
+        long long sumq = 0;
 #pragma unroll
-        for (int d = 0; d < 3; ++d) {
-            const int dg = (int8_t)(b & 0xFF);
-            dst[d * 16] = (uint8_t)dg;
-            b = (b - dg) >> 8;
+        for (int i = 0; i < 4; ++i) {
+            const int kk = lane * 4 + i;  // position in the group
+            int q, b;
+            if (FMT == BQ_Q1G128) {
+                q = __float2int_rn(ldexpf(xv[i], E - 7)) * 128;
+                b = q >> (kk & 7);  // exact: q is a multiple of 2^7
+            } else {
+                q = __float2int_rn(ldexpf(xv[i], E));
+                b = q;
+            }
+            sumq += q;
+            const int d0 = (int8_t)(b & 0xFF);
+            b = (b - d0) >> 8;
+            const int d1 = (int8_t)(b & 0xFF);
+            b = (b - d1) >> 8;
+            const int d2 = (int8_t)(b & 0xFF);
+            const int d3 = (b - d2) >> 8;
+            int8_t* dst = dig[bb][G * 128 + kk];
+            dst[0] = (int8_t)d0; dst[1] = (int8_t)d1; dst[2] = (int8_t)d2; dst[3] = (int8_t)d3;
         }
-        dst[3 * 16] = (uint8_t)b;
-        long long sq = q;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-        if (lane == 0) s_sum[warp] = sq;
-        __syncthreads();
-        if (kk == 0) {
-            const long long tot = s_sum[0] + s_sum[1] + s_sum[2] + s_sum[3];
-            const int e = Fmt<FMT>::kCoefShift - E;
+        for (int off = 16; off > 0; off >>= 1) sumq += __shfl_xor_sync(0xffffffffu, sumq, off);
+        if (lane < 2) {
+            const int h = lane;  // digit pair (0,1) or (2,3)
+            const int t = 2 * (bb & 1) + h;
+            const int nt = bb >> 1;
+            const int e = Fmt<FMT>::kCoefShift - E + 16 * h;
             const int a = max(-60, min(60, e));
             float4 tab;
             tab.x = ldexpf(1.0f, a);
             tab.y = ldexpf(1.0f, e - a);
-            tab.z = (float)ldexp((double)tot, -E);
+            tab.z = (h == 0) ? (float)ldexp((double)sumq, -E) : 0.0f;
             tab.w = 0.0f;
-            *reinterpret_cast<float4*>(tile + XTile<NT>::kBBytes + (G * 2 * NT + bb) * 16) = tab;
+            *reinterpret_cast<float4*>(out + nt * kXTileBytes + kGroupsPerStage * kBfragBytesPerGroup +
+                                       (G * 4 + t) * 16) = tab;
         }
-        __syncthreads();
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < NT * kGroupsPerStage * 4 * 32; idx += blockDim.x) {
+        const int ln = idx & 31, q = (idx >> 5) & 3, g8 = (idx >> 7) & 7, nt = idx >> 10;
+        const int gq = ln >> 2, t = ln & 3;
+        const int bb = nt * 2 + (gq >> 2), dg = gq & 3;
+        uint32_t b0 = 0, b1 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int k0, k1;
+            if (FMT == BQ_Q1G128) {
+                k0 = 32 * t + 8 * j + 2 * q;
+                k1 = k0 + 1;
+            } else {
+                k0 = 16 * t + 4 * j + q;
+                k1 = 16 * (t + 4) + 4 * j + q;
+            }
+            b0 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k0][dg] << (8 * j);
+            b1 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k1][dg] << (8 * j);
+        }
+        // lane-contiguous 16 bytes hold (b0, b1) of MMAs 2j and 2j+1 of the group
+        *reinterpret_cast<uint2*>(out + nt * kXTileBytes + ((g8 * 2 + (q >> 1)) * 32 + ln) * 16 + (q & 1) * 8) =
+            make_uint2(b0, b1);
     }
 }
 
 // ----------------------------------------------------------------- main
+// Persistent stream-K kernel.  The work is the sequence of items
+// (row block, stage) in row-block-major order; CTA c takes items
+// [c*T/C, (c+1)*T/C).  A row block whose stages all fall inside one CTA is
+// written directly; a row block split between CTAs is combined by the CTA that
+// finishes it last, adding the partial sums in CTA order (deterministic).
+__host__ __device__ __forceinline__ int64_t item_begin(int64_t c, int64_t T, int64_t C) { return c * T / C; }
+__device__ __forceinline__ int64_t cta_of_item(int64_t i, int64_t T, int64_t C) { return ((i + 1) * C - 1) / T; }
+
 template <int FMT, int NT>
-__global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
+__global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_codes,
                                                               const __grid_constant__ CUtensorMap tm_scales,
                                                               const Params p) {
     using L = Layout<FMT, NT>;
-    constexpr int NB = 2 * NT;  // batch slots
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
     uint64_t* empty = full + L::kStages;
-    uint64_t* a_full = empty + L::kStages;
-    uint64_t* mma_done = a_full + kGroupsPerStage;
-    uint64_t* final_bar = mma_done + kGroupsPerStage;
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(final_bar + 1);
-    float* combine = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(tmem_base_smem) + 16);
     __shared__ int s_last;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,24 +228,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::kStages; ++i) {
             ptx::mbar_init(&full[i], 1);
-            ptx::mbar_init(&empty[i], kDecodeWarps + 1);
+            ptx::mbar_init(&empty[i], kComputeWarps);
         }
-        for (int i = 0; i < kGroupsPerStage; ++i) {
-            ptx::mbar_init(&a_full[i], 4);  // the four quadrant warps of the group's sub
-            ptx::mbar_init(&mma_done[i], 1);
-        }
-        ptx::mbar_init(final_bar, 1);
         ptx::fence_barrier_init();
     }
-    if (warp == kMmaWarp) ptx::tmem_alloc(tmem_base_smem, kTmemCols);
-    ptx::tc_fence_before();
     __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_base_smem;
+    // The next grid in the stream may start its prologue (and its own weight
+    // prefetch) as soon as SMs free up; it waits for this grid before it reads
+    // anything this grid writes.
     ptx::pdl_launch_dependents();
 
-    if (warp == kProducerWarp) {
-        // ------------------------------------------------ TMA producer
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------ producer
         if (lane == 0) {
             ptx::prefetch_tensormap(&tm_codes);
             ptx::prefetch_tensormap(&tm_scales);
@@ -272,7 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
                 ptx::bulk_load(sb + L::kCodesBytes + L::kScalesBytes, p.xdata + (size_t)st * L::kXBytes,
                                L::kXBytes, &full[slot]);
             };
-            // weights do not depend on the previous kernel: stream them first
+            // The weights do not depend on the previous kernel: start streaming
+            // them before waiting for it; the activation operands come after.
             const int pre = nit < L::kStages ? nit : L::kStages;
             for (int it = 0; it < pre; ++it) issue_weights(it);
             ptx::pdl_wait();
@@ -288,232 +280,184 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_tc_kernel(const __grid_const
                 issue_x(it);
                 issued = it + 1;
             }
+            // every copy this CTA issued must land before it may exit
             for (int it = (issued > L::kStages ? issued - L::kStages : 0); it < issued; ++it)
                 if (!ptx::mbar_wait_bounded(&full[it % L::kStages], (it / L::kStages) & 1, kWaitPolls))
                     record_status(p.status, BQ_ERR_TIMEOUT);
         }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            // D s32, A u8, B s8, both K-major, N = 8 NT, M = 128
-            const uint32_t idesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)NT << 17) | (8u << 24);
-            bool ok = true;
-            for (int it = 0; it < nit && ok; ++it) {
-                const int slot = it % L::kStages;
-                if (!ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
-                    record_status(p.status, BQ_ERR_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-                const uint32_t b_s = ptx::smem_u32(smem + slot * L::kStageBytes + L::kCodesBytes + L::kScalesBytes);
+        return;
+    }
+
+    // ---------------------------------------------------- compute warps
+    const int g = lane >> 2, t = lane & 3;
+    const bool writer = (t & 1) == 0;
+    float yacc[kRowTiles][NT][2];
 #pragma unroll
-                for (int G = 0; G < kGroupsPerStage; ++G) {
-                    if (!ptx::mbar_wait_bounded(&a_full[G], it & 1, kWaitPolls)) {
-                        record_status(p.status, BQ_ERR_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
+    for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
+
+    bool alive = true;
+    for (int it = 0; it < nit; ++it) {
+        const int slot = it % L::kStages;
+        const int64_t item = it0 + it;
+        const int rb = (int)(item / S), st = (int)(item % S);
+        if (alive && !ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
+            record_status(p.status, BQ_ERR_TIMEOUT);
+            alive = false;
+        }
+        if (alive) {
+            const uint8_t* stage = smem + slot * L::kStageBytes;
+            const uint8_t* codes_s = stage;
+            const uint16_t* scales_s = reinterpret_cast<const uint16_t*>(stage + L::kCodesBytes);
+            const uint8_t* x_s = stage + L::kCodesBytes + L::kScalesBytes;
+            const int r0 = warp * 16 + g;  // this thread's rows: r0 and r0 + 8
+            // the 8 group scales of both rows (FP16 pairs)
+            const uint4 sv0 = *reinterpret_cast<const uint4*>(scales_s + r0 * kGroupsPerStage);
+            const uint4 sv1 = *reinterpret_cast<const uint4*>(scales_s + (r0 + 8) * kGroupsPerStage);
+            const uint32_t s0w[4] = {sv0.x, sv0.y, sv0.z, sv0.w};
+            const uint32_t s1w[4] = {sv1.x, sv1.y, sv1.z, sv1.w};
+#pragma unroll
+            for (int G = 0; G < kGroupsPerStage; ++G) {
+                uint4 bf[NT][2];
+                float4 tab[NT];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const uint8_t* xt = x_s + nt * kXTileBytes;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        bf[nt][h] = *reinterpret_cast<const uint4*>(xt + ((G * 2 + h) * 32 + lane) * 16);
+                    tab[nt] = *reinterpret_cast<const float4*>(xt + kGroupsPerStage * kBfragBytesPerGroup + (G * 4 + t) * 16);
+                }
+                int acc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
+                if (FMT == BQ_Q1G128) {
+                    const int off = ((G ^ g) << 4) + 4 * t;
+                    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_s + r0 * 128 + off);
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_s + (r0 + 8) * 128 + off);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint64_t bd = ptx::smem_desc_kmajor_noswizzle(b_s + (G * 4 + q) * 256 * NT, 128 * NT, 128);
-                        ptx::mma_i8_ts(tmem + kDCol0 + G * 16, tmem + G * 32 + q * 8, bd, idesc, q > 0 ? 1u : 0u);
-                    }
-                    ptx::tc_commit(&mma_done[G]);
-                }
-                if (ok) ptx::tc_commit(&empty[slot]);
-            }
-            // all MMAs of this CTA finished before TMEM is released
-            ptx::tc_commit(final_bar);
-            if (!ptx::mbar_wait_bounded(final_bar, 0, kWaitPolls)) record_status(p.status, BQ_ERR_TIMEOUT);
-        }
-    } else {
-        // ------------------------------------------------ decode + epilogue warps
-        const int quad = warp & 3, sub = warp >> 2;
-        const int row = quad * 32 + lane;  // row in the CTA tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-        float y[NB];
-        float c1[2][NB], f2[2][NB], cx[2][NB];  // coefficients of groups sub and sub + 4
+                        const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
 #pragma unroll
-        for (int b = 0; b < NB; ++b) y[b] = 0.0f;
-        bool alive = true;
-        bool prev_stage_open = false;  // this warp's groups of the previous stage await their fold
-
-        auto epi_load = [&](int G, uint32_t (&d)[8 * NT]) {
-#pragma unroll
-            for (int h = 0; h < NT; ++h) {
-                uint32_t t8[8];
-                ptx::tmem_ld_x8(tmem + lane_base + kDCol0 + G * 16 + 8 * h, t8);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) d[8 * h + e] = t8[e];
-            }
-        };
-        auto epi_fold = [&](int j, const uint32_t (&d)[8 * NT]) {
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                // columns 4b..4b+3 hold the four digit sums of batch slot b
-                const int lo = (int)d[4 * b] + 256 * (int)d[4 * b + 1];
-                const int hi = (int)d[4 * b + 2] + 256 * (int)d[4 * b + 3];
-                const float v = fmaf((float)hi, 65536.0f, (float)lo);
-                y[b] = fmaf(v * c1[j][b], f2[j][b], y[b]) - cx[j][b];
-            }
-        };
-
-        for (int it = 0; it < nit; ++it) {
-            const int slot = it % L::kStages;
-            const int64_t item = it0 + it;
-            const int rb = (int)(item / S), st = (int)(item % S);
-            if (alive && !ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
-                record_status(p.status, BQ_ERR_TIMEOUT);
-                alive = false;
-            }
-            if (alive) {
-                const uint8_t* stage = smem + slot * L::kStageBytes;
-                const uint16_t* scales_s = reinterpret_cast<const uint16_t*>(stage + L::kCodesBytes);
-                const uint8_t* tab_s = stage + L::kCodesBytes + L::kScalesBytes + XTile<NT>::kBBytes;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int G = sub + 4 * j;
-                    // previous stage's group G: wait for its MMAs, start reading its sums
-                    uint32_t d[8 * NT];
-                    const bool fold = it > 0 && prev_stage_open;
-                    if (it > 0) {
-                        if (!ptx::mbar_wait_bounded(&mma_done[G], (it & 1) ^ 1, kWaitPolls)) {
-                            record_status(p.status, BQ_ERR_TIMEOUT);
-                            alive = false;
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            ptx::mma_u8s8(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1);
                         }
-                        if (fold && alive) {
-                            ptx::tc_fence_after();
-                            epi_load(G, d);
-                        }
-                    }
-                    // decode group G into its 32 TMEM columns
-                    uint32_t a[32];
-                    if (FMT == BQ_Q1G128) {
-                        const uint4 w = *reinterpret_cast<const uint4*>(stage + row * 128 + ((G ^ (row & 7)) << 4));
-                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-#pragma unroll
-                            for (int pp = 0; pp < 8; ++pp) a[8 * q + pp] = wv[q] & (0x01010101u << pp);
-                    } else {
-                        const uint8_t* box = stage + (G >> 2) * (kRowsPerCta * 128) + row * 128;
-                        const int c0 = 2 * (G & 3);
-                        const uint4 wa = *reinterpret_cast<const uint4*>(box + ((c0 ^ (row & 7)) << 4));
-                        const uint4 wb = *reinterpret_cast<const uint4*>(box + (((c0 + 1) ^ (row & 7)) << 4));
-                        const uint32_t wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-                        for (int w8 = 0; w8 < 8; ++w8)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) a[4 * w8 + i] = (wv[w8] >> (2 * i)) & 0x03030303u;
-                    }
-                    ptx::tmem_st_x32(tmem + lane_base + G * 32, a);
-                    if (fold && alive) {
-                        ptx::tc_wait_ld();
-                        epi_fold(j, d);
-                    }
-                    // coefficients of group G
-                    const float s = half_bits_to_float(scales_s[row * kGroupsPerStage + G]);
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        const float4 tab = *reinterpret_cast<const float4*>(tab_s + (G * NB + b) * 16);
-                        c1[j][b] = s * tab.x;
-                        f2[j][b] = tab.y;
-                        cx[j][b] = s * tab.z;
-                    }
-                    ptx::tc_wait_st();
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&a_full[G]);
-                }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&empty[slot]);
-            }
-            prev_stage_open = true;
-            // ---------------------------------------- row block finished here?
-            if (st != S - 1 && it != nit - 1) continue;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int G = sub + 4 * j;
-                if (alive && !ptx::mbar_wait_bounded(&mma_done[G], it & 1, kWaitPolls)) {
-                    record_status(p.status, BQ_ERR_TIMEOUT);
-                    alive = false;
-                }
-                if (alive) {
-                    uint32_t d[8 * NT];
-                    ptx::tc_fence_after();
-                    epi_load(G, d);
-                    ptx::tc_wait_ld();
-                    epi_fold(j, d);
-                }
-            }
-            prev_stage_open = false;
-            // combine the four subs' partial sums of each row (fixed order)
-            if (sub > 0) {
-#pragma unroll
-                for (int b = 0; b < NB; ++b) combine[((sub - 1) * NB + b) * kRowsPerCta + row] = y[b];
-            }
-            decode_barrier();
-            if (sub == 0) {
-#pragma unroll
-                for (int k2 = 0; k2 < kSubs - 1; ++k2)
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) y[b] += combine[(k2 * NB + b) * kRowsPerCta + row];
-                const int64_t rb_first = (int64_t)rb * S, rb_last = rb_first + S - 1;
-                const bool whole = rb_first >= it0 && rb_last < it1;
-                const int64_t grow = (int64_t)rb * kRowsPerCta + row;
-                if (whole) {
-                    if (grow < p.n) {
-#pragma unroll
-                        for (int b = 0; b < NB; ++b)
-                            if (b < p.batch) {
-                                if (p.y_dtype == BQ_F32)
-                                    static_cast<float*>(p.y)[b * p.n + grow] = y[b];
-                                else
-                                    static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(y[b]);
-                            }
                     }
                 } else {
-                    const int slot_p = (it0 / S == rb) ? 0 : 1;
-                    float* mine = p.partial + ((c * 2 + slot_p) * p.batch) * kRowsPerCta;
+                    const uint8_t* box = codes_s + (G >> 2) * (kRowsPerCta * 128);
+                    const int c0 = 2 * (G & 3), c1 = c0 + 1;
+                    const int offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
+                    const uint32_t w0a = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offa);
+                    const uint32_t w0b = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offb);
+                    const uint32_t w1a = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offa);
+                    const uint32_t w1b = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offb);
 #pragma unroll
-                    for (int b = 0; b < NB; ++b)
-                        if (b < p.batch) mine[b * kRowsPerCta + row] = y[b];
-                    writer_barrier();
-                    const int64_t c_first = cta_of_item(rb_first, T, C), c_last = cta_of_item(rb_last, T, C);
-                    if (threadIdx.x == 0) {
-                        __threadfence();
-                        const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
-                        s_last = (prev == (unsigned int)(c_last - c_first));
-                        if (s_last) __threadfence();
-                    }
-                    writer_barrier();
-                    if (s_last && grow < p.n) {
-                        for (int b = 0; b < p.batch; ++b) {
-                            float acc = 0.0f;
-                            for (int64_t cc = c_first; cc <= c_last; ++cc) {
-                                const int sl = (item_begin(cc, T, C) / S == rb) ? 0 : 1;
-                                acc += __ldcg(p.partial + ((cc * 2 + sl) * p.batch + b) * kRowsPerCta + row);
-                            }
-                            if (p.y_dtype == BQ_F32)
-                                static_cast<float*>(p.y)[b * p.n + grow] = acc;
-                            else
-                                static_cast<uint16_t*>(p.y)[b * p.n + grow] = float_to_bf16_bits(acc);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
+                        const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
+                        const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            ptx::mma_u8s8(acc[nt], a0, a1, a2, a3, b0, b1);
                         }
                     }
-                    if (s_last && threadIdx.x == 0) p.counters[rb] = 0u;
+                }
+                const float s0 = half_bits_to_float((uint16_t)(s0w[G >> 1] >> (16 * (G & 1))));
+                const float s1 = half_bits_to_float((uint16_t)(s1w[G >> 1] >> (16 * (G & 1))));
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    // D0 + 256 D1 is exact in int32 (|D| < 2^21)
+                    const float v0 = (float)(acc[nt][0] + 256 * acc[nt][1]);
+                    const float v1 = (float)(acc[nt][2] + 256 * acc[nt][3]);
+                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    yacc[0][nt][0] = fmaf(s0, u0, yacc[0][nt][0]);
+                    yacc[0][nt][1] = fmaf(s1, u1, yacc[0][nt][1]);
                 }
             }
-            decode_barrier();  // combine buffer reusable
-#pragma unroll
-            for (int b = 0; b < NB; ++b) y[b] = 0.0f;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&empty[slot]);
         }
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == kMmaWarp) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, kTmemCols);
+        // ---------------------------------------- row block finished here?
+        if (st != S - 1 && it != nit - 1) continue;
+#pragma unroll
+        for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) yacc[j][nt][r] += __shfl_xor_sync(0xffffffffu, yacc[j][nt][r], 1);
+        const int64_t rb_first = (int64_t)rb * S, rb_last = rb_first + S - 1;
+        const bool whole = rb_first >= it0 && rb_last < it1;
+        if (whole) {
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int bb = nt * 2 + (t >> 1);
+                            const int64_t row = (int64_t)rb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r;
+                            if (bb < p.batch && row < p.n) {
+                                if (p.y_dtype == BQ_F32)
+                                    static_cast<float*>(p.y)[bb * p.n + row] = yacc[j][nt][r];
+                                else
+                                    static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[j][nt][r]);
+                            }
+                        }
+            }
+        } else {
+            const int slot_p = (item_begin(c, T, C) / S == rb) ? 0 : 1;
+            float* mine = p.partial + ((c * 2 + slot_p) * p.batch) * kRowsPerCta;
+            if (writer) {
+#pragma unroll
+                for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int bb = nt * 2 + (t >> 1);
+                            if (bb < p.batch)
+                                mine[bb * kRowsPerCta + warp * (16 * kRowTiles) + j * 16 + g + 8 * r] = yacc[j][nt][r];
+                        }
+            }
+            __threadfence();
+            named_barrier_compute();
+            const int64_t c_first = cta_of_item(rb_first, T, C), c_last = cta_of_item(rb_last, T, C);
+            if (threadIdx.x == 0) {
+                const unsigned int prev = atomicAdd(&p.counters[rb], 1u);
+                s_last = (prev == (unsigned int)(c_last - c_first));
+            }
+            named_barrier_compute();
+            if (s_last) {
+                __threadfence();
+                for (int i = threadIdx.x; i < kRowsPerCta * p.batch; i += kComputeWarps * 32) {
+                    const int bb = i / kRowsPerCta, rin = i % kRowsPerCta;
+                    const int64_t row = (int64_t)rb * kRowsPerCta + rin;
+                    if (row >= p.n) continue;
+                    float acc = 0.0f;
+                    for (int64_t cc = c_first; cc <= c_last; ++cc) {
+                        const int sl = (item_begin(cc, T, C) / S == rb) ? 0 : 1;
+                        acc += __ldcg(p.partial + ((cc * 2 + sl) * p.batch + bb) * kRowsPerCta + rin);
+                    }
+                    if (p.y_dtype == BQ_F32)
+                        static_cast<float*>(p.y)[bb * p.n + row] = acc;
+                    else
+                        static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(acc);
+                }
+                if (threadIdx.x == 0) p.counters[rb] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kRowTiles; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
     }
 }
 
@@ -560,10 +504,11 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.nt = (batch + 1) / 2;
     pl.stages_total = (int)(k / 1024);
     pl.row_blocks = (int)((n + kRowsPerCta - 1) / kRowsPerCta);
+    const int ctas_per_sm = 2;
     const int64_t items = (int64_t)pl.row_blocks * pl.stages_total;
-    const int64_t cap = (int64_t)sm_count();
+    const int64_t cap = (int64_t)sm_count() * ctas_per_sm;
     pl.grid = (int)(items < cap ? items : cap);
-    pl.xdata_bytes = (size_t)pl.stages_total * (pl.nt == 1 ? XTile<1>::kBytes : XTile<2>::kBytes);
+    pl.xdata_bytes = (size_t)pl.stages_total * pl.nt * kXTileBytes;
     pl.counters_off = (pl.xdata_bytes + 255) / 256 * 256;
     pl.partial_off = (pl.counters_off + (size_t)pl.row_blocks * 4 + 255) / 256 * 256;
     pl.total = pl.partial_off + (size_t)pl.grid * 2 * batch * kRowsPerCta * 4;
@@ -618,15 +563,15 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     prm.row_blocks = pl.row_blocks;
     prm.status = device_status_ptr();
     if (!prm.status) return cudaErrorUnknown;
-    // Both kernels are programmatic dependents of whatever precedes them in the
-    // stream and wait (griddepcontrol.wait) before touching data that it may
-    // still produce or read.
+    // Both kernels are launched as programmatic dependents of whatever precedes
+    // them in the stream; each waits (griddepcontrol.wait) before touching data
+    // the predecessor may still produce or read.
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr.val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)G);
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3(pl.stages_total);
+    cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cfg.attrs = &attr;
