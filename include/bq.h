@@ -125,6 +125,25 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
                   const uint16_t* x, int batch, void* y, int y_dtype,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free GEMV.  (The pages have no counterpart: this serves callers,
+ * not the method.)  Same product, arguments and layouts as bq_gemv, but with no
+ * workspace argument: for callers that cannot allocate device memory where they
+ * run it -- a host that owns all device memory and passes a plugin only its
+ * inputs and outputs, or a path where cudaMalloc's possible device
+ * synchronisation is not acceptable.  The scratch it needs lives in one fixed
+ * array of BQ_NOALLOC_SCRATCH_BYTES bytes inside the library, held on every GPU
+ * that loads the library until the process exits.  Shapes whose scratch need
+ * (bq_gemv_workspace_bytes) exceeds that size return BQ_ERR_WORKSPACE and
+ * nothing is launched.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before capturing a stream.  All calls share the array and it keeps the
+ * last call's contents (what must start at zero is cleared by every call); two
+ * calls that overlap on the GPU race on it, so order them on one stream.
+ * Allocates nothing (no cudaMalloc / cudaFree).  Asynchronous on `stream`. */
+#define BQ_NOALLOC_SCRATCH_BYTES (4u << 20)
+bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                          const uint16_t* x, int batch, void* y, int y_dtype, void* stream);
+
 /* ------------------------------------------------------------------- GEMM */
 /* Workspace bytes bq_gemm needs for T tokens (0 if none); -1 if invalid. */
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t);

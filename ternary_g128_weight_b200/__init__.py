@@ -27,7 +27,7 @@ FORMATS = {"q1g128": BQ_Q1G128, "t2g128": BQ_T2G128, "t5p8": BQ_T5P8G128}
 EXPORTED = [
     "bq_codes_bytes", "bq_scales_bytes", "bq_effective_bits",
     "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8",
-    "bq_gemv_workspace_bytes", "bq_gemv", "bq_gemm_workspace_bytes", "bq_gemm",
+    "bq_gemv_workspace_bytes", "bq_gemv", "bq_gemv_noalloc", "bq_gemm_workspace_bytes", "bq_gemm",
     "bq_check", "bq_debug_wait_timeout", "bq_status_string", "bq_version",
 ]
 
@@ -59,6 +59,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f.restype = i32
     L.bq_gemv_workspace_bytes.argtypes = [i32, i64, i64, i32]; L.bq_gemv_workspace_bytes.restype = i64
     L.bq_gemv.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, i32, vp, sz, vp]; L.bq_gemv.restype = i32
+    L.bq_gemv_noalloc.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, i32, vp]; L.bq_gemv_noalloc.restype = i32
     L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]; L.bq_gemm_workspace_bytes.restype = i64
     L.bq_gemm.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]; L.bq_gemm.restype = i32
     L.bq_check.argtypes = [vp]; L.bq_check.restype = i32
@@ -167,6 +168,26 @@ def bq_gemv(fmt, codes, scales, n: int, k: int, x, y=None, y_dtype: int = BQ_BF1
     st = load().bq_gemv(f, _ptr(codes), _ptr(scales), n, k, _ptr(x), batch, _ptr(y), int(y_dtype),
                         _ptr(workspace), wsb, _stream(stream))
     _check(st, "bq_gemv")
+    return y
+
+
+BQ_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def bq_gemv_noalloc(fmt, codes, scales, n: int, k: int, x, y=None, y_dtype: int = BQ_BF16, stream=None):
+    """bq_gemv without a workspace argument: the library's fixed scratch array is
+    used instead (for callers that cannot allocate device memory).  Calls that
+    overlap on the GPU race on that array; make the first call on a device
+    before capturing a stream."""
+    import torch
+    f = _fmt(fmt)
+    batch = x.shape[0] if x.dim() == 2 else 1
+    if y is None:
+        y = torch.empty((batch, n), dtype=torch.float32 if y_dtype == BQ_F32 else torch.bfloat16,
+                        device=x.device)
+    st = load().bq_gemv_noalloc(f, _ptr(codes), _ptr(scales), n, k, _ptr(x), batch, _ptr(y), int(y_dtype),
+                                _stream(stream))
+    _check(st, "bq_gemv_noalloc")
     return y
 
 
