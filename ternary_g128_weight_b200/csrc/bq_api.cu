@@ -142,19 +142,19 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-// Token chunk the GEMM hands to the GEMV kernels while no tensor-core GEMM
-// covers the shape: 4 (tensor-core decode path) or 16 (CUDA-core path).
-static int gemm_chunk(int fmt, int64_t n, int64_t k, int64_t t) {
-    const int c = (int)(t < 4 ? t : 4);
-    return (c > 0 && gemv_tc_eligible(fmt, n, k, c)) ? 4 : BQ_MAX_BATCH;
+// Prefill dispatch: up to 4 tokens run the GEMV tensor-core path (the weight
+// stream dominates and it is bit-identical with bq_gemv); more tokens run the
+// tcgen05 GEMM; shapes neither takes run the CUDA-core GEMV in chunks of 16.
+static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
+    return t <= 4 && gemv_tc_eligible(fmt, n, k, (int)t);
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
-    if (t == 0) return 0;
-    const int chunk = gemm_chunk(fmt, n, k, t);
-    const int b = (int)(t < chunk ? t : chunk);
-    return gemv_tc_workspace_bytes(fmt, n, k, b);
+    if (t == 0 || n == 0 || k == 0) return 0;
+    if (gemm_uses_gemv(fmt, n, k, t)) return gemv_tc_workspace_bytes(fmt, n, k, (int)t);
+    if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_workspace_bytes(n, k, t);
+    return 0;
 }
 
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -172,17 +172,18 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     cudaStream_t s = as_stream(stream);
     if (k == 0)
         return cudaMemsetAsync(y, 0, (size_t)t * n * 2, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
-    const int chunk = gemm_chunk(fmt, n, k, t);
-    for (int64_t t0 = 0; t0 < t; t0 += chunk) {
-        const int b = (int)((t - t0) < chunk ? (t - t0) : chunk);
-        cudaError_t e;
-        if (need > 0 && gemv_tc_eligible(fmt, n, k, b))
-            e = launch_gemv_tc(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, workspace, s);
-        else
+    cudaError_t e = cudaSuccess;
+    if (gemm_uses_gemv(fmt, n, k, t)) {
+        e = launch_gemv_tc(fmt, codes, scales, n, k, x, (int)t, y, BQ_BF16, workspace, s);
+    } else if (gemm_tc_eligible(fmt, n, k, t)) {
+        e = launch_gemm_tc(fmt, codes, scales, n, k, x, t, y, workspace, s);
+    } else {
+        for (int64_t t0 = 0; t0 < t && e == cudaSuccess; t0 += BQ_MAX_BATCH) {
+            const int b = (int)((t - t0) < BQ_MAX_BATCH ? (t - t0) : BQ_MAX_BATCH);
             e = launch_gemv_simt(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, s);
-        if (e != cudaSuccess) return BQ_ERR_CUDA;
+        }
     }
-    return BQ_OK;
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 bq_status bq_check(void* stream) {

@@ -61,4 +61,10 @@ int64_t gemv_tc_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                            const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s);
 
+// tcgen05 prefill GEMM (all formats, K % 128 == 0).
+bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t);
+int64_t gemm_tc_workspace_bytes(int64_t n, int64_t k, int64_t t);
+cudaError_t launch_gemm_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                           const uint16_t* x, int64_t t, uint16_t* y, void* workspace, cudaStream_t s);
+
 }  // namespace bq
