@@ -96,55 +96,93 @@ __global__ void __launch_bounds__(256) xprep_f16_kernel(const uint16_t* __restri
 }
 
 // ----------------------------------------------------------------- dequant
-// 64 weights of one row (k0 .. k0+63) -> 32 FP16 pairs s*q.
+// The packed bytes and the scale of 64 weights of one row (k0 .. k0+63).
+// Loaded several stages ahead of their use so that the load latency overlaps
+// the dequantisation and the MMAs of the stages in between.
+struct RowChunk {
+    uint4 codes;     // binary: 8 bytes; 2-bit: 16 bytes; 5-per-byte: 14 bytes from an even offset
+    uint32_t scale;  // FP16 bits (0 for rows past the end)
+};
+
 template <int FMT>
-__device__ __forceinline__ void dequant_row64(const Params& p, int64_t row, int64_t k0, uint32_t (&h)[32]) {
-    if (row >= p.n) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) h[i] = 0u;
-        return;
-    }
+__device__ __forceinline__ RowChunk load_chunk(const Params& p, int64_t row, int64_t k0) {
+    RowChunk c;
+    c.codes = make_uint4(0u, 0u, 0u, 0u);
+    c.scale = 0u;
+    if (row >= p.n) return c;
     const int64_t G = p.k / 128;
-    const uint32_t s = p.scales[row * G + (k0 >> 7)];
+    c.scale = __ldg(p.scales + row * G + (k0 >> 7));
+    if (FMT == BQ_Q1G128) {
+        const uint2 b = __ldg(reinterpret_cast<const uint2*>(p.codes + row * (p.k / 8) + (k0 >> 3)));
+        c.codes = make_uint4(b.x, b.y, 0u, 0u);
+    } else if (FMT == BQ_T2G128) {
+        c.codes = __ldg(reinterpret_cast<const uint4*>(p.codes + row * (p.k / 4) + (k0 >> 2)));
+    } else {
+        // trits 64h .. 64h+63 of the group live in bytes 12h .. 12h+13 (even offset)
+        const uint16_t* src =
+            reinterpret_cast<const uint16_t*>(p.codes + row * (26 * G) + (k0 >> 7) * 26 + ((k0 & 127) ? 12 : 0));
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = __ldg(src + 2 * i);
+            const uint32_t hi = (2 * i + 1 < 7) ? (uint32_t)__ldg(src + 2 * i + 1) : 0u;
+            w[i] = lo | (hi << 16);
+        }
+        c.codes = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return c;
+}
+
+// Base-3 digits of trits BASE .. BASE+63 of a group (5 per byte, least
+// significant first) from the bytes load_chunk fetched.
+template <int BASE>
+__device__ __forceinline__ void t5p8_codes(const RowChunk& c, uint32_t (&code)[64]) {
+    const uint32_t wv[4] = {c.codes.x, c.codes.y, c.codes.z, c.codes.w};
+    constexpr int kByte0 = BASE ? 12 : 0;  // first loaded byte
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const int kk = BASE + i, j = kk / 5 - kByte0, d = kk % 5;
+        uint32_t v = (wv[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+        // floor(v / 3^d) by multiply-shift (exact for v < 256), then mod 3
+#pragma unroll
+        for (int e = 0; e < d; ++e) v = (v * 171u) >> 9;
+        code[i] = v - 3u * ((v * 171u) >> 9);
+    }
+}
+
+// 64 weights -> 32 FP16 pairs s*q.
+template <int FMT>
+__device__ __forceinline__ void dequant_chunk(const RowChunk& c, int64_t k0, uint32_t (&h)[32]) {
+    const uint32_t s = c.scale;
     const uint32_t ss = s | (s << 16);
     if (FMT == BQ_Q1G128) {
         // bit 1 -> +s, bit 0 -> -s: flip the FP16 sign where the bit is 0
-        const uint2 b = *reinterpret_cast<const uint2*>(p.codes + row * (p.k / 8) + (k0 >> 3));
-        const uint32_t nb[2] = {~b.x, ~b.y};
+        const uint32_t nb[2] = {~c.codes.x, ~c.codes.y};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const uint32_t w = nb[i >> 4];
             const int j = 2 * (i & 15);
             h[i] = ss ^ (((w >> j) & 1u) << 15) ^ (((w >> (j + 1)) & 1u) << 31);
         }
-    } else if (FMT == BQ_T2G128) {
-        const uint4 b = *reinterpret_cast<const uint4*>(p.codes + row * (p.k / 4) + (k0 >> 2));
-        const uint32_t wv[4] = {b.x, b.y, b.z, b.w};
+    } else {
+        // code c in {0, 1, 2} -> -s, 0, +s: magnitude s unless c == 1, sign when c == 0
+        uint32_t code[64];
+        if (FMT == BQ_T2G128) {
+            const uint32_t wv[4] = {c.codes.x, c.codes.y, c.codes.z, c.codes.w};
+#pragma unroll
+            for (int i = 0; i < 64; ++i) code[i] = (wv[i >> 4] >> (2 * (i & 15))) & 3u;
+        } else if ((k0 & 127) == 0) {
+            t5p8_codes<0>(c, code);
+        } else {
+            t5p8_codes<64>(c, code);
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const uint32_t w = wv[i >> 3];
-            const int j = 4 * (i & 7);
-            const uint32_t c0 = (w >> j) & 3u, c1 = (w >> (j + 2)) & 3u;
-            // code 0 -> -s, 1 -> 0, 2 -> +s
-            const uint32_t lo = (c0 == 1u) ? 0u : (s | (c0 == 0u ? 0x8000u : 0u));
-            const uint32_t hi = (c1 == 1u) ? 0u : (s | (c1 == 0u ? 0x8000u : 0u));
+            const uint32_t c0 = code[2 * i], c1 = code[2 * i + 1];
+            const uint32_t lo = (c0 == 1u) ? 0u : (s | ((c0 == 0u) ? 0x8000u : 0u));
+            const uint32_t hi = (c1 == 1u) ? 0u : (s | ((c1 == 0u) ? 0x8000u : 0u));
             h[i] = lo | (hi << 16);
         }
-    } else {
-        const int64_t G = p.k / 128;
-        const uint8_t* grp = p.codes + row * (26 * G) + (k0 >> 7) * 26;
-        const int base = (int)(k0 & 127);  // 0 or 64
-        uint32_t q[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const int kk = base + i, j = kk / 5, d = kk % 5;
-            uint32_t v = grp[j];
-            v = (d == 0) ? v : (d == 1) ? v / 3u : (d == 2) ? v / 9u : (d == 3) ? v / 27u : v / 81u;
-            const uint32_t c = v % 3u;
-            q[i] = (c == 1u) ? 0u : (s | (c == 0u ? 0x8000u : 0u));
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) h[i] = q[2 * i] | (q[2 * i + 1] << 16);
     }
 }
 
@@ -189,29 +227,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (warp < kDequantWarps) {
         // ------------------------------------------------ dequant producers
         const int r = warp * 32 + lane;
-        int64_t it = 0;
-        bool alive = true;
-        for (int64_t tile = blockIdx.x; tile < tiles && alive; tile += gridDim.x) {
-            const int64_t mb = tile % mb_count;
-            for (int st = 0; st < stages_per_tile; ++st, ++it) {
-                const int slot = (int)(it % kStages);
-                if (it >= kStages &&
-                    !ptx::mbar_wait_bounded(&empty[slot], (uint32_t)(((it / kStages) - 1) & 1), kWaitPolls)) {
-                    record_status(p.status, BQ_ERR_TIMEOUT);
-                    alive = false;
-                    break;
-                }
-                uint32_t h[32];
-                dequant_row64<FMT>(p, mb * kTileM + r, (int64_t)st * kStageK, h);
-                uint8_t* a = smem + slot * kStageBytes + r * 128;
+        const int64_t my_tiles = (tiles > blockIdx.x) ? (tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+        const int64_t total = my_tiles * stages_per_tile;
+        // the chunk of stage g of this CTA's sequence (tile-major, then K)
+        auto chunk_of = [&](int64_t g) {
+            const int64_t tile = blockIdx.x + (g / stages_per_tile) * gridDim.x;
+            const int64_t st = g % stages_per_tile;
+            return load_chunk<FMT>(p, (tile % mb_count) * kTileM + r, st * kStageK);
+        };
+        constexpr int kAhead = 3;
+        RowChunk pipe[kAhead];
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) =
-                        make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
-                ptx::fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&full_a[slot]);
+        for (int i = 0; i < kAhead; ++i) pipe[i] = (i < total) ? chunk_of(i) : RowChunk{};
+        for (int64_t it = 0; it < total; ++it) {
+            const RowChunk cur = pipe[0];
+#pragma unroll
+            for (int i = 0; i < kAhead - 1; ++i) pipe[i] = pipe[i + 1];
+            if (it + kAhead < total) pipe[kAhead - 1] = chunk_of(it + kAhead);
+            const int slot = (int)(it % kStages);
+            if (it >= kStages &&
+                !ptx::mbar_wait_bounded(&empty[slot], (uint32_t)(((it / kStages) - 1) & 1), kWaitPolls)) {
+                record_status(p.status, BQ_ERR_TIMEOUT);
+                break;
             }
+            uint32_t h[32];
+            dequant_chunk<FMT>(cur, (it % stages_per_tile) * kStageK, h);
+            uint8_t* a = smem + slot * kStageBytes + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+            ptx::fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&full_a[slot]);
         }
     } else if (warp == kTmaWarp) {
         // ------------------------------------------------ activation TMA
