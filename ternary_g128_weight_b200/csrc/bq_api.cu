@@ -78,6 +78,27 @@ int* device_status_ptr() {
 
 }  // namespace bq
 
+namespace bq {
+GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
+    if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
+    if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
+    return GemvPath::Simt;
+}
+
+int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
+    return gemv_path(fmt, n, k, batch) == GemvPath::SplitK ? gemv_tc_workspace_bytes(fmt, n, k, batch) : 0;
+}
+
+cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                        const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s) {
+    switch (gemv_path(fmt, n, k, batch)) {
+        case GemvPath::Rows: return launch_gemv_rows(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
+        case GemvPath::SplitK: return launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
+        default: return launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
+    }
+}
+}  // namespace bq
+
 using namespace bq;
 
 extern "C" {
@@ -112,9 +133,11 @@ bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* sca
     return pack_common(BQ_T5P8G128, w, n, k, scales_in, codes, scales, stream);
 }
 
+
 int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
-    return gemv_tc_workspace_bytes(fmt, n, k, batch);
+    if (n == 0 || k == 0) return 0;
+    return gemv_workspace_bytes(fmt, n, k, batch);
 }
 
 bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -134,25 +157,22 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
         const size_t bytes = (size_t)batch * n * (y_dtype == BQ_F32 ? 4 : 2);
         return cudaMemsetAsync(y, 0, bytes, as_stream(stream)) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     }
-    cudaError_t e;
-    if (need > 0 && gemv_tc_eligible(fmt, n, k, batch))
-        e = launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, as_stream(stream));
-    else
-        e = launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, as_stream(stream));
+    const cudaError_t e = launch_gemv(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, as_stream(stream));
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-// Prefill dispatch: up to 4 tokens run the GEMV tensor-core path (the weight
-// stream dominates and it is bit-identical with bq_gemv); more tokens run the
-// tcgen05 GEMM; shapes neither takes run the CUDA-core GEMV in chunks of 16.
+// Prefill dispatch: up to 4 tokens run the tensor-core GEMV paths (the weight
+// stream dominates and the result is bit-identical with bq_gemv); more tokens
+// run the tcgen05 GEMM; shapes neither takes run the CUDA-core GEMV in chunks
+// of 16.
 static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
-    return t <= 4 && gemv_tc_eligible(fmt, n, k, (int)t);
+    return t <= 4 && gemv_path(fmt, n, k, (int)t) != GemvPath::Simt;
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
     if (t == 0 || n == 0 || k == 0) return 0;
-    if (gemm_uses_gemv(fmt, n, k, t)) return gemv_tc_workspace_bytes(fmt, n, k, (int)t);
+    if (gemm_uses_gemv(fmt, n, k, t)) return gemv_workspace_bytes(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_workspace_bytes(n, k, t);
     return 0;
 }
@@ -174,7 +194,7 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
         return cudaMemsetAsync(y, 0, (size_t)t * n * 2, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (gemm_uses_gemv(fmt, n, k, t)) {
-        e = launch_gemv_tc(fmt, codes, scales, n, k, x, (int)t, y, BQ_BF16, workspace, s);
+        e = launch_gemv(fmt, codes, scales, n, k, x, (int)t, y, BQ_BF16, workspace, s);
     } else if (gemm_tc_eligible(fmt, n, k, t)) {
         e = launch_gemm_tc(fmt, codes, scales, n, k, x, t, y, workspace, s);
     } else {

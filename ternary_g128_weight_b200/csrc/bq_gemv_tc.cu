@@ -20,12 +20,14 @@
 //             word w -- eight masks turn one 32-bit word into eight operand
 //             registers with no shift.  The activation operand of that k-slot
 //             carries Q_k / 2^p, so the product is bit * Q_k exactly.
-//   2-bit   : byte j of ((w >> 2i) & 0x03030303) is the code c = q+1 of trit
-//             4j+i; the activation operand carries Q_k.
+//   2-bit   : byte j of (w & (0x03030303 << 2i)) is 4^i * c, c = q+1 the code
+//             of trit 4j+i -- four masks per word, again no shift; the
+//             activation operand of that k-slot carries Q_k / 4^i.
 //
 // Q_k is the activation in fixed point: per (batch row b, group g) a power of
 // two 2^E maps the group's largest |x| into [2^29, 2^30); Q = round(x 2^E)
-// (binary: rounded to a multiple of 2^7 so that Q / 2^p stays an integer).
+// (rounded to a multiple of 2^7, binary, or 2^6, 2-bit, so that Q / 2^p and
+// Q / 4^i stay integers).
 // Q is split into four signed base-256 digits, one MMA column each, and the
 // int32 column sums are recombined in FP32.  Per group and row:
 //   binary : y += s * (2 * 2^-E * sum_k bit_k Q_k - 2^-E * sum_k Q_k)
@@ -126,6 +128,22 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
 
     const int G = warp;  // 8 warps <-> 8 groups of the stage
     const int64_t kbase = ((int64_t)st * kGroupsPerStage + G) * 128;
+    // Per n-tile: does any batch row of this group need the two-factor
+    // recombination (2^e below the normal FP32 range)?  The flag is shared by
+    // the group's four table entries so that the GEMV kernel's choice is
+    // uniform across the warp.
+    bool two_factor[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) two_factor[nt] = false;
+    for (int bb = 0; bb < 2 * NT && bb < batch; ++bb) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(x + bb * k + kbase + lane * 4);
+        float m = fmaxf(fmaxf(fabsf(bf16_lo(raw.x)), fabsf(bf16_hi(raw.x))),
+                        fmaxf(fabsf(bf16_lo(raw.y)), fabsf(bf16_hi(raw.y))));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const int E = (m > 0.f) ? 29 - ilogbf(m) : 0;
+        if (Fmt<FMT>::kCoefShift - E < -126) two_factor[bb >> 1] = true;
+    }
     for (int bb = 0; bb < 2 * NT; ++bb) {
         float xv[4] = {0.f, 0.f, 0.f, 0.f};
         if (bb < batch) {
@@ -145,8 +163,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
                 q = __float2int_rn(ldexpf(xv[i], E - 7)) * 128;
                 b = q >> (kk & 7);  // exact: q is a multiple of 2^7
             } else {
-                q = __float2int_rn(ldexpf(xv[i], E));
-                b = q;
+                q = __float2int_rn(ldexpf(xv[i], E - 6)) * 64;
+                b = q >> (2 * (kk & 3));  // exact: q is a multiple of 2^6
             }
             sumq += q;
             const int d0 = (int8_t)(b & 0xFF);
@@ -165,12 +183,14 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
             const int t = 2 * (bb & 1) + h;
             const int nt = bb >> 1;
             const int e = Fmt<FMT>::kCoefShift - E + 16 * h;
-            const int a = max(-60, min(60, e));
+            // one factor 2^e when it is a normal float, else 2^a * 2^(e-a)
+            const bool two = two_factor[nt];
+            const int a = two ? max(-60, min(60, e)) : e;
             float4 tab;
             tab.x = ldexpf(1.0f, a);
             tab.y = ldexpf(1.0f, e - a);
             tab.z = (h == 0) ? (float)ldexp((double)sumq, -E) : 0.0f;
-            tab.w = 0.0f;
+            tab.w = two ? 1.0f : 0.0f;
             *reinterpret_cast<float4*>(out + nt * kXTileBytes + kGroupsPerStage * kBfragBytesPerGroup +
                                        (G * 4 + t) * 16) = tab;
         }
@@ -188,8 +208,8 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t* __restrict__ 
                 k0 = 32 * t + 8 * j + 2 * q;
                 k1 = k0 + 1;
             } else {
-                k0 = 16 * t + 4 * j + q;
-                k1 = 16 * (t + 4) + 4 * j + q;
+                k0 = 32 * t + 4 * j + q;  // word 2t of the row's group, class q
+                k1 = k0 + 16;             // word 2t+1
             }
             b0 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k0][dg] << (8 * j);
             b1 |= (uint32_t)(uint8_t)dig[bb][g8 * 128 + k1][dg] << (8 * j);
@@ -243,11 +263,17 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
         if (lane == 0) {
             ptx::prefetch_tensormap(&tm_codes);
             ptx::prefetch_tensormap(&tm_scales);
+            // (row block, stage) of the next weight tile and stage of the next
+            // activation tile, advanced without divisions
+            int w_rb = (int)(it0 / S), w_st = (int)(it0 % S), x_st = w_st;
             auto issue_weights = [&](int it) {
                 const int slot = it % L::kStages;
                 uint8_t* sb = smem + slot * L::kStageBytes;
-                const int64_t item = it0 + it;
-                const int rb = (int)(item / S), st = (int)(item % S);
+                const int rb = w_rb, st = w_st;
+                if (++w_st == (int)S) {
+                    w_st = 0;
+                    ++w_rb;
+                }
                 ptx::mbar_arrive_expect_tx(&full[slot], L::kCodesBytes + L::kScalesBytes + L::kXBytes);
 #pragma unroll
                 for (int box = 0; box < Fmt<FMT>::kRowBytesPerStage / 128; ++box)
@@ -259,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
             auto issue_x = [&](int it) {
                 const int slot = it % L::kStages;
                 uint8_t* sb = smem + slot * L::kStageBytes;
-                const int st = (int)((it0 + it) % S);
+                const int st = x_st;
+                if (++x_st == (int)S) x_st = 0;
                 ptx::bulk_load(sb + L::kCodesBytes + L::kScalesBytes, p.xdata + (size_t)st * L::kXBytes,
                                L::kXBytes, &full[slot]);
             };
@@ -298,10 +325,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
         for (int nt = 0; nt < NT; ++nt) yacc[j][nt][0] = yacc[j][nt][1] = 0.0f;
 
     bool alive = true;
-    for (int it = 0; it < nit; ++it) {
+    // (row block, stage) of the current item, advanced without divisions
+    int rb = (int)(it0 / S), st = (int)(it0 % S);
+    const int Si = (int)S;
+    // lanes whose B-fragment columns hold batch rows that exist (at batch 1 the
+    // upper four columns are zero and are not read)
+    const bool b_live = g < 4 * (p.batch < 2 ? p.batch : 2);
+    for (int it = 0; it < nit; ++it, (++st == Si) ? (st = 0, ++rb) : 0) {
         const int slot = it % L::kStages;
-        const int64_t item = it0 + it;
-        const int rb = (int)(item / S), st = (int)(item % S);
         if (alive && !ptx::mbar_wait_bounded(&full[slot], (it / L::kStages) & 1, kWaitPolls)) {
             record_status(p.status, BQ_ERR_TIMEOUT);
             alive = false;
@@ -326,7 +357,9 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                     const uint8_t* xt = x_s + nt * kXTileBytes;
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
-                        bf[nt][h] = *reinterpret_cast<const uint4*>(xt + ((G * 2 + h) * 32 + lane) * 16);
+                        bf[nt][h] = (nt > 0 || b_live)
+                                        ? *reinterpret_cast<const uint4*>(xt + ((G * 2 + h) * 32 + lane) * 16)
+                                        : make_uint4(0u, 0u, 0u, 0u);
                     tab[nt] = *reinterpret_cast<const float4*>(xt + kGroupsPerStage * kBfragBytesPerGroup + (G * 4 + t) * 16);
                 }
                 int acc[NT][4];
@@ -347,19 +380,16 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                         }
                     }
                 } else {
+                    // words 2t, 2t+1 of the row's 32-byte group: one 8-byte load per row
                     const uint8_t* box = codes_s + (G >> 2) * (kRowsPerCta * 128);
-                    const int c0 = 2 * (G & 3), c1 = c0 + 1;
-                    const int offa = ((c0 ^ g) << 4) + 4 * t, offb = ((c1 ^ g) << 4) + 4 * t;
-                    const uint32_t w0a = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offa);
-                    const uint32_t w0b = *reinterpret_cast<const uint32_t*>(box + r0 * 128 + offb);
-                    const uint32_t w1a = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offa);
-                    const uint32_t w1b = *reinterpret_cast<const uint32_t*>(box + (r0 + 8) * 128 + offb);
+                    const int chunk = 2 * (G & 3) + (t >> 1);
+                    const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
+                    const uint2 wr0 = *reinterpret_cast<const uint2*>(box + r0 * 128 + off);
+                    const uint2 wr1 = *reinterpret_cast<const uint2*>(box + (r0 + 8) * 128 + off);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint32_t a0 = (w0a >> (2 * q)) & 0x03030303u;
-                        const uint32_t a1 = (w1a >> (2 * q)) & 0x03030303u;
-                        const uint32_t a2 = (w0b >> (2 * q)) & 0x03030303u;
-                        const uint32_t a3 = (w1b >> (2 * q)) & 0x03030303u;
+                        const uint32_t m = 0x03030303u << (2 * q);
+                        const uint32_t a0 = wr0.x & m, a1 = wr1.x & m, a2 = wr0.y & m, a3 = wr1.y & m;
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
@@ -375,8 +405,14 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                     // D0 + 256 D1 is exact in int32 (|D| < 2^21)
                     const float v0 = (float)(acc[nt][0] + 256 * acc[nt][1]);
                     const float v1 = (float)(acc[nt][2] + 256 * acc[nt][3]);
-                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    float u0, u1;
+                    if (tab[nt].w == 0.0f) {  // uniform across the warp (one group)
+                        u0 = fmaf(v0, tab[nt].x, -tab[nt].z);
+                        u1 = fmaf(v1, tab[nt].x, -tab[nt].z);
+                    } else {
+                        u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                        u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    }
                     yacc[0][nt][0] = fmaf(s0, u0, yacc[0][nt][0]);
                     yacc[0][nt][1] = fmaf(s1, u1, yacc[0][nt][1]);
                 }

@@ -61,6 +61,21 @@ int64_t gemv_tc_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                            const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s);
 
+// Row-owning decode GEMV (binary and 2-bit ternary, batch <= 4, K % 1024 == 0,
+// activation operand resident in shared memory): no workspace.
+bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch);
+cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                             const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
+
+// GEMV path choice shared by bq_gemv, bq_gemm (T <= 4) and bq_gemv_noalloc:
+// the row-owning kernel where eligible, else the split-K tensor-core kernel
+// (needs the workspace gemv_workspace_bytes reports), else the CUDA-core one.
+enum class GemvPath { Rows, SplitK, Simt };
+GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch);
+int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
+cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                        const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s);
+
 // tcgen05 prefill GEMM (all formats, K % 128 == 0).
 bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t);
 int64_t gemm_tc_workspace_bytes(int64_t n, int64_t k, int64_t t);

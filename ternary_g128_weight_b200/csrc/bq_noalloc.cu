@@ -64,16 +64,14 @@ extern "C" bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16
         const size_t bytes = (size_t)batch * n * (y_dtype == BQ_F32 ? 4 : 2);
         return cudaMemsetAsync(y, 0, bytes, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     }
-    const int64_t need = gemv_tc_workspace_bytes(fmt, n, k, batch);
-    cudaError_t e;
+    // same path choice as bq_gemv; only the split-K kernel needs scratch
+    const int64_t need = gemv_workspace_bytes(fmt, n, k, batch);
+    uint8_t* scratch = nullptr;
     if (need > 0) {
         if (need > (int64_t)BQ_NOALLOC_SCRATCH_BYTES) return BQ_ERR_WORKSPACE;
-        uint8_t* scratch = nullptr;
         const bq_status st = noalloc_scratch(&scratch);
         if (st != BQ_OK) return st;
-        e = launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, scratch, s);
-    } else {
-        e = launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
     }
+    const cudaError_t e = launch_gemv(fmt, codes, scales, n, k, x, batch, y, y_dtype, scratch, s);
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

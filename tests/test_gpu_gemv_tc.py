@@ -1,7 +1,9 @@
-"""The tensor-core decode GEMV (binary and 2-bit ternary, batch 1..4,
-K % 1024 == 0) against the oracle: ragged row counts, split-K row blocks,
-every batch size it takes, activations whose magnitudes span the BF16 range,
-and the check that eligible shapes really take that path."""
+"""The tensor-core decode GEMVs (binary and 2-bit ternary, batch 1..4,
+K % 1024 == 0) against the oracle: the row-owning kernel (no workspace) and
+the split-K kernel it falls back to when the activation operand does not fit
+in shared memory; ragged row counts, every chunk size of the row-owning
+kernel, every batch size, activations whose magnitudes span the BF16 range,
+and the check that shapes take the path they should."""
 import numpy as np
 import pytest
 
@@ -15,9 +17,13 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
-def test_eligible_shapes_use_workspace(fmt):
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 1) > 0
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 4) > 0
+def test_path_workspace(fmt):
+    # row-owning kernel: no workspace
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 1) == 0
+    assert bq.bq_gemv_workspace_bytes(fmt, 151936, 4096, 4) == 0
+    # batch 4 at K = 17408: the activation operand exceeds shared memory -> split-K (workspace)
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 17408, 4) > 0
+    # CUDA-core kernel: no workspace
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) == 0   # K % 1024 != 0
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 5) == 0   # batch > 4
     assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) == 0
@@ -25,7 +31,8 @@ def test_eligible_shapes_use_workspace(fmt):
 
 @pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
 @pytest.mark.parametrize("batch", [1, 2, 3, 4])
-@pytest.mark.parametrize("n,k", [(777, 4096), (1, 1024), (128, 2048), (129, 3072), (5000, 1024), (96, 12288)])
+@pytest.mark.parametrize("n,k", [(777, 4096), (1, 1024), (128, 2048), (129, 3072), (5000, 1024), (96, 12288),
+                                 (12000, 2048), (20000, 1024), (96, 17408)])
 def test_tc_parity(fmt, batch, n, k):
     codes, scales = host_weights(fmt, n, k, synth.SEED_BASE + 200 + n + batch)
     x = synth.x_bf16(synth.rng(n + 3 * batch + k), batch, k)
