@@ -19,10 +19,13 @@
 //
 // CTA (one per SM): 16 compute warps and one producer warp.
 //   * The producer streams the CTA's weights -- per (chunk of up to 8 row
-//     tiles of 16 rows, stage of 1024 K) one TMA box of codes (128-byte
-//     swizzle) and one of scales per row tile -- into a ring of shared-memory
-//     slots, starting before the wait on the previous kernel in the stream
-//     (programmatic dependent launch): the weights do not depend on it.
+//     tiles of 16 rows, stage of 1024 K) TMA boxes of codes (128-byte
+//     swizzle) and scales -- into a ring of shared-memory slots, starting
+//     before the wait on the previous kernel in the stream (programmatic
+//     dependent launch): the weights do not depend on it.  A full chunk is
+//     one 128-row box per 128-byte column (one TMA instruction per 16 KB:
+//     with one box per 16-row tile the TMA issue, not HBM, limited the
+//     stream to ~43% of the HBM bandwidth); a partial chunk uses 16-row boxes.
 //   * After that wait the compute warps turn x into the MMA B fragments and
 //     the per-group recombination table for all of K, once per CTA, into
 //     shared memory.
@@ -62,8 +65,12 @@ struct Fmt<BQ_T2G128> {
     static constexpr int kCoefShift = 0;     // sum(c * x) - sum(x)
     static constexpr int kQuantShift = 6;    // Q multiple of 2^6
 };
+// Slot layout: codes [column box b][row tile i][16 rows][128 B] (so that a
+// 128-row box of column b lands on all 8 row tiles at once), then scales
+// [row tile i][16 rows][8 groups] FP16.
 template <int FMT>
 constexpr int tile_code_bytes() { return Fmt<FMT>::kBoxes * 16 * 128; }
+constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
 template <int FMT>
 constexpr int slot_bytes() { return kMaxChunkTiles * (tile_code_bytes<FMT>() + kTileScaleBytes); }
 
@@ -235,7 +242,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
             continue;
         }
         const uint8_t* sb = smem + slot * slot_bytes<FMT>();
-        const uint8_t* codes_t = sb + my_rt * TCB;
+        const uint8_t* codes_t = sb + my_rt * 2048;  // column box 0 of this row tile
         const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + kMaxChunkTiles * TCB + my_rt * kTileScaleBytes);
         const uint8_t* xs = xres + (size_t)st * NT * X_NT;
 #pragma unroll
@@ -270,7 +277,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                 }
             } else {
                 // words 2t, 2t+1 of the row's 32-byte group
-                const uint8_t* box = codes_t + (G >> 2) * 2048;
+                const uint8_t* box = codes_t + (G >> 2) * kBoxColumnBytes;
                 const int chunk = 2 * (G & 3) + (t >> 1);
                 const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
                 const uint2 wr0 = *reinterpret_cast<const uint2*>(box + g * 128 + off);
@@ -351,10 +358,14 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
 }
 
 // ------------------------------------------------------------ kernel
+// Tensor maps: codes and scales with 16-row boxes (partial chunks) and
+// 128-row boxes (full chunks).
+struct Maps {
+    CUtensorMap codes16, scales16, codes128, scales128;
+};
+
 template <int FMT, int NT, int LANES>
-__global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_constant__ CUtensorMap tm_codes,
-                                                                const __grid_constant__ CUtensorMap tm_scales,
-                                                                const Params p) {
+__global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_constant__ Maps tm, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
@@ -376,8 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     if (warp == kProducerWarp) {
         // ------------------------------------------------ weight producer
         if (lane == 0) {
-            ptx::prefetch_tensormap(&tm_codes);
-            ptx::prefetch_tensormap(&tm_scales);
+            ptx::prefetch_tensormap(&tm.codes16);
+            ptx::prefetch_tensormap(&tm.scales16);
+            ptx::prefetch_tensormap(&tm.codes128);
+            ptx::prefetch_tensormap(&tm.scales128);
             constexpr int TCB = tile_code_bytes<FMT>();
             int it = 0;
             bool alive = true;
@@ -393,13 +406,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                     }
                     uint8_t* sb = smem + slot * slot_bytes<FMT>();
                     ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
-                    for (int i = 0; i < ct; ++i) {
+                    if (ct == kMaxChunkTiles) {
 #pragma unroll
                         for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
-                            ptx::tma_load_2d(sb + i * TCB + b * 2048, &tm_codes,
-                                             st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + i) * 16, &full[slot]);
-                        ptx::tma_load_2d(sb + kMaxChunkTiles * TCB + i * kTileScaleBytes, &tm_scales,
-                                         st * kGroupsPerStage, (r + i) * 16, &full[slot]);
+                            ptx::tma_load_2d(sb + b * kBoxColumnBytes, &tm.codes128,
+                                             st * (Fmt<FMT>::kBoxes * 128) + b * 128, r * 16, &full[slot]);
+                        ptx::tma_load_2d(sb + kMaxChunkTiles * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
+                                         &full[slot]);
+                    } else {
+                        for (int i = 0; i < ct; ++i) {
+#pragma unroll
+                            for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
+                                ptx::tma_load_2d(sb + b * kBoxColumnBytes + i * 2048, &tm.codes16,
+                                                 st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + i) * 16, &full[slot]);
+                            ptx::tma_load_2d(sb + kMaxChunkTiles * TCB + i * kTileScaleBytes, &tm.scales16,
+                                             st * kGroupsPerStage, (r + i) * 16, &full[slot]);
+                        }
                     }
                 }
                 r += ct;
@@ -514,26 +536,30 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     }
     const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : k / 4;
     const int64_t G = k / 128;
-    CUtensorMap tm_codes, tm_scales;
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n};
-        cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-        cuuint32_t box[2] = {128, 16};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
-    {
-        cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)n};
-        cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
-        cuuint32_t box[2] = {(cuuint32_t)kGroupsPerStage, 16};
-        cuuint32_t es[2] = {1, 1};
-        if (enc(&tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales), dims, strides, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
+    Maps tm;
+    for (int v = 0; v < 2; ++v) {
+        const cuuint32_t rows = v == 0 ? 16u : 128u;
+        {
+            cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n};
+            cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+            cuuint32_t box[2] = {128, rows};
+            cuuint32_t es[2] = {1, 1};
+            if (enc(v == 0 ? &tm.codes16 : &tm.codes128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes),
+                    dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        {
+            cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)n};
+            cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
+            cuuint32_t box[2] = {(cuuint32_t)kGroupsPerStage, rows};
+            cuuint32_t es[2] = {1, 1};
+            if (enc(v == 0 ? &tm.scales16 : &tm.scales128, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                    const_cast<uint16_t*>(scales), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
     }
     Params prm;
     prm.x = x;
@@ -560,7 +586,7 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     cfg.stream = s;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<FMT, NT, LANES>, tm_codes, tm_scales, prm);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<FMT, NT, LANES>, tm, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
