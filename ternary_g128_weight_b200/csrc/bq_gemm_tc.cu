@@ -277,7 +277,7 @@ template <int FMT>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = ptx::align_smem<1024>(smem_raw);
     uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
     uint64_t* full_b = full_a + kStages;
     uint64_t* empty = full_b + kStages;

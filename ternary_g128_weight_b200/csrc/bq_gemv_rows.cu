@@ -367,7 +367,7 @@ struct Maps {
 template <int FMT, int NT, int LANES>
 __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_constant__ Maps tm, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = ptx::align_smem<1024>(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
     uint64_t* empty = full + kMaxSlots;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
                                                               const Params p) {
     using L = Layout<FMT, NT>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = ptx::align_smem<1024>(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kStages * L::kStageBytes);
     uint64_t* empty = full + L::kStages;
     __shared__ int s_last;

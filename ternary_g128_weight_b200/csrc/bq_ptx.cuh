@@ -11,6 +11,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory base rounded up to ALIGN bytes.  Derived by
+// pointer arithmetic from the shared array, so that the compiler keeps the
+// accesses through it in the shared state space (a round trip through an
+// integer would turn them into generic loads and stores).
+template <int ALIGN>
+__device__ __forceinline__ uint8_t* align_smem(uint8_t* raw) {
+    const uint32_t a = smem_u32(raw);
+    return raw + ((ALIGN - (a & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
