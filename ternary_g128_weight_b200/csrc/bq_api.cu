@@ -82,11 +82,16 @@ namespace bq {
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
     if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
     if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
+    if (gemm_tc_eligible(fmt, n, k, batch)) return GemvPath::Gemm;
     return GemvPath::Simt;
 }
 
 int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
-    return gemv_path(fmt, n, k, batch) == GemvPath::SplitK ? gemv_tc_workspace_bytes(fmt, n, k, batch) : 0;
+    switch (gemv_path(fmt, n, k, batch)) {
+        case GemvPath::SplitK: return gemv_tc_workspace_bytes(fmt, n, k, batch);
+        case GemvPath::Gemm: return gemm_tc_workspace_bytes(n, k, batch);
+        default: return 0;
+    }
 }
 
 cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -94,6 +99,7 @@ cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, i
     switch (gemv_path(fmt, n, k, batch)) {
         case GemvPath::Rows: return launch_gemv_rows(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
         case GemvPath::SplitK: return launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
+        case GemvPath::Gemm: return launch_gemm_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
         default: return launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
     }
 }
@@ -166,7 +172,9 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
 // run the tcgen05 GEMM; shapes neither takes run the CUDA-core GEMV in chunks
 // of 16.
 static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
-    return t <= 4 && gemv_path(fmt, n, k, (int)t) != GemvPath::Simt;
+    if (t > 4) return false;
+    const GemvPath p = gemv_path(fmt, n, k, (int)t);
+    return p == GemvPath::Rows || p == GemvPath::SplitK;
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
@@ -196,7 +204,7 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     if (gemm_uses_gemv(fmt, n, k, t)) {
         e = launch_gemv(fmt, codes, scales, n, k, x, (int)t, y, BQ_BF16, workspace, s);
     } else if (gemm_tc_eligible(fmt, n, k, t)) {
-        e = launch_gemm_tc(fmt, codes, scales, n, k, x, t, y, workspace, s);
+        e = launch_gemm_tc(fmt, codes, scales, n, k, x, t, y, BQ_BF16, workspace, s);
     } else {
         for (int64_t t0 = 0; t0 < t && e == cudaSuccess; t0 += BQ_MAX_BATCH) {
             const int b = (int)((t - t0) < BQ_MAX_BATCH ? (t - t0) : BQ_MAX_BATCH);

@@ -61,7 +61,8 @@ struct Params {
     const uint8_t* codes;
     const uint16_t* scales;
     const float* inv_scale;  // [T] 2^-e_t
-    uint16_t* y;             // [T][N] BF16 (splits == 1)
+    void* y;                 // [T][N] BF16 or FP32 (splits == 1)
+    int y_f32;               // output type: FP32 (1) or BF16 (0)
     float* partial;          // [splits][T][N] FP32 sums without the 2^-e_t factor (splits > 1)
     int64_t n, k, t;
     int64_t units;           // row tiles x token tiles x splits
@@ -464,9 +465,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int64_t tok = t0 + j;
-                            if (tok < p.t)
-                                p.y[tok * p.n + row] =
-                                    float_to_bf16_bits(__uint_as_float(v[j]) * __ldg(p.inv_scale + tok));
+                            if (tok < p.t) {
+                                const float yv = __uint_as_float(v[j]) * __ldg(p.inv_scale + tok);
+                                if (p.y_f32)
+                                    static_cast<float*>(p.y)[tok * p.n + row] = yv;
+                                else
+                                    static_cast<uint16_t*>(p.y)[tok * p.n + row] = float_to_bf16_bits(yv);
+                            }
                         }
                     } else {
 #pragma unroll
@@ -490,16 +495,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
 }
 
-// Sum of the split partial tiles in split order, times 2^-e_t, rounded to BF16.
+// Sum of the split partial tiles in split order, times 2^-e_t, as BF16 or FP32.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restrict__ partial, int splits,
-                                                            const float* __restrict__ inv_scale,
-                                                            uint16_t* __restrict__ y, int64_t t, int64_t n) {
+                                                            const float* __restrict__ inv_scale, void* __restrict__ y,
+                                                            int y_f32, int64_t t, int64_t n) {
     ptx::pdl_wait();
     const int64_t total = t * n;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         float acc = 0.0f;
         for (int s = 0; s < splits; ++s) acc += partial[s * total + i];
-        y[i] = float_to_bf16_bits(acc * inv_scale[i / n]);
+        const float yv = acc * inv_scale[i / n];
+        if (y_f32)
+            static_cast<float*>(y)[i] = yv;
+        else
+            static_cast<uint16_t*>(y)[i] = float_to_bf16_bits(yv);
     }
 }
 
@@ -605,7 +614,7 @@ cudaError_t launch_typed(Params prm, const Plan& pl, const uint16_t* x, uint16_t
         cfg.blockDim = dim3(256);
         cfg.dynamicSmemBytes = 0;
         e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, (const float*)prm.partial, pl.splits,
-                               (const float*)inv_scale, prm.y, prm.t, prm.n);
+                               (const float*)inv_scale, prm.y, prm.y_f32, prm.t, prm.n);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
@@ -631,7 +640,7 @@ bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t) {
 }
 
 cudaError_t launch_gemm_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
-                           const uint16_t* x, int64_t t, uint16_t* y, void* workspace, cudaStream_t s) {
+                           const uint16_t* x, int64_t t, void* y, int y_dtype, void* workspace, cudaStream_t s) {
     const gemm::Plan pl = gemm::plan_of(n, k, t);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint16_t* xh = reinterpret_cast<uint16_t*>(ws);
@@ -642,6 +651,7 @@ cudaError_t launch_gemm_tc(int fmt, const uint8_t* codes, const uint16_t* scales
     prm.scales = scales;
     prm.inv_scale = inv;
     prm.y = y;
+    prm.y_f32 = y_dtype == BQ_F32 ? 1 : 0;
     prm.partial = pl.splits > 1 ? part : nullptr;
     prm.n = n;
     prm.k = k;

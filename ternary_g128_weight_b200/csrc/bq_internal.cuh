@@ -68,9 +68,10 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
 
 // GEMV path choice shared by bq_gemv, bq_gemm (T <= 4) and bq_gemv_noalloc:
-// the row-owning kernel where eligible, else the split-K tensor-core kernel
-// (needs the workspace gemv_workspace_bytes reports), else the CUDA-core one.
-enum class GemvPath { Rows, SplitK, Simt };
+// the row-owning kernel where eligible, else the split-K tensor-core kernel,
+// else the tcgen05 GEMM with T = batch (5-trit format, batch 5..16), else the
+// CUDA-core kernel.  gemv_workspace_bytes reports the workspace of the choice.
+enum class GemvPath { Rows, SplitK, Gemm, Simt };
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch);
 int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -80,6 +81,6 @@ cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, i
 bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t);
 int64_t gemm_tc_workspace_bytes(int64_t n, int64_t k, int64_t t);
 cudaError_t launch_gemm_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
-                           const uint16_t* x, int64_t t, uint16_t* y, void* workspace, cudaStream_t s);
+                           const uint16_t* x, int64_t t, void* y, int y_dtype, void* workspace, cudaStream_t s);
 
 }  // namespace bq

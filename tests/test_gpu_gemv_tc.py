@@ -23,10 +23,10 @@ def test_path_workspace(fmt):
     assert bq.bq_gemv_workspace_bytes(fmt, 151936, 4096, 4) == 0
     # batch 4 at K = 17408: the activation operand exceeds shared memory -> split-K (workspace)
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 17408, 4) > 0
-    # CUDA-core kernel: no workspace
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) == 0   # K % 1024 != 0
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 5) == 0   # batch > 4
-    assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) == 0
+    # tcgen05 GEMM with T = batch: workspace for the FP16 activations
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) >= 1152 * 2   # K % 1024 != 0
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 5) >= 5 * 4096 * 2   # batch > 4
+    assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) >= 4096 * 2
 
 
 @pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
