@@ -42,31 +42,47 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--fmt", choices=list(FMT_NAMES), default="q1g128")
     p.add_argument("--batch", type=int, default=1)
-    p.add_argument("--layers", type=int, default=36)
+    p.add_argument("--model", choices=["qwen3-8b", "27b"], default="qwen3-8b",
+                   help="layer shapes: Qwen3-8B (36 blocks, head 151936x4096) or the 27B class "
+                        "(64 blocks, head 248320x5120)")
+    p.add_argument("--layers", type=int, default=None, help="blocks per pass (default: the model's)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM leg")
+    p.add_argument("--gemm-only", action="store_true",
+                   help="run only the prefill GEMM leg (a diagnostic line, e.g. for a profiler)")
     return p.parse_args()
 
 
-def step_shapes(layers):
-    """One decode weight pass: per layer q|k|v (one launch, rows concatenated),
-    o, gate|up (one launch), down; then the LM head."""
+def model_shapes(model):
     import synth
-    L = synth.QWEN3_8B_LAYER
+    if model == "27b":
+        return synth.CLASS27B_LAYER, synth.CLASS27B_LM_HEAD, synth.CLASS27B_BLOCKS
+    return synth.QWEN3_8B_LAYER, synth.QWEN3_8B_LM_HEAD, synth.QWEN3_8B_BLOCKS
+
+
+def step_shapes(model, layers):
+    """One decode weight pass: per layer q|k|v (one launch, rows concatenated:
+    the three share x), o, gate|up (one launch), down; then the LM head."""
+    L, head, _ = model_shapes(model)
     qkv = (L["q"][0] + L["k"][0] + L["v"][0], L["q"][1])
     gate_up = (L["gate"][0] + L["up"][0], L["gate"][1])
     shapes = []
     for layer in range(layers):
         shapes += [(f"L{layer}.qkv",) + qkv, (f"L{layer}.o",) + L["o"],
                    (f"L{layer}.gate_up",) + gate_up, (f"L{layer}.down",) + L["down"]]
-    shapes.append(("lm_head",) + synth.QWEN3_8B_LM_HEAD)
+    shapes.append(("lm_head",) + head)
     return shapes
 
 
-def workload_name(fmt, batch, layers):
-    return (f"qwen3-8b-shapes {fmt} GEMV batch {batch}: {layers} x (q|k|v 6144x4096 [q 4096, k 1024, "
-            f"v 1024 rows], o 4096x4096, gate|up 24576x4096 [2 x 12288 rows], down 4096x12288) + LM head "
-            f"151936x4096, distinct weights per layer, one CUDA graph per step")
+def workload_name(model, fmt, batch, layers):
+    L, head, _ = model_shapes(model)
+    qkv = L["q"][0] + L["k"][0] + L["v"][0]
+    return (f"{model}-shapes {fmt} GEMV batch {batch}: {layers} x (q|k|v {qkv}x{L['q'][1]} "
+            f"[q {L['q'][0]}, k {L['k'][0]}, v {L['v'][0]} rows], o {L['o'][0]}x{L['o'][1]}, "
+            f"gate|up {2 * L['gate'][0]}x{L['gate'][1]} [2 x {L['gate'][0]} rows], "
+            f"down {L['down'][0]}x{L['down'][1]}) + LM head {head[0]}x{head[1]}, distinct weights per layer, "
+            f"one CUDA graph per step")
 
 
 # --------------------------------------------------------------------- clocks
@@ -131,6 +147,97 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("bq_gemv_rows.cu", "bq_gemv_tc.cu", "bq_gemm_tc.cu", "bq_ptx.cuh", "bq_api.cu")
+
+
+def kernel_source_hash():
+    """Identifies the kernel sources a recorded profiler capture belongs to."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "ternary_g128_weight_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(model, fmt, batch, layers):
+    """DRAM bytes per step from profiles/ncu_traffic.json when it was taken on
+    this workload with the current kernel sources, else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rows = json.load(fh)
+    for tr in rows if isinstance(rows, list) else [rows]:
+        if (tr.get("model"), tr.get("fmt"), tr.get("batch"), tr.get("layers"), tr.get("kernel_src")) == \
+                (model, fmt, batch, layers, kernel_source_hash()):
+            return tr.get("dram_bytes_per_step")
+    return None
+
+
+def measured_tensor_peak():
+    """Dense 16-bit tensor peak (TFLOP/s) for a kernel timed alone: the measured
+    burst cuBLAS BF16 figure (FP16 runs at the same nominal rate)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------- prefill GEMM
+GEMM_SHAPES = [(17408, 5120), (5120, 17408)]
+GEMM_TOKENS = 4096
+
+
+def gemm_leg(fmt, dev, reps):
+    """Prefill GEMM Y = X W^T at T = 4096 on the pages' two prefill shapes
+    (tensor-bound); each launch timed alone with CUDA events, L2 flushed by a
+    256 MB write before every timed launch."""
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+    peak, src = measured_tensor_peak()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = []
+    for (n, k) in GEMM_SHAPES:
+        gen = synth.device_generator(synth.SEED_BASE + 4, device=dev)
+        if fmt == "q1g128":
+            codes, scales = bq.bq_pack(fmt, synth.device_weights_normal(gen, n, k, device=dev))
+        else:
+            t = synth.device_trits(gen, n, k, device=dev)
+            s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
+            w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
+            codes, scales = bq.bq_pack(fmt, w, scales_in=s)
+            del w
+        x = synth.device_x_bf16(gen, GEMM_TOKENS, k, device=dev)
+        y = torch.empty((GEMM_TOKENS, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(bq.bq_gemm_workspace_bytes(fmt, n, k, GEMM_TOKENS), 256), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        assert bq.bq_check() == bq.BQ_OK
+        ms = statistics.median(times)
+        tf = 2.0 * GEMM_TOKENS * n * k / (ms / 1000.0) / 1e12
+        out.append({"shape": f"{n}x{k}", "tokens": GEMM_TOKENS, "us": round(ms * 1000, 1),
+                    "tflops": round(tf, 1), "frac": round(tf / peak, 4),
+                    "launches": bq.bq_gemm_launches(fmt, n, k, GEMM_TOKENS)})
+        del codes, scales, x, y, ws
+    return {"bound": "tensor", "peak": peak, "unit": "TFLOP/s",
+            "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst; FP16 operands at the same rate)",
+            "kernel": "xprep_f16_kernel + gemm_tc_kernel (tcgen05 kind::f16, TMEM accumulators)",
+            "dtype": "f16 operands (exact s*q and pre-scaled x), f32 accumulate", "cases": out}
+
+
 # ------------------------------------------------------------------ reference
 def run_reference(args):
     """The CPU oracle as it stands, on a bounded sample of the workload."""
@@ -168,7 +275,7 @@ def run_reference(args):
         "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_name(fmt, args.batch, args.layers), "fmt": fmt,
+        "config": {"workload": workload_name(args.model, fmt, args.batch, args.layers), "fmt": fmt,
                    "batch": args.batch, "sample": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.max_threads(),
                          "kind": "oracle", "sample": sample},
@@ -189,20 +296,25 @@ def cpu_baseline(fmt, mats, batch):
     for m in sample:
         host.append((m["n"], m["k"], m["codes"].cpu().numpy(), m["scales"].cpu().numpy().view(np.uint16),
                      m["x"].view(torch.int16).cpu().numpy().view(np.uint16)))
-    total_bytes, t0 = 0, time.perf_counter()
-    for (n, k, c, s, x) in host:
-        oracle.matmul(fmt, c, s, n, k, x)
-        total_bytes += c.nbytes + s.nbytes
+    # repeat the sample until about 10 s of host work is done (bounded: 200 passes)
+    total_bytes, passes, t0 = 0, 0, time.perf_counter()
+    while passes < 200 and (passes == 0 or time.perf_counter() - t0 < 10.0):
+        for (n, k, c, s, x) in host:
+            oracle.matmul(fmt, c, s, n, k, x)
+            total_bytes += c.nbytes + s.nbytes
+        passes += 1
     dt = time.perf_counter() - t0
     return {"value": round(total_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
             "kind": "oracle",
-            "sample": f"LM head 151936x4096 + one layer's q|k|v, o, gate|up, down ({fmt}, batch {batch}), "
+            "sample": f"LM head + one layer's q|k|v, o, gate|up, down ({fmt}, batch {batch}) x {passes} passes, "
                       f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s"}
 
 
 # ----------------------------------------------------------------------- ours
 def main():
     args = parse()
+    if args.layers is None:
+        args.layers = model_shapes(args.model)[2]
     if args.impl == "reference":
         return run_reference(args)
 
@@ -225,8 +337,13 @@ def main():
 
     fmt, batch = args.fmt, args.batch
     f = FMT_NAMES[fmt]
+    if args.gemm_only:
+        if rank == 0:
+            print(json.dumps({"metric": "prefill GEMM TFLOP/s", "fmt": fmt,
+                              "prefill_gemm": gemm_leg(fmt, dev, max(args.steps, 1))}), flush=True)
+        return 0
     gen = synth.device_generator(synth.SEED_BASE + 1 + 1000 * rank, device=dev)
-    shapes = step_shapes(args.layers)
+    shapes = step_shapes(args.model, args.layers)
 
     # ---- activations and outputs: one contiguous buffer each (one copy per step for e2e)
     def offsets(sizes):
@@ -260,7 +377,12 @@ def main():
     workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
     weight_bytes = sum(m["codes"].numel() + 2 * m["scales"].numel() for m in mats)
     algo_bytes = weight_bytes + sum(2 * m["k"] * batch + 2 * m["n"] * batch for m in mats)
-    launches_per_step = sum(2 if bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) > 0 else 1 for m in mats)
+    launches_per_step = sum(bq.bq_gemv_launches(f, m["n"], m["k"], batch) for m in mats)
+    # the arithmetic of the path bq_gemv takes for this format and batch
+    int8_path = fmt in ("q1g128", "t2g128") and batch <= 4
+    path_dtype = "s8xu8->s32 (warp MMA), f32 recombine" if int8_path else "f16 (tcgen05) -> f32"
+    path_kernel = ("gemv_rows_kernel (row-owning tensor-core GEMV)" if int8_path
+                   else "xprep_f16_kernel + gemm_tc_kernel (tcgen05 GEMM with T = batch)")
 
     def step():
         for m in mats:
@@ -361,17 +483,18 @@ def main():
     peak, peak_src = measured_peaks()
     value = weight_bytes * world / (ms_per_step / 1000.0) / 1e9
     achieved = algo_bytes / (ms_per_step / 1000.0) / 1e9
-    traffic = None
-    traffic_path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-    if os.path.exists(traffic_path):
-        with open(traffic_path) as fh:
-            tr = json.load(fh)
-        if tr.get("fmt") == fmt and tr.get("batch") == batch and tr.get("kernel_rev") == bq.bq_version():
-            traffic = tr.get("bytes_per_step")
+    traffic = recorded_traffic(args.model, fmt, batch, args.layers)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(fmt, mats, batch)
+    prefill = None
+    if rank == 0 and not args.no_gemm:
+        del graph, hg
+        graph = hg = None
+        mats.clear()
+        torch.cuda.empty_cache()
+        prefill = gemm_leg(fmt, dev, 5)
 
     if rank == 0:
         line = {
@@ -379,17 +502,17 @@ def main():
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
-            "config": {"workload": workload_name(fmt, batch, args.layers), "fmt": fmt, "batch": batch,
+            "dtype": path_dtype, "data": "synthetic",
+            "config": {"workload": workload_name(args.model, fmt, batch, args.layers), "fmt": fmt, "batch": batch,
                        "weight_bytes_per_step": weight_bytes, "gemv_calls_per_step": len(mats),
-                       "l2": "inputs larger than L2 (1.06 GB of weights per step at q1g128), no flush",
+                       "l2": f"inputs larger than L2 ({weight_bytes / 1e9:.2f} GB of weights per step, L2 126 MB), no flush",
                        "parallelism": f"replicas x{world}"},
             "hbm_roofline_pct": round(100.0 * value / world / peak, 2),
             "tokens_per_s_equiv": round(1000.0 / ms_per_step, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, burst copy)",
-                         "kernel": "bq GEMV (prep + decode kernels), every launch of a step back to back",
+                         "kernel": path_kernel + ", every launch of a step back to back",
                          "algorithmic_bytes_per_step": algo_bytes},
             "lm_head_launch": {"us": round(head_ms * 1000, 2), "bytes": head_bytes,
                                "GB_s": round(head_bytes / (head_ms / 1000.0) / 1e9, 2),
@@ -403,6 +526,8 @@ def main():
                            "d2h_bytes_per_step": e2e["d2h"]}
         if cpu:
             line["cpu_baseline"] = cpu
+        if prefill:
+            line["prefill_gemm"] = prefill
         print(json.dumps(line), flush=True)
 
     del graph, hg

@@ -112,6 +112,12 @@ bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* sca
  * -1 for an invalid format or shape. */
 int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 
+/* Number of kernels one bq_gemv (or bq_gemv_noalloc) call of this shape
+ * launches (0 for an empty shape); -1 for an invalid format or shape.  An
+ * introspection helper for callers that count launches (graph building,
+ * benchmarks); it launches nothing. */
+int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
+
 /* y[b][r] = sum_g s[r][g] * sum_{k in g} q[r][k] * x[b][k],   b < batch <= 16.
  * The weight-streaming decode product ("1-bit Bonsai 8B" section 2: token
  * generation is bound by streaming the weights; section 4.1: codes decoded
@@ -153,6 +159,10 @@ bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16_t* scales,
 /* ------------------------------------------------------------------- GEMM */
 /* Workspace bytes bq_gemm needs for T tokens (0 if none); -1 if invalid. */
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t);
+
+/* Number of kernels one bq_gemm call of this shape launches (0 for an empty
+ * shape); -1 if invalid.  Introspection only; launches nothing. */
+int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t);
 
 /* Prefill: Y[t][r] = sum_k X[t][k] * s[r][g(k)] q[r][k] for t < T, BF16 out
  * ("1-bit Bonsai 8B" summary section 3 and Table 3 pp512: prompt processing is

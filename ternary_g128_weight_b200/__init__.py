@@ -27,7 +27,8 @@ FORMATS = {"q1g128": BQ_Q1G128, "t2g128": BQ_T2G128, "t5p8": BQ_T5P8G128}
 EXPORTED = [
     "bq_codes_bytes", "bq_scales_bytes", "bq_effective_bits",
     "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8",
-    "bq_gemv_workspace_bytes", "bq_gemv", "bq_gemv_noalloc", "bq_gemm_workspace_bytes", "bq_gemm",
+    "bq_gemv_workspace_bytes", "bq_gemv_launches", "bq_gemv", "bq_gemv_noalloc",
+    "bq_gemm_workspace_bytes", "bq_gemm_launches", "bq_gemm",
     "bq_check", "bq_debug_wait_timeout", "bq_status_string", "bq_version",
 ]
 
@@ -58,9 +59,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         f.restype = i32
     L.bq_gemv_workspace_bytes.argtypes = [i32, i64, i64, i32]; L.bq_gemv_workspace_bytes.restype = i64
+    L.bq_gemv_launches.argtypes = [i32, i64, i64, i32]; L.bq_gemv_launches.restype = i32
     L.bq_gemv.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, i32, vp, sz, vp]; L.bq_gemv.restype = i32
     L.bq_gemv_noalloc.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, i32, vp]; L.bq_gemv_noalloc.restype = i32
     L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]; L.bq_gemm_workspace_bytes.restype = i64
+    L.bq_gemm_launches.argtypes = [i32, i64, i64, i64]; L.bq_gemm_launches.restype = i32
     L.bq_gemm.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]; L.bq_gemm.restype = i32
     L.bq_check.argtypes = [vp]; L.bq_check.restype = i32
     L.bq_debug_wait_timeout.argtypes = [i64, vp]; L.bq_debug_wait_timeout.restype = i32
@@ -152,6 +155,10 @@ def bq_gemv_workspace_bytes(fmt, n: int, k: int, batch: int) -> int:
     return int(load().bq_gemv_workspace_bytes(_fmt(fmt), n, k, batch))
 
 
+def bq_gemv_launches(fmt, n: int, k: int, batch: int) -> int:
+    return int(load().bq_gemv_launches(_fmt(fmt), n, k, batch))
+
+
 def bq_gemv(fmt, codes, scales, n: int, k: int, x, y=None, y_dtype: int = BQ_BF16,
             workspace=None, stream=None):
     """y[b][r] = sum_k s q x (see bq.h).  x: BF16 CUDA tensor [batch][K]."""
@@ -194,6 +201,10 @@ def bq_gemv_noalloc(fmt, codes, scales, n: int, k: int, x, y=None, y_dtype: int 
 # -------------------------------------------------------------------- GEMM
 def bq_gemm_workspace_bytes(fmt, n: int, k: int, t: int) -> int:
     return int(load().bq_gemm_workspace_bytes(_fmt(fmt), n, k, t))
+
+
+def bq_gemm_launches(fmt, n: int, k: int, t: int) -> int:
+    return int(load().bq_gemm_launches(_fmt(fmt), n, k, t))
 
 
 def bq_gemm(fmt, codes, scales, n: int, k: int, x, y=None, workspace=None, stream=None):

@@ -140,6 +140,18 @@ bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* sca
 }
 
 
+int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
+    if (n == 0) return 0;
+    if (k == 0) return 0;  // the output is cleared with a memset, no kernel
+    switch (gemv_path(fmt, n, k, batch)) {
+        case GemvPath::Rows: return 1;
+        case GemvPath::SplitK: return 2;  // activation prep + split-K kernel
+        case GemvPath::Gemm: return gemm_tc_launches(n, k, batch);
+        default: return 1;
+    }
+}
+
 int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
     if (n == 0 || k == 0) return 0;
@@ -183,6 +195,14 @@ int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
     if (gemm_uses_gemv(fmt, n, k, t)) return gemv_workspace_bytes(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_workspace_bytes(n, k, t);
     return 0;
+}
+
+int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
+    if (t == 0 || n == 0 || k == 0) return 0;
+    if (gemm_uses_gemv(fmt, n, k, t)) return bq_gemv_launches(fmt, n, k, (int)t);
+    if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_launches(n, k, t);
+    return (int)((t + BQ_MAX_BATCH - 1) / BQ_MAX_BATCH);
 }
 
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,

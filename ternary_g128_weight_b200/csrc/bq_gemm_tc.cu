@@ -632,6 +632,10 @@ int64_t gemm_tc_workspace_bytes(int64_t n, int64_t k, int64_t t) {
     return b;
 }
 
+// Kernels one call launches: activation prep, GEMM, and the split-K reduction
+// when K is split.
+int gemm_tc_launches(int64_t n, int64_t k, int64_t t) { return gemm::plan_of(n, k, t).splits > 1 ? 3 : 2; }
+
 bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t) {
     if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && n > 0 && k > 0 && k % 128 == 0 &&
           t > 0 && t <= (int64_t)INT32_MAX && n <= (int64_t)INT32_MAX && k / 64 <= (int64_t)(1 << 22)))

@@ -80,6 +80,7 @@ cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, i
 // tcgen05 prefill GEMM (all formats, K % 128 == 0).
 bool gemm_tc_eligible(int fmt, int64_t n, int64_t k, int64_t t);
 int64_t gemm_tc_workspace_bytes(int64_t n, int64_t k, int64_t t);
+int gemm_tc_launches(int64_t n, int64_t k, int64_t t);
 cudaError_t launch_gemm_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                            const uint16_t* x, int64_t t, void* y, int y_dtype, void* workspace, cudaStream_t s);
 

@@ -96,6 +96,17 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_gemv_workspace_bytes(1, 4, 100, 1) == -1
     assert lib.bq_gemv_workspace_bytes(1, 4, 128, 17) == -1
     assert lib.bq_gemv_workspace_bytes(1, 4096, 4096, 1) >= 0
+    # launch counts (host-side planning only)
+    assert lib.bq_gemv_launches(9, 4096, 4096, 1) == -1
+    assert lib.bq_gemv_launches(1, 4096, 100, 1) == -1
+    assert lib.bq_gemv_launches(1, 0, 4096, 1) == 0
+    assert lib.bq_gemv_launches(1, 4096, 4096, 1) == 1      # row-owning kernel
+    assert lib.bq_gemv_launches(2, 4096, 4096, 4) == 1
+    assert lib.bq_gemv_launches(3, 4096, 4096, 1) in (2, 3)  # 5-trit format: tcgen05 GEMM
+    assert lib.bq_gemv_launches(1, 4096, 4096, 16) in (2, 3)
+    assert lib.bq_gemm_launches(1, 17408, 5120, 4096) == 2     # prep + GEMM, no K split
+    assert lib.bq_gemm_launches(1, 4096, 4096, 1) == 1         # T <= 4: the GEMV
+    assert lib.bq_gemm_launches(1, 4096, 100, 8) == -1
     assert lib.bq_gemm_workspace_bytes(2, 4096, 4096, 512) >= 0
     assert lib.bq_debug_wait_timeout(-1, None) == bq.BQ_ERR_SHAPE
 
