@@ -120,10 +120,20 @@ __device__ __forceinline__ int ilog2f(float m) {
 //                 u = (D0 + 256 D1) 2^a 2^(e-a) - z.
 // Rows past the batch get zero entries with the group's flag (so that the
 // kernel's choice stays uniform across the warp).
-template <int FMT, int NT, int LANES>
-__device__ void prep_group(const Params& p, uint8_t* xst, int st, int G, int lane) {
-    constexpr int X_NT = x_nt_bytes(LANES);
+// This lane's 4 BF16 activations of group G of stage st for the batch rows of
+// the n-tiles (zero past the batch).
+template <int NT>
+__device__ __forceinline__ void load_group_x(const Params& p, int st, int G, int lane, uint2 (&raw)[2 * NT]) {
     const int64_t kbase = (int64_t)st * 1024 + G * 128;
+#pragma unroll
+    for (int bb = 0; bb < 2 * NT; ++bb)
+        raw[bb] = bb < p.batch ? __ldg(reinterpret_cast<const uint2*>(p.x + bb * p.k + kbase + lane * 4))
+                               : make_uint2(0u, 0u);
+}
+
+template <int FMT, int NT, int LANES>
+__device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const uint2 (&xraw)[2 * NT]) {
+    constexpr int X_NT = x_nt_bytes(LANES);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         uint8_t* xt = xst + nt * X_NT;
@@ -132,16 +142,11 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int st, int G, int lan
         bool two = false;
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
-            const int bb = 2 * nt + hb;
-            if (bb < p.batch) {
-                const uint2 raw = *reinterpret_cast<const uint2*>(p.x + bb * p.k + kbase + lane * 4);
-                xv[hb][0] = bf16_lo(raw.x);
-                xv[hb][1] = bf16_hi(raw.x);
-                xv[hb][2] = bf16_lo(raw.y);
-                xv[hb][3] = bf16_hi(raw.y);
-            } else {
-                xv[hb][0] = xv[hb][1] = xv[hb][2] = xv[hb][3] = 0.0f;
-            }
+            const uint2 raw = xraw[2 * nt + hb];
+            xv[hb][0] = bf16_lo(raw.x);
+            xv[hb][1] = bf16_hi(raw.x);
+            xv[hb][2] = bf16_lo(raw.y);
+            xv[hb][3] = bf16_hi(raw.y);
             float m = fmaxf(fmaxf(fabsf(xv[hb][0]), fabsf(xv[hb][1])), fmaxf(fabsf(xv[hb][2]), fabsf(xv[hb][3])));
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -437,10 +442,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     // ---------------------------------------------------- compute warps
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
     {
+        // items (stage, group) i = warp + 16 j; the x loads of up to kPrepBatch
+        // items are issued before any of them is processed
+        constexpr int kPrepBatch = 4;
         uint8_t* xres = smem + p.x_off;
-        for (int i = warp; i < p.stages * kGroupsPerStage; i += kComputeWarps) {
-            const int st = i / kGroupsPerStage, G = i % kGroupsPerStage;
-            prep_group<FMT, NT, LANES>(p, xres + (size_t)st * NT * x_nt_bytes(LANES), st, G, lane);
+        const int items = p.stages * kGroupsPerStage;
+        for (int i0 = warp; i0 < items; i0 += kComputeWarps * kPrepBatch) {
+            uint2 raw[kPrepBatch][2 * NT];
+#pragma unroll
+            for (int j = 0; j < kPrepBatch; ++j) {
+                const int i = i0 + j * kComputeWarps;
+                if (i < items) load_group_x<NT>(p, i / kGroupsPerStage, i % kGroupsPerStage, lane, raw[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < kPrepBatch; ++j) {
+                const int i = i0 + j * kComputeWarps;
+                if (i < items)
+                    prep_group<FMT, NT, LANES>(p, xres + (size_t)(i / kGroupsPerStage) * NT * x_nt_bytes(LANES),
+                                               i % kGroupsPerStage, lane, raw[j]);
+            }
         }
     }
     bar_compute();
