@@ -379,7 +379,7 @@ def main():
     algo_bytes = weight_bytes + sum(2 * m["k"] * batch + 2 * m["n"] * batch for m in mats)
     launches_per_step = sum(bq.bq_gemv_launches(f, m["n"], m["k"], batch) for m in mats)
     # the arithmetic of the path bq_gemv takes for this format and batch
-    int8_path = fmt in ("q1g128", "t2g128") and batch <= 4
+    int8_path = batch <= 4 and all(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) == 0 for m in mats)
     path_dtype = "s8xu8->s32 (warp MMA), f32 recombine" if int8_path else "f16 (tcgen05) -> f32"
     path_kernel = ("gemv_rows_kernel (row-owning tensor-core GEMV)" if int8_path
                    else "xprep_f16_kernel + gemm_tc_kernel (tcgen05 GEMM with T = batch)")

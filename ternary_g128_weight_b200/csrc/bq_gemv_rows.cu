@@ -1,12 +1,16 @@
 // Decode GEMV, one launch per call: each CTA owns a contiguous range of whole
 // weight rows and reduces over all of K itself, so there is no workspace, no
-// preparation kernel and no cross-CTA reduction (binary g128 and 2-bit-slot
-// ternary g128, batch 1..4, K % 1024 == 0).
+// preparation kernel and no cross-CTA reduction (binary g128, 2-bit-slot and
+// 5-trits-per-byte ternary g128, batch 1..4, K % 1024 == 0).
 //
 // Arithmetic (as in the split-K tensor-core GEMV): the codes are expanded with
 // one LOP3 per four weights into int8 operands of the warp MMA m16n8k32,
 //   binary : byte j of (w & (0x01010101 << p)) = 2^p * bit(8j+p),
 //   2-bit  : byte j of (w & (0x03030303 << 2i)) = 4^i * c(4j+i), c = q+1,
+//   5-trit : a byte v = sum c_i 3^i ("把 27B 模型压到 4GB" section 2.4: 3^5 <= 256)
+//            gives c0..c3 as the four bytes of a 256-entry table word (one
+//            copy per lane in shared memory, so lookups never conflict) and
+//            c4 = (810 v) >> 16 (exact for v < 243),
 // against activations in per-(batch row, group) fixed point Q (largest |x| of
 // the group mapped into [2^29, 2^30), Q a multiple of 2^7 resp. 2^6), split
 // into four signed base-256 digits, one MMA column each; the k-slot of class
@@ -65,11 +69,20 @@ struct Fmt<BQ_T2G128> {
     static constexpr int kCoefShift = 0;     // sum(c * x) - sum(x)
     static constexpr int kQuantShift = 6;    // Q multiple of 2^6
 };
+template <>
+struct Fmt<BQ_T5P8G128> {
+    static constexpr int kBoxes = 1;         // one unswizzled 208-byte column (8 groups x 26 bytes)
+    static constexpr int kCoefShift = 0;     // sum(c * x) - sum(x)
+    static constexpr int kQuantShift = 0;    // plain bytes c, operand Q
+};
+constexpr int kT5RowBytes = kGroupsPerStage * 26;  // 208
+constexpr int kLutBytes = 256 * 32 * 4;           // byte -> c0..c3, one copy per lane
 // Slot layout: codes [column box b][row tile i][16 rows][128 B] (so that a
-// 128-row box of column b lands on all 8 row tiles at once), then scales
-// [row tile i][16 rows][8 groups] FP16.
+// 128-row box of column b lands on all 8 row tiles at once; 5-trit format:
+// [row tile i][16 rows][208 B]), then scales [row tile i][16 rows][8 groups]
+// FP16.
 template <int FMT>
-constexpr int tile_code_bytes() { return Fmt<FMT>::kBoxes * 16 * 128; }
+constexpr int tile_code_bytes() { return FMT == BQ_T5P8G128 ? 16 * kT5RowBytes : Fmt<FMT>::kBoxes * 16 * 128; }
 constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
 template <int FMT>
 constexpr int slot_bytes() { return kMaxChunkTiles * (tile_code_bytes<FMT>() + kTileScaleBytes); }
@@ -82,7 +95,7 @@ struct Params {
     int stages;         // K / 1024
     int row_tiles;      // ceil(N / 16)
     int slots;          // ring slots
-    uint32_t x_off, red_off, bar_off;  // shared-memory offsets
+    uint32_t x_off, red_off, lut_off, bar_off;  // shared-memory offsets
     int* status;
 };
 
@@ -113,6 +126,10 @@ __device__ __forceinline__ int ilog2f(float m) {
 // where (t, q, h, j) is the k-slot the A decode gives weight k:
 //   binary: k = 32t + 8j + 2q + h   (word t of the row's group, class 2q+h)
 //   2-bit : k = 32t + 16h + 4j + q  (word 2t+h of the row's group, class q)
+//   5-trit: A register i = 2q + h of thread t holds, for i < 6, digits 0..3
+//           of byte 6t+i; i = 6 digit 4 of bytes 6t..6t+3; i = 7 digit 4 of
+//           bytes 6t+4, 6t+5 and trits 120+2t, 121+2t (the group's last
+//           eight trits, in bytes 24 and 25)
 // Table entry (G, t) of an n-tile, t = 2 (bb & 1) + hh for digit pair hh, with
 // e = coef - E + 16 hh and z = [hh == 0] 2^-E sum Q:
 //   one factor  : {2^e, 1, z, 0}, u = (D0 + 256 D1) 2^e - z;
@@ -179,9 +196,23 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const
                 if (FMT == BQ_Q1G128) {
                     b = Q >> (kk & 7);  // exact: Q is a multiple of 2^7
                     t = kk >> 5; j = (kk >> 3) & 3; q = (kk >> 1) & 3; h = kk & 1;
-                } else {
+                } else if (FMT == BQ_T2G128) {
                     b = Q >> (2 * (kk & 3));  // exact: Q is a multiple of 2^6
                     t = kk >> 5; h = (kk >> 4) & 1; j = (kk >> 2) & 3; q = kk & 3;
+                } else {
+                    b = Q;
+                    int ri;  // A register of the thread
+                    if (kk < 120) {
+                        const int byte = kk / 5, d = kk - 5 * byte, ib = byte % 6;
+                        t = byte / 6;
+                        if (d < 4) { ri = ib; j = d; }
+                        else if (ib < 4) { ri = 6; j = ib; }
+                        else { ri = 7; j = ib - 4; }
+                    } else {
+                        const int e = kk - 120;
+                        t = e >> 1; ri = 7; j = 2 + (e & 1);
+                    }
+                    q = ri >> 1; h = ri & 1;
                 }
                 const int boff = (q & 1) * 8 + h * 4 + j;
                 int rem = b;
@@ -211,6 +242,32 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const
     }
 }
 
+// ------------------------------------------------------------ 5-trit decode
+// The 8 A registers of one row of a 5-trit group for thread t (see the
+// mapping above).  p: the group's 26 bytes in shared memory; lut: the table
+// (word of byte v for lane l at lut[32 v + l]); sel: byte selector of lane t.
+__device__ __forceinline__ uint32_t lds_u16(const uint8_t* p) { return *reinterpret_cast<const uint16_t*>(p); }
+
+__device__ __forceinline__ void t5_row(const uint8_t* p, const uint32_t* lut, int t, int lane, uint32_t sel,
+                                       uint32_t (&R)[8]) {
+    const uint32_t u0 = lds_u16(p + 6 * t), u1 = lds_u16(p + 6 * t + 2), u2 = lds_u16(p + 6 * t + 4);
+    const uint32_t ue = lds_u16(p + 24);
+    const uint32_t v[6] = {u0 & 0xFFu, u0 >> 8, u1 & 0xFFu, u1 >> 8, u2 & 0xFFu, u2 >> 8};
+    uint32_t c4[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+        R[i] = lut[v[i] * 32 + lane];
+        c4[i] = (v[i] * 810u) >> 16;
+    }
+    const uint32_t b24 = ue & 0xFFu, b25 = ue >> 8;
+    const uint32_t e24 = lut[b24 * 32 + lane], e25 = lut[b25 * 32 + lane];
+    // bytes 0..7 = trits 120..127: b24 digits 0..3, b24 digit 4, b25 digits 0..2
+    const uint32_t hi = ((b24 * 810u) >> 16) | (e25 << 8);
+    const uint32_t x01 = __byte_perm(e24, hi, sel);
+    R[6] = c4[0] | (c4[1] << 8) | (c4[2] << 16) | (c4[3] << 24);
+    R[7] = c4[4] | (c4[5] << 8) | (x01 << 16);
+}
+
 // ------------------------------------------------------------ one chunk
 // CT row tiles (16 rows each) starting at row tile rt, all stages.  Warp w
 // takes row tile w / WPR and groups G = w % WPR + WPR i (i < 8 / WPR), with
@@ -230,6 +287,8 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     // lower lanes' fragments: their sums are never stored
     const int blane = lane & (LANES - 1);
     const uint8_t* xres = smem + p.x_off;
+    const uint32_t* lut = reinterpret_cast<const uint32_t*>(smem + p.lut_off);
+    const uint32_t t5sel = (uint32_t)(2 * t) | ((uint32_t)(2 * t + 1) << 4);
     float yacc[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = 0.0f;
@@ -278,6 +337,23 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                             ptx::mma_u8s8_init(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1, 0);
                         else
                             ptx::mma_u8s8(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1);
+                    }
+                }
+            } else if (FMT == BQ_T5P8G128) {
+                const uint8_t* g0 = sb + my_rt * TCB + g * kT5RowBytes + 26 * G;
+                uint32_t R0[8], R1[8];
+                t5_row(g0, lut, t, lane, t5sel, R0);
+                t5_row(g0 + 8 * kT5RowBytes, lut, t, lane, t5sel, R1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                        const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                        if (q == 0)
+                            ptx::mma_u8s8_init(acc[nt], R0[0], R1[0], R0[1], R1[1], b0, b1, 0);
+                        else
+                            ptx::mma_u8s8(acc[nt], R0[2 * q], R1[2 * q], R0[2 * q + 1], R1[2 * q + 1], b0, b1);
                     }
                 }
             } else {
@@ -411,7 +487,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                     }
                     uint8_t* sb = smem + slot * slot_bytes<FMT>();
                     ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
-                    if (ct == kMaxChunkTiles) {
+                    if (FMT == BQ_T5P8G128) {
+                        if (ct == kMaxChunkTiles) {
+                            ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
+                            ptx::tma_load_2d(sb + kMaxChunkTiles * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
+                                             &full[slot]);
+                        } else {
+                            for (int i = 0; i < ct; ++i) {
+                                ptx::tma_load_2d(sb + i * TCB, &tm.codes16, st * kT5RowBytes, (r + i) * 16, &full[slot]);
+                                ptx::tma_load_2d(sb + kMaxChunkTiles * TCB + i * kTileScaleBytes, &tm.scales16,
+                                                 st * kGroupsPerStage, (r + i) * 16, &full[slot]);
+                            }
+                        }
+                    } else if (ct == kMaxChunkTiles) {
 #pragma unroll
                         for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
                             ptx::tma_load_2d(sb + b * kBoxColumnBytes, &tm.codes128,
@@ -440,6 +528,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     }
 
     // ---------------------------------------------------- compute warps
+    if (FMT == BQ_T5P8G128) {
+        // digit table: lut[32 v + l] = c0 | c1 << 8 | c2 << 16 | c3 << 24 of byte v
+        uint32_t* lut = reinterpret_cast<uint32_t*>(smem + p.lut_off);
+        for (int i = threadIdx.x; i < 256 * 32; i += kComputeWarps * 32) {
+            const uint32_t v = (uint32_t)i >> 5;
+            lut[i] = (v % 3u) | ((v / 3u % 3u) << 8) | ((v / 9u % 3u) << 16) | ((v / 27u % 3u) << 24);
+        }
+    }
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
     {
         // items (stage, group) i = warp + 16 j; the x loads of up to kPrepBatch
@@ -511,30 +607,34 @@ int sm_count() {
 
 struct Plan {
     int nt = 0, lanes = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0;
-    uint32_t x_off = 0, red_off = 0, bar_off = 0, smem = 0;
+    uint32_t x_off = 0, red_off = 0, lut_off = 0, bar_off = 0, smem = 0;
     bool ok = false;
 };
 
 Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     Plan pl;
-    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128) && batch >= 1 && batch <= 4 && k > 0 && k % 1024 == 0 && n > 0 &&
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 4 && k > 0 &&
+          k % 1024 == 0 && n > 0 &&
           n <= (int64_t)INT32_MAX - 16 && k / 4 <= (int64_t)INT32_MAX / 4 && k <= (int64_t)1 << 20))
         return pl;
     pl.nt = (batch + 1) / 2;
     pl.lanes = batch == 1 ? 16 : 32;
     pl.stages = (int)(k / 1024);
     pl.row_tiles = (int)((n + 15) / 16);
-    const int64_t slot = fmt == BQ_Q1G128 ? slot_bytes<BQ_Q1G128>() : slot_bytes<BQ_T2G128>();
+    const int64_t slot = fmt == BQ_Q1G128 ? slot_bytes<BQ_Q1G128>()
+                         : fmt == BQ_T2G128 ? slot_bytes<BQ_T2G128>() : slot_bytes<BQ_T5P8G128>();
+    const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
     const int64_t red = (int64_t)kComputeWarps * 32 * pl.nt * 2 * 4;
-    const int64_t fixed = 1024 + x_area + red + 2 * kMaxSlots * 8;
+    const int64_t fixed = 1024 + x_area + red + lut + 2 * kMaxSlots * 8;
     int64_t slots = (kSmemLimit - fixed) / slot;
     if (slots > kMaxSlots) slots = kMaxSlots;
     if (slots < 2) return pl;
     pl.slots = (int)slots;
     pl.x_off = (uint32_t)(slots * slot);
     pl.red_off = (uint32_t)(pl.x_off + x_area);
-    pl.bar_off = (uint32_t)(pl.red_off + red);
+    pl.lut_off = (uint32_t)(pl.red_off + red);
+    pl.bar_off = (uint32_t)(pl.lut_off + lut);
     pl.smem = (uint32_t)(1024 + pl.bar_off + 2 * kMaxSlots * 8);
     const int sms = sm_count();
     pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
@@ -554,7 +654,7 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : k / 4;
+    const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : (FMT == BQ_T2G128) ? k / 4 : (k / 128) * 26;
     const int64_t G = k / 128;
     Maps tm;
     for (int v = 0; v < 2; ++v) {
@@ -562,10 +662,12 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
         {
             cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n};
             cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
-            cuuint32_t box[2] = {128, rows};
+            // 5-trit rows: 208-byte boxes, unswizzled (the 128-byte swizzle needs <= 128-byte boxes)
+            cuuint32_t box[2] = {FMT == BQ_T5P8G128 ? (cuuint32_t)kT5RowBytes : 128u, rows};
             cuuint32_t es[2] = {1, 1};
             if (enc(v == 0 ? &tm.codes16 : &tm.codes128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes),
-                    dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    FMT == BQ_T5P8G128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
                 return cudaErrorInvalidValue;
         }
@@ -593,6 +695,7 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     prm.slots = pl.slots;
     prm.x_off = pl.x_off;
     prm.red_off = pl.red_off;
+    prm.lut_off = pl.lut_off;
     prm.bar_off = pl.bar_off;
     prm.status = device_status_ptr();
     if (!prm.status) return cudaErrorUnknown;
@@ -624,9 +727,14 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
         if (pl.nt == 1) return rows::launch_typed<BQ_Q1G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
         return rows::launch_typed<BQ_Q1G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     }
-    if (batch == 1) return rows::launch_typed<BQ_T2G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    if (pl.nt == 1) return rows::launch_typed<BQ_T2G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    return rows::launch_typed<BQ_T2G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (fmt == BQ_T2G128) {
+        if (batch == 1) return rows::launch_typed<BQ_T2G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        if (pl.nt == 1) return rows::launch_typed<BQ_T2G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        return rows::launch_typed<BQ_T2G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    }
+    if (batch == 1) return rows::launch_typed<BQ_T5P8G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.nt == 1) return rows::launch_typed<BQ_T5P8G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return rows::launch_typed<BQ_T5P8G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 }  // namespace bq

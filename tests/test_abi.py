@@ -102,7 +102,8 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_gemv_launches(1, 0, 4096, 1) == 0
     assert lib.bq_gemv_launches(1, 4096, 4096, 1) == 1      # row-owning kernel
     assert lib.bq_gemv_launches(2, 4096, 4096, 4) == 1
-    assert lib.bq_gemv_launches(3, 4096, 4096, 1) in (2, 3)  # 5-trit format: tcgen05 GEMM
+    assert lib.bq_gemv_launches(3, 4096, 4096, 1) == 1       # 5-trit format, row-owning kernel too
+    assert lib.bq_gemv_launches(3, 4096, 17408, 4) in (2, 3)  # operand too large: tcgen05 GEMM
     assert lib.bq_gemv_launches(1, 4096, 4096, 16) in (2, 3)
     assert lib.bq_gemm_launches(1, 17408, 5120, 4096) == 2     # prep + GEMM, no K split
     assert lib.bq_gemm_launches(1, 4096, 4096, 1) == 1         # T <= 4: the GEMV

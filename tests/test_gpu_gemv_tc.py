@@ -1,4 +1,4 @@
-"""The tensor-core decode GEMVs (binary and 2-bit ternary, batch 1..4,
+"""The tensor-core decode GEMVs (binary, 2-bit and 5-trit ternary, batch 1..4,
 K % 1024 == 0) against the oracle: the row-owning kernel (no workspace) and
 the split-K kernel it falls back to when the activation operand does not fit
 in shared memory; ragged row counts, every chunk size of the row-owning
@@ -26,10 +26,11 @@ def test_path_workspace(fmt):
     # tcgen05 GEMM with T = batch: workspace for the FP16 activations
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) >= 1152 * 2   # K % 1024 != 0
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 5) >= 5 * 4096 * 2   # batch > 4
-    assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) >= 4096 * 2
+    assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) == 0       # row-owning kernel
+    assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2   # GEMM
 
 
-@pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
 @pytest.mark.parametrize("batch", [1, 2, 3, 4])
 @pytest.mark.parametrize("n,k", [(777, 4096), (1, 1024), (128, 2048), (129, 3072), (5000, 1024), (96, 12288),
                                  (12000, 2048), (20000, 1024), (96, 17408)])
@@ -42,7 +43,7 @@ def test_tc_parity(fmt, batch, n, k):
                     what=f"tc {fmt} {n}x{k} b{batch} {name}")
 
 
-@pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
 def test_tc_activation_range(fmt):
     """Groups whose activations are all tiny (BF16 subnormals), all huge, mixed
     within a group, or all zero."""
