@@ -1,7 +1,8 @@
 // Decode GEMV, one launch per call: each CTA owns a contiguous range of whole
 // weight rows and reduces over all of K itself, so there is no workspace, no
 // preparation kernel and no cross-CTA reduction (binary g128, 2-bit-slot and
-// 5-trits-per-byte ternary g128, batch 1..4, K % 1024 == 0).
+// 5-trits-per-byte ternary g128, batch 1..8, K % 1024 == 0, while the
+// activation operand of all of K fits in shared memory).
 //
 // Arithmetic (as in the split-K tensor-core GEMV): the codes are expanded with
 // one LOP3 per four weights into int8 operands of the warp MMA m16n8k32,
@@ -613,11 +614,11 @@ struct Plan {
 
 Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     Plan pl;
-    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 4 && k > 0 &&
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 8 && k > 0 &&
           k % 1024 == 0 && n > 0 &&
           n <= (int64_t)INT32_MAX - 16 && k / 4 <= (int64_t)INT32_MAX / 4 && k <= (int64_t)1 << 20))
         return pl;
-    pl.nt = (batch + 1) / 2;
+    pl.nt = batch <= 2 ? 1 : batch <= 4 ? 2 : 4;  // n-tiles of two batch rows (5..8 -> 4)
     pl.lanes = batch == 1 ? 16 : 32;
     pl.stages = (int)(k / 1024);
     pl.row_tiles = (int)((n + 15) / 16);
@@ -725,16 +726,19 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
     if (fmt == BQ_Q1G128) {
         if (batch == 1) return rows::launch_typed<BQ_Q1G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
         if (pl.nt == 1) return rows::launch_typed<BQ_Q1G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        return rows::launch_typed<BQ_Q1G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        if (pl.nt == 2) return rows::launch_typed<BQ_Q1G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        return rows::launch_typed<BQ_Q1G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     }
     if (fmt == BQ_T2G128) {
         if (batch == 1) return rows::launch_typed<BQ_T2G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
         if (pl.nt == 1) return rows::launch_typed<BQ_T2G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        return rows::launch_typed<BQ_T2G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        if (pl.nt == 2) return rows::launch_typed<BQ_T2G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        return rows::launch_typed<BQ_T2G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     }
     if (batch == 1) return rows::launch_typed<BQ_T5P8G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     if (pl.nt == 1) return rows::launch_typed<BQ_T5P8G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    return rows::launch_typed<BQ_T5P8G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.nt == 2) return rows::launch_typed<BQ_T5P8G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return rows::launch_typed<BQ_T5P8G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 }  // namespace bq

@@ -1,4 +1,4 @@
-"""The tensor-core decode GEMVs (binary, 2-bit and 5-trit ternary, batch 1..4,
+"""The tensor-core decode GEMVs (binary, 2-bit and 5-trit ternary, batch 1..8,
 K % 1024 == 0) against the oracle: the row-owning kernel (no workspace) and
 the split-K kernel it falls back to when the activation operand does not fit
 in shared memory; ragged row counts, every chunk size of the row-owning
@@ -25,13 +25,14 @@ def test_path_workspace(fmt):
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 17408, 4) > 0
     # tcgen05 GEMM with T = batch: workspace for the FP16 activations
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) >= 1152 * 2   # K % 1024 != 0
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 5) >= 5 * 4096 * 2   # batch > 4
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 8) == 0               # batch 5..8 while x fits
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 9) >= 9 * 4096 * 2   # batch > 8
     assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) == 0       # row-owning kernel
     assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2   # GEMM
 
 
 @pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
-@pytest.mark.parametrize("batch", [1, 2, 3, 4])
+@pytest.mark.parametrize("batch", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("n,k", [(777, 4096), (1, 1024), (128, 2048), (129, 3072), (5000, 1024), (96, 12288),
                                  (12000, 2048), (20000, 1024), (96, 17408)])
 def test_tc_parity(fmt, batch, n, k):
