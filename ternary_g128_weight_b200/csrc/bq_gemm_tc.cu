@@ -24,14 +24,15 @@
 // swizzle row of FP16).  When the row tiles alone cannot fill the GPU, each
 // tile's K range is split over several CTAs and a second kernel adds the FP32
 // partial tiles in a fixed order.
-//   warps 0-3 : dequantise the tile's 128 weight rows into the stage's A
-//               buffer (K-major, 128-byte swizzle, the UMMA canonical layout),
-//               packed codes fetched four stages ahead;
-//   warp 4    : TMA loads of the FP16 activation tile (same layout) into B;
-//   warp 5    : allocates TMEM (2 x 256 columns) and issues
-//               tcgen05.mma.kind::f16 (M = 128, N = tile_n, K = 16);
-//   warps 6-9 : epilogue: TMEM -> registers -> Y (or the partial tile), while
-//               the MMAs of the next work unit accumulate in the other buffer.
+//   warps 0-7  : dequantise the tile's 128 weight rows into the stage's A
+//                buffer (K-major, 128-byte swizzle, the UMMA canonical
+//                layout), two sets of four warps on alternate stages, packed
+//                codes fetched four of their stages ahead;
+//   warp 8     : TMA loads of the FP16 activation tile (same layout) into B;
+//   warp 9     : allocates TMEM (2 x 256 columns) and issues
+//                tcgen05.mma.kind::f16 (M = 128, N = tile_n, K = 16);
+//   warps 10-13: epilogue: TMEM -> registers -> Y (or the partial tile), while
+//                the MMAs of the next work unit accumulate in the other buffer.
 // Work units are taken token-tile-major so that the activation tile in flight
 // and the packed weights stay resident in L2.
 #include <cuda.h>
@@ -49,7 +50,9 @@ constexpr int kStages = 4;
 constexpr int kABytes = kTileM * kStageK * 2;     // 16 KB
 constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kDequantWarps = 4, kTmaWarp = 4, kMmaWarp = 5, kEpiWarp0 = 6, kEpiWarps = 4;
+// two sets of 4 dequant warps take alternate stages
+constexpr int kDequantSetWarps = 4, kDequantSets = 2, kDequantWarps = kDequantSets * kDequantSetWarps;
+constexpr int kTmaWarp = kDequantWarps, kMmaWarp = kTmaWarp + 1, kEpiWarp0 = kMmaWarp + 1, kEpiWarps = 4;
 constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
 constexpr int kTmemCols = 2 * kMaxTileN;
 constexpr int kBarriers = 3 * kStages + 4;
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
-            ptx::mbar_init(&full_a[i], kDequantWarps);
+            ptx::mbar_init(&full_a[i], kDequantSetWarps);
             ptx::mbar_init(&full_b[i], 1);
             ptx::mbar_init(&empty[i], 1);
         }
@@ -312,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 
     if (warp < kDequantWarps) {
         // ------------------------------------------------ dequant producers
-        const int r = warp * 32 + lane;
+        const int set = warp / kDequantSetWarps;            // stages it with it % kDequantSets == set
+        const int r = (warp % kDequantSetWarps) * 32 + lane;
         int64_t total = 0;  // stages of this CTA
         for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x) {
             const Unit w = unit_of(p, mb_count, spt, u);
@@ -323,32 +327,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         Unit pw = unit_of(p, mb_count, spt, pu);
         int64_t prow = pw.mb * kTileM + r;
         int pst = pw.st_begin;
-        auto next_chunk = [&]() {
-            RowChunk c = {make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
-            if (pu < p.units) {
-                c = load_chunk<FMT>(p, prow, pst);
-                if (++pst == pw.st_end) {
-                    pu += gridDim.x;
-                    if (pu < p.units) {
-                        pw = unit_of(p, mb_count, spt, pu);
-                        prow = pw.mb * kTileM + r;
-                        pst = pw.st_begin;
-                    }
+        auto advance = [&]() {
+            if (pu < p.units && ++pst == pw.st_end) {
+                pu += gridDim.x;
+                if (pu < p.units) {
+                    pw = unit_of(p, mb_count, spt, pu);
+                    prow = pw.mb * kTileM + r;
+                    pst = pw.st_begin;
                 }
             }
+        };
+        // this set's next stage: load it, then step over the other sets' stages
+        auto next_chunk = [&]() {
+            RowChunk c = {make_uint4(0u, 0u, 0u, 0u), 0u, 0u};
+            if (pu < p.units) c = load_chunk<FMT>(p, prow, pst);
+#pragma unroll
+            for (int i = 0; i < kDequantSets; ++i) advance();
             return c;
         };
+        for (int i = 0; i < set; ++i) advance();
+        const int64_t mine = (total - set + kDequantSets - 1) / kDequantSets;  // stages of this set
         RowChunk pipe[kAhead];
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) pipe[i] = next_chunk();
         bool alive = true;
         // unrolled by kAhead so that each ring entry is a fixed set of registers:
         // a chunk is consumed kAhead stages after its load was issued
-        for (int64_t base = 0; base < total && alive; base += kAhead) {
+        for (int64_t base = 0; base < mine && alive; base += kAhead) {
 #pragma unroll
             for (int i = 0; i < kAhead; ++i) {
-                const int64_t it = base + i;
-                if (it < total && alive) {
+                const int64_t it = (base + i) * kDequantSets + set;  // stage index of the CTA's sequence
+                if (base + i < mine && alive) {
                     const int slot = (int)(it % kStages);
                     if (it >= kStages &&
                         !ptx::mbar_wait_bounded(&empty[slot], (uint32_t)(((it / kStages) - 1) & 1), kWaitPolls)) {
