@@ -100,6 +100,18 @@ struct Params {
     int* status;
 };
 
+// Position in the slot ring (the ring depth is a runtime value: no divisions).
+struct Ring {
+    int slot = 0, depth = 1;
+    uint32_t round = 0;  // times the ring has wrapped
+    __device__ __forceinline__ void next() {
+        if (++slot == depth) {
+            slot = 0;
+            ++round;
+        }
+    }
+};
+
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory"); }
 
 __device__ __forceinline__ int chunk_tiles(int remaining) {
@@ -275,7 +287,7 @@ __device__ __forceinline__ void t5_row(const uint8_t* p, const uint32_t* lut, in
 // WPR = min(16 / CT, 8) warps per row tile; warps past CT row tiles only
 // keep the stage barriers going.
 template <int FMT, int NT, int LANES, int CT>
-__device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, int& it,
+__device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, Ring& rp,
                           int warp, int lane) {
     constexpr int WPR = (kComputeWarps / CT) < kGroupsPerStage ? (kComputeWarps / CT) : kGroupsPerStage;
     constexpr int GPW = kGroupsPerStage / WPR;  // groups per warp and stage
@@ -294,9 +306,9 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = 0.0f;
     bool alive = true;
-    for (int st = 0; st < p.stages; ++st, ++it) {
-        const int slot = it % p.slots;
-        if (!ptx::mbar_wait_bounded(&full[slot], (uint32_t)((it / p.slots) & 1), kWaitPolls)) {
+    for (int st = 0; st < p.stages; ++st, rp.next()) {
+        const int slot = rp.slot;
+        if (!ptx::mbar_wait_bounded(&full[slot], rp.round & 1u, kWaitPolls)) {
             record_status(p.status, BQ_ERR_TIMEOUT);
             alive = false;
             break;
@@ -475,13 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
             ptx::prefetch_tensormap(&tm.scales128);
             constexpr int TCB = tile_code_bytes<FMT>();
             int it = 0;
+            Ring rp;
+            rp.depth = p.slots;
             bool alive = true;
             for (int r = rt0; r < rt1 && alive;) {
                 const int ct = chunk_tiles(rt1 - r);
-                for (int st = 0; st < p.stages; ++st, ++it) {
-                    const int slot = it % p.slots;
-                    if (it >= p.slots &&
-                        !ptx::mbar_wait_bounded(&empty[slot], (uint32_t)(((it / p.slots) - 1) & 1), kWaitPolls)) {
+                for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
+                    const int slot = rp.slot;
+                    if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
                         record_status(p.status, BQ_ERR_TIMEOUT);
                         alive = false;
                         break;
@@ -561,18 +574,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
         }
     }
     bar_compute();
-    int it = 0;
+    Ring rp;
+    rp.depth = p.slots;
     for (int r = rt0; r < rt1;) {
         const int ct = chunk_tiles(rt1 - r);
         bool ok;
         if (ct == 8)
-            ok = run_chunk<FMT, NT, LANES, 8>(p, smem, full, empty, r, it, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, 8>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 4)
-            ok = run_chunk<FMT, NT, LANES, 4>(p, smem, full, empty, r, it, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, 4>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 2)
-            ok = run_chunk<FMT, NT, LANES, 2>(p, smem, full, empty, r, it, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, 2>(p, smem, full, empty, r, rp, warp, lane);
         else
-            ok = run_chunk<FMT, NT, LANES, 1>(p, smem, full, empty, r, it, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, 1>(p, smem, full, empty, r, rp, warp, lane);
         if (!ok) break;
         r += ct;
     }
