@@ -50,7 +50,7 @@ constexpr int kGroupsPerStage = 8;  // 1024 K per stage
 constexpr int kComputeWarps = 16;
 constexpr int kProducerWarp = kComputeWarps;
 constexpr int kThreads = (kComputeWarps + 1) * 32;
-constexpr int kMaxChunkTiles = 8;
+constexpr int kMaxChunkTiles = 8;  // chunk bound of the 2-bit and 5-trit formats
 constexpr int kTileScaleBytes = 16 * kGroupsPerStage * 2;  // 256
 constexpr int kMaxSlots = 8;
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per block on sm_100
@@ -85,8 +85,13 @@ constexpr int kLutBytes = 256 * 32 * 4;           // byte -> c0..c3, one copy pe
 template <int FMT>
 constexpr int tile_code_bytes() { return FMT == BQ_T5P8G128 ? 16 * kT5RowBytes : Fmt<FMT>::kBoxes * 16 * 128; }
 constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
-template <int FMT>
-constexpr int slot_bytes() { return kMaxChunkTiles * (tile_code_bytes<FMT>() + kTileScaleBytes); }
+// Row tiles per chunk, at most: 16 for the binary format up to batch 4 (each
+// of the 16 compute warps then owns one row tile and all 8 groups of a
+// stage), else 8 (larger slots, or room needed for a larger operand).
+template <int FMT, int NT>
+constexpr int mct() { return (FMT == BQ_Q1G128 && NT <= 2) ? 16 : kMaxChunkTiles; }
+template <int FMT, int NT>
+constexpr int slot_bytes() { return mct<FMT, NT>() * (tile_code_bytes<FMT>() + kTileScaleBytes); }
 
 struct Params {
     const uint16_t* x;  // [batch][K] BF16
@@ -114,8 +119,9 @@ struct Ring {
 
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory"); }
 
+template <int FMT, int NT>
 __device__ __forceinline__ int chunk_tiles(int remaining) {
-    return remaining >= 8 ? 8 : remaining >= 4 ? 4 : remaining >= 2 ? 2 : 1;
+    return (mct<FMT, NT>() >= 16 && remaining >= 16) ? 16 : remaining >= 8 ? 8 : remaining >= 4 ? 4 : remaining >= 2 ? 2 : 1;
 }
 
 // Bytes of the resident activation operand per (stage, n-tile): B fragments
@@ -318,9 +324,9 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
             if (lane == 0) ptx::mbar_arrive(&empty[slot]);
             continue;
         }
-        const uint8_t* sb = smem + slot * slot_bytes<FMT>();
+        const uint8_t* sb = smem + slot * slot_bytes<FMT, NT>();
         const uint8_t* codes_t = sb + my_rt * 2048;  // column box 0 of this row tile
-        const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + kMaxChunkTiles * TCB + my_rt * kTileScaleBytes);
+        const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + mct<FMT, NT>() * TCB + my_rt * kTileScaleBytes);
         const uint8_t* xs = xres + (size_t)st * NT * X_NT;
 #pragma unroll
         for (int gi = 0; gi < GPW; ++gi) {
@@ -491,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
             rp.depth = p.slots;
             bool alive = true;
             for (int r = rt0; r < rt1 && alive;) {
-                const int ct = chunk_tiles(rt1 - r);
+                const int ct = chunk_tiles<FMT, NT>(rt1 - r);
                 for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
                     const int slot = rp.slot;
                     if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
@@ -499,34 +505,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                         alive = false;
                         break;
                     }
-                    uint8_t* sb = smem + slot * slot_bytes<FMT>();
+                    uint8_t* sb = smem + slot * slot_bytes<FMT, NT>();
                     ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
                     if (FMT == BQ_T5P8G128) {
                         if (ct == kMaxChunkTiles) {
                             ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + kMaxChunkTiles * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
+                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
                                              &full[slot]);
                         } else {
                             for (int i = 0; i < ct; ++i) {
                                 ptx::tma_load_2d(sb + i * TCB, &tm.codes16, st * kT5RowBytes, (r + i) * 16, &full[slot]);
-                                ptx::tma_load_2d(sb + kMaxChunkTiles * TCB + i * kTileScaleBytes, &tm.scales16,
+                                ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + i * kTileScaleBytes, &tm.scales16,
                                                  st * kGroupsPerStage, (r + i) * 16, &full[slot]);
                             }
                         }
-                    } else if (ct == kMaxChunkTiles) {
+                    } else if (ct >= kMaxChunkTiles) {
+                        // 128-row boxes: one per 128-byte column (2-bit) or per 8 row tiles (binary)
+                        for (int h8 = 0; h8 < ct / kMaxChunkTiles; ++h8) {
 #pragma unroll
-                        for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
-                            ptx::tma_load_2d(sb + b * kBoxColumnBytes, &tm.codes128,
-                                             st * (Fmt<FMT>::kBoxes * 128) + b * 128, r * 16, &full[slot]);
-                        ptx::tma_load_2d(sb + kMaxChunkTiles * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
-                                         &full[slot]);
+                            for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
+                                ptx::tma_load_2d(sb + b * kBoxColumnBytes + h8 * kBoxColumnBytes, &tm.codes128,
+                                                 st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + 8 * h8) * 16, &full[slot]);
+                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + h8 * kMaxChunkTiles * kTileScaleBytes,
+                                             &tm.scales128, st * kGroupsPerStage, (r + 8 * h8) * 16, &full[slot]);
+                        }
                     } else {
                         for (int i = 0; i < ct; ++i) {
 #pragma unroll
                             for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
                                 ptx::tma_load_2d(sb + b * kBoxColumnBytes + i * 2048, &tm.codes16,
                                                  st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + i) * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + kMaxChunkTiles * TCB + i * kTileScaleBytes, &tm.scales16,
+                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + i * kTileScaleBytes, &tm.scales16,
                                              st * kGroupsPerStage, (r + i) * 16, &full[slot]);
                         }
                     }
@@ -577,9 +586,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     Ring rp;
     rp.depth = p.slots;
     for (int r = rt0; r < rt1;) {
-        const int ct = chunk_tiles(rt1 - r);
+        const int ct = chunk_tiles<FMT, NT>(rt1 - r);
         bool ok;
-        if (ct == 8)
+        if (mct<FMT, NT>() >= 16 && ct == 16)
+            ok = run_chunk<FMT, NT, LANES, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 8)
             ok = run_chunk<FMT, NT, LANES, 8>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 4)
             ok = run_chunk<FMT, NT, LANES, 4>(p, smem, full, empty, r, rp, warp, lane);
@@ -636,8 +647,9 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.lanes = batch == 1 ? 16 : 32;
     pl.stages = (int)(k / 1024);
     pl.row_tiles = (int)((n + 15) / 16);
-    const int64_t slot = fmt == BQ_Q1G128 ? slot_bytes<BQ_Q1G128>()
-                         : fmt == BQ_T2G128 ? slot_bytes<BQ_T2G128>() : slot_bytes<BQ_T5P8G128>();
+    const int64_t slot =
+        fmt == BQ_Q1G128 ? (pl.nt <= 2 ? slot_bytes<BQ_Q1G128, 1>() : slot_bytes<BQ_Q1G128, 4>())
+        : fmt == BQ_T2G128 ? slot_bytes<BQ_T2G128, 1>() : slot_bytes<BQ_T5P8G128, 1>();
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
     const int64_t red = (int64_t)kComputeWarps * 32 * pl.nt * 2 * 4;
