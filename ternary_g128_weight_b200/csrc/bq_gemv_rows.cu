@@ -85,13 +85,13 @@ constexpr int kLutBytes = 256 * 32 * 4;           // byte -> c0..c3, one copy pe
 template <int FMT>
 constexpr int tile_code_bytes() { return FMT == BQ_T5P8G128 ? 16 * kT5RowBytes : Fmt<FMT>::kBoxes * 16 * 128; }
 constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
-// Row tiles per chunk, at most: 16 for the binary format up to batch 4 (each
-// of the 16 compute warps then owns one row tile and all 8 groups of a
-// stage), else 8 (larger slots, or room needed for a larger operand).
+// Row tiles per chunk the kernel is built for: 16 for the binary format up
+// to batch 4 (each of the 16 compute warps then owns one row tile and all 8
+// groups of a stage), else 8; a call uses 16 only where a CTA owns at least
+// 16 row tiles (see make_plan).
 template <int FMT, int NT>
 constexpr int mct() { return (FMT == BQ_Q1G128 && NT <= 2) ? 16 : kMaxChunkTiles; }
-template <int FMT, int NT>
-constexpr int slot_bytes() { return mct<FMT, NT>() * (tile_code_bytes<FMT>() + kTileScaleBytes); }
+
 
 struct Params {
     const uint16_t* x;  // [batch][K] BF16
@@ -101,6 +101,9 @@ struct Params {
     int stages;         // K / 1024
     int row_tiles;      // ceil(N / 16)
     int slots;          // ring slots
+    int slot_bytes;     // bytes per slot (chunk_cap row tiles)
+    int scales_off;     // offset of the scale tiles within a slot
+    int chunk_cap;      // row tiles per chunk, at most (8, or 16 for binary)
     uint32_t x_off, red_off, lut_off, bar_off;  // shared-memory offsets
     int* status;
 };
@@ -119,9 +122,8 @@ struct Ring {
 
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory"); }
 
-template <int FMT, int NT>
-__device__ __forceinline__ int chunk_tiles(int remaining) {
-    return (mct<FMT, NT>() >= 16 && remaining >= 16) ? 16 : remaining >= 8 ? 8 : remaining >= 4 ? 4 : remaining >= 2 ? 2 : 1;
+__device__ __forceinline__ int chunk_tiles(int remaining, int cap) {
+    return (cap >= 16 && remaining >= 16) ? 16 : remaining >= 8 ? 8 : remaining >= 4 ? 4 : remaining >= 2 ? 2 : 1;
 }
 
 // Bytes of the resident activation operand per (stage, n-tile): B fragments
@@ -324,9 +326,9 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
             if (lane == 0) ptx::mbar_arrive(&empty[slot]);
             continue;
         }
-        const uint8_t* sb = smem + slot * slot_bytes<FMT, NT>();
+        const uint8_t* sb = smem + slot * p.slot_bytes;
         const uint8_t* codes_t = sb + my_rt * 2048;  // column box 0 of this row tile
-        const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + mct<FMT, NT>() * TCB + my_rt * kTileScaleBytes);
+        const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + p.scales_off + my_rt * kTileScaleBytes);
         const uint8_t* xs = xres + (size_t)st * NT * X_NT;
 #pragma unroll
         for (int gi = 0; gi < GPW; ++gi) {
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
             rp.depth = p.slots;
             bool alive = true;
             for (int r = rt0; r < rt1 && alive;) {
-                const int ct = chunk_tiles<FMT, NT>(rt1 - r);
+                const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
                 for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
                     const int slot = rp.slot;
                     if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
@@ -505,17 +507,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                         alive = false;
                         break;
                     }
-                    uint8_t* sb = smem + slot * slot_bytes<FMT, NT>();
+                    uint8_t* sb = smem + slot * p.slot_bytes;
                     ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
                     if (FMT == BQ_T5P8G128) {
                         if (ct == kMaxChunkTiles) {
                             ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB, &tm.scales128, st * kGroupsPerStage, r * 16,
+                            ptx::tma_load_2d(sb + p.scales_off, &tm.scales128, st * kGroupsPerStage, r * 16,
                                              &full[slot]);
                         } else {
                             for (int i = 0; i < ct; ++i) {
                                 ptx::tma_load_2d(sb + i * TCB, &tm.codes16, st * kT5RowBytes, (r + i) * 16, &full[slot]);
-                                ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + i * kTileScaleBytes, &tm.scales16,
+                                ptx::tma_load_2d(sb + p.scales_off + i * kTileScaleBytes, &tm.scales16,
                                                  st * kGroupsPerStage, (r + i) * 16, &full[slot]);
                             }
                         }
@@ -526,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                             for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
                                 ptx::tma_load_2d(sb + b * kBoxColumnBytes + h8 * kBoxColumnBytes, &tm.codes128,
                                                  st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + 8 * h8) * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + h8 * kMaxChunkTiles * kTileScaleBytes,
+                            ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes,
                                              &tm.scales128, st * kGroupsPerStage, (r + 8 * h8) * 16, &full[slot]);
                         }
                     } else {
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
                             for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
                                 ptx::tma_load_2d(sb + b * kBoxColumnBytes + i * 2048, &tm.codes16,
                                                  st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + i) * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + mct<FMT, NT>() * TCB + i * kTileScaleBytes, &tm.scales16,
+                            ptx::tma_load_2d(sb + p.scales_off + i * kTileScaleBytes, &tm.scales16,
                                              st * kGroupsPerStage, (r + i) * 16, &full[slot]);
                         }
                     }
@@ -586,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     Ring rp;
     rp.depth = p.slots;
     for (int r = rt0; r < rt1;) {
-        const int ct = chunk_tiles<FMT, NT>(rt1 - r);
+        const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
         bool ok;
         if (mct<FMT, NT>() >= 16 && ct == 16)
             ok = run_chunk<FMT, NT, LANES, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
@@ -632,7 +634,7 @@ int sm_count() {
 }
 
 struct Plan {
-    int nt = 0, lanes = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0;
+    int nt = 0, lanes = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0, chunk_cap = 8, slot_bytes = 0, scales_off = 0;
     uint32_t x_off = 0, red_off = 0, lut_off = 0, bar_off = 0, smem = 0;
     bool ok = false;
 };
@@ -647,9 +649,15 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.lanes = batch == 1 ? 16 : 32;
     pl.stages = (int)(k / 1024);
     pl.row_tiles = (int)((n + 15) / 16);
-    const int64_t slot =
-        fmt == BQ_Q1G128 ? (pl.nt <= 2 ? slot_bytes<BQ_Q1G128, 1>() : slot_bytes<BQ_Q1G128, 4>())
-        : fmt == BQ_T2G128 ? slot_bytes<BQ_T2G128, 1>() : slot_bytes<BQ_T5P8G128, 1>();
+    const int sms = sm_count();
+    pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
+    // 16-tile chunks (binary, batch <= 4) only where a CTA owns at least 16
+    // row tiles; otherwise 8-tile slots keep the ring deep
+    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + kTileScaleBytes;
+    pl.chunk_cap = (fmt == BQ_Q1G128 && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
+    const int64_t slot = pl.chunk_cap * tile_bytes;
+    pl.slot_bytes = (int)slot;
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
     const int64_t red = (int64_t)kComputeWarps * 32 * pl.nt * 2 * 4;
@@ -663,8 +671,6 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.lut_off = (uint32_t)(pl.red_off + red);
     pl.bar_off = (uint32_t)(pl.lut_off + lut);
     pl.smem = (uint32_t)(1024 + pl.bar_off + 2 * kMaxSlots * 8);
-    const int sms = sm_count();
-    pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
     pl.ok = true;
     return pl;
 }
@@ -720,6 +726,9 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     prm.stages = pl.stages;
     prm.row_tiles = pl.row_tiles;
     prm.slots = pl.slots;
+    prm.slot_bytes = pl.slot_bytes;
+    prm.scales_off = pl.scales_off;
+    prm.chunk_cap = pl.chunk_cap;
     prm.x_off = pl.x_off;
     prm.red_off = pl.red_off;
     prm.lut_off = pl.lut_off;
