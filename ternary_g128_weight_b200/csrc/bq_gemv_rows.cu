@@ -185,11 +185,14 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const
             xv[hb][1] = bf16_hi(raw.x);
             xv[hb][2] = bf16_lo(raw.y);
             xv[hb][3] = bf16_hi(raw.y);
-            float m = fmaxf(fmaxf(fabsf(xv[hb][0]), fabsf(xv[hb][1])), fmaxf(fabsf(xv[hb][2]), fabsf(xv[hb][3])));
+            E[hb] = 0;
+            if (2 * nt + hb < p.batch) {  // (warp-uniform)
+                float m = fmaxf(fmaxf(fabsf(xv[hb][0]), fabsf(xv[hb][1])), fmaxf(fabsf(xv[hb][2]), fabsf(xv[hb][3])));
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            E[hb] = (m > 0.f) ? 29 - ilog2f(m) : 0;
-            if (Fmt<FMT>::kCoefShift - E[hb] < -126) two = true;
+                for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+                E[hb] = (m > 0.f) ? 29 - ilog2f(m) : 0;
+                if (Fmt<FMT>::kCoefShift - E[hb] < -126) two = true;
+            }
         }
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
@@ -208,6 +211,8 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const
             const int e1 = max(-126, min(127, es));
             const float p1 = exp2i(e1), p2 = exp2i(es - e1);
             long long sumq = 0;
+            // (k-slot of this lane's first value; the others differ by compile-time offsets)
+            uint8_t* xb = xt + (G * 2) * LANES * 16;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int kk = lane * 4 + i;
@@ -235,15 +240,13 @@ __device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const
                     }
                     q = ri >> 1; h = ri & 1;
                 }
-                const int boff = (q & 1) * 8 + h * 4 + j;
-                int rem = b;
+                // balanced base-256 digits d0..d3 of b (|b| < 2^30): the bytes of
+                // (b + 0x808080) ^ 0x808080 (adding 128 to the three low digits
+                // keeps every byte in [0, 255], so no carry crosses a byte)
+                const uint32_t w = ((uint32_t)b + 0x808080u) ^ 0x808080u;
+                uint8_t* dst = xb + ((q >> 1) * LANES + 4 * (4 * hb) + t) * 16 + (q & 1) * 8 + h * 4 + j;
 #pragma unroll
-                for (int d = 0; d < 4; ++d) {
-                    const int dv = (d < 3) ? (int)(int8_t)(rem & 0xFF) : rem;  // balanced base-256 digit
-                    rem = (rem - dv) >> 8;
-                    const int ln = 4 * (d + 4 * hb) + t;
-                    xt[((G * 2 + (q >> 1)) * LANES + ln) * 16 + boff] = (uint8_t)(dv & 0xFF);
-                }
+                for (int d = 0; d < 4; ++d) dst[d * 4 * 16] = (uint8_t)(w >> (8 * d));  // lane 4 (d + 4 hb) + t
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) sumq += __shfl_xor_sync(0xffffffffu, sumq, off);
