@@ -151,12 +151,17 @@ KERNEL_SOURCES = ("bq_gemv_rows.cu", "bq_gemv_tc.cu", "bq_gemm_tc.cu", "bq_ptx.c
 
 
 def kernel_source_hash():
-    """Identifies the kernel sources a recorded profiler capture belongs to."""
+    """Identifies the kernel sources a recorded profiler capture belongs to
+    (their code: comments and whitespace do not count)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "ternary_g128_weight_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "ternary_g128_weight_b200", "csrc", name)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

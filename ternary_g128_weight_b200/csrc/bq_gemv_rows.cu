@@ -103,7 +103,8 @@ struct Params {
     int slots;          // ring slots
     int slot_bytes;     // bytes per slot (chunk_cap row tiles)
     int scales_off;     // offset of the scale tiles within a slot
-    int chunk_cap;      // row tiles per chunk, at most (8, or 16 for binary)
+    int chunk_cap;      // row tiles per chunk, at most (1 .. 8, or 16 for binary); column boxes
+                        // of 2-bit codes are chunk_cap * 2 KB apart in a slot
     uint32_t x_off, red_off, lut_off, bar_off;  // shared-memory offsets
     int* status;
 };
@@ -123,7 +124,8 @@ struct Ring {
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory"); }
 
 __device__ __forceinline__ int chunk_tiles(int remaining, int cap) {
-    return (cap >= 16 && remaining >= 16) ? 16 : remaining >= 8 ? 8 : remaining >= 4 ? 4 : remaining >= 2 ? 2 : 1;
+    const int c = remaining < cap ? remaining : cap;
+    return c >= 16 ? 16 : c >= 8 ? 8 : c >= 4 ? 4 : c >= 2 ? 2 : 1;
 }
 
 // Bytes of the resident activation operand per (stage, n-tile): B fragments
@@ -141,8 +143,7 @@ __device__ __forceinline__ int ilog2f(float m) {
 }
 
 // ------------------------------------------------------------ activation prep
-// Warp-wide: group G of stage st for all n-tiles.  Lane l holds k = 4l .. 4l+3
-// of the group.  The byte of digit d of batch row bb for weight k goes to the
+// The byte of digit d of batch row bb for weight k goes to the
 // B fragment of lane (4 (d + 4 (bb & 1)) + t), MMA q, register h, byte j,
 // where (t, q, h, j) is the k-slot the A decode gives weight k:
 //   binary: k = 32t + 8j + 2q + h   (word t of the row's group, class 2q+h)
@@ -152,117 +153,126 @@ __device__ __forceinline__ int ilog2f(float m) {
 //           bytes 6t+4, 6t+5 and trits 120+2t, 121+2t (the group's last
 //           eight trits, in bytes 24 and 25)
 // Table entry (G, t) of an n-tile, t = 2 (bb & 1) + hh for digit pair hh, with
-// e = coef - E + 16 hh and z = [hh == 0] 2^-E sum Q:
+// e = coef - E + 16 hh and z = [hh == 0] times the group's activation sum
+// (FP32; it stands in for 2^-E sum Q, which differs by the rounding of Q):
 //   one factor  : {2^e, 1, z, 0}, u = (D0 + 256 D1) 2^e - z;
 //   two factors : {2^a, 2^(e-a), z, 1} when 2^e is not a normal float,
 //                 u = (D0 + 256 D1) 2^a 2^(e-a) - z.
-// Rows past the batch get zero entries with the group's flag (so that the
-// kernel's choice stays uniform across the warp).
-// This lane's 4 BF16 activations of group G of stage st for the batch rows of
-// the n-tiles (zero past the batch).
-template <int NT>
-__device__ __forceinline__ void load_group_x(const Params& p, int st, int G, int lane, uint2 (&raw)[2 * NT]) {
-    const int64_t kbase = (int64_t)st * 1024 + G * 128;
-#pragma unroll
-    for (int bb = 0; bb < 2 * NT; ++bb)
-        raw[bb] = bb < p.batch ? __ldg(reinterpret_cast<const uint2*>(p.x + bb * p.k + kbase + lane * 4))
-                               : make_uint2(0u, 0u);
+// Rows past the batch are prepared as zero activations (zero digits, z = 0).
+//
+// Work split: lane 4 G + t of a warp prepares group G of one stage and one
+// batch row for B-fragment thread t, i.e. the 32 activations that land in the
+// slots of thread t: k = 32 t .. 32 t + 31 (binary, 2-bit), or k = 30 t ..
+// 30 t + 29 and 120 + 2 t, 121 + 2 t (5-trit); r numbers them in that order.
+// Byte 4 m + j of the 16-byte chunk (pair P, digit d) is digit d of value
+// prep_src(P, m, j), so the lane assembles all eight of its chunks in
+// registers (a 4 x 4 byte transpose per (P, m)) and stores them whole.
+template <int FMT>
+__device__ __forceinline__ constexpr int prep_src(int P, int m, int j) {
+    if (FMT == BQ_Q1G128) return 8 * j + 4 * P + m;                    // k = 32t + 8j + 2q + h
+    if (FMT == BQ_T2G128) return 16 * (m & 1) + 4 * j + 2 * P + (m >> 1);  // k = 32t + 16h + 4j + q
+    if (P == 0) return 5 * m + j;                 // digits 0..3 of bytes 6t .. 6t+3
+    if (m < 2) return 20 + 5 * m + j;             // digits 0..3 of bytes 6t+4, 6t+5
+    if (m == 2) return 5 * j + 4;                 // digit 4 of bytes 6t .. 6t+3
+    return j == 0 ? 24 : j == 1 ? 29 : 28 + j;    // digit 4 of 6t+4, 6t+5; trits 120+2t, 121+2t
 }
 
-template <int FMT, int NT, int LANES>
-__device__ void prep_group(const Params& p, uint8_t* xst, int G, int lane, const uint2 (&xraw)[2 * NT]) {
-    constexpr int X_NT = x_nt_bytes(LANES);
+// Left shift taking the rounded value to the operand byte stream b:
+// Q = round(x 2^es) 2^kQuantShift, and the class of value r divides Q by
+// 2^(r mod 8) (binary) or 4^(r mod 4) (2-bit).
+template <int FMT>
+__device__ __forceinline__ constexpr int prep_shift(int r) {
+    return FMT == BQ_Q1G128 ? 7 - (r & 7) : FMT == BQ_T2G128 ? 6 - 2 * (r & 3) : 0;
+}
+
+// The lane's 32 activations as 16 words of two BF16 values (value r in half
+// r & 1 of word r >> 1); xg is the group's first activation (16-byte aligned).
+template <int FMT>
+__device__ __forceinline__ void load_lane_x(const uint16_t* xg, int t, uint32_t (&raw)[16]) {
+    if (FMT == BQ_T5P8G128) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(xg + 30 * t);  // 60 t bytes: 4-byte aligned
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        uint8_t* xt = xst + nt * X_NT;
-        float xv[2][4];
-        int E[2];
-        bool two = false;
+        for (int i = 0; i < 15; ++i) raw[i] = __ldg(src + i);
+        raw[15] = __ldg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
+    } else {
+        const uint4* src = reinterpret_cast<const uint4*>(xg + 32 * t);
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-            const uint2 raw = xraw[2 * nt + hb];
-            xv[hb][0] = bf16_lo(raw.x);
-            xv[hb][1] = bf16_hi(raw.x);
-            xv[hb][2] = bf16_lo(raw.y);
-            xv[hb][3] = bf16_hi(raw.y);
-            E[hb] = 0;
-            if (2 * nt + hb < p.batch) {  // (warp-uniform)
-                float m = fmaxf(fmaxf(fabsf(xv[hb][0]), fabsf(xv[hb][1])), fmaxf(fabsf(xv[hb][2]), fabsf(xv[hb][3])));
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(src + i);
+            raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
+        }
+    }
+}
+
+__device__ __forceinline__ float raw_value(const uint32_t (&raw)[16], int r) {
+    return __uint_as_float((r & 1) ? (raw[r >> 1] & 0xFFFF0000u) : (raw[r >> 1] << 16));
+}
+
+// Rows 0 .. 3 of a 4 x 4 byte matrix given as rows a, b, c, e, returned as
+// its columns: out[d] = {a.d, b.d, c.d, e.d}.
+__device__ __forceinline__ void transpose_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t e, uint32_t (&out)[4]) {
+    const uint32_t ab_lo = __byte_perm(a, b, 0x5140), ab_hi = __byte_perm(a, b, 0x7362);
+    const uint32_t ce_lo = __byte_perm(c, e, 0x5140), ce_hi = __byte_perm(c, e, 0x7362);
+    out[0] = __byte_perm(ab_lo, ce_lo, 0x5410);
+    out[1] = __byte_perm(ab_lo, ce_lo, 0x7632);
+    out[2] = __byte_perm(ab_hi, ce_hi, 0x5410);
+    out[3] = __byte_perm(ab_hi, ce_hi, 0x7632);
+}
+
+// One lane's share (group G, thread t, batch row parity hb of the n-tile at
+// xt): its eight B-fragment chunks and, on t = 0 / 1, the table entry of digit
+// pair t.  All four lanes of the group run it together (shuffles).
+template <int FMT, int LANES>
+__device__ __forceinline__ void prep_lane(uint8_t* xt, int G, int t, int hb, const uint32_t (&raw)[16]) {
+    // group maximum of |x| on the BF16 bits (a larger magnitude has larger bits)
+    uint32_t mx = 0;
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-                E[hb] = (m > 0.f) ? 29 - ilog2f(m) : 0;
-                if (Fmt<FMT>::kCoefShift - E[hb] < -126) two = true;
+    for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, raw[i] & 0x7FFF7FFFu);
+    mx = max(mx & 0xFFFFu, mx >> 16);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m = __uint_as_float(mx << 16);
+    const int E = (m > 0.f) ? 29 - ilog2f(m) : 0;
+    const int es = E - Fmt<FMT>::kQuantShift;  // x * 2^es -> Q / 2^shift
+    const int e1 = max(-126, min(127, es));
+    const float p1 = exp2i(e1), p2 = exp2i(es - e1);
+    float zs = 0.0f;
+    uint8_t* xb = xt + ((G * 2) * LANES + 16 * hb + t) * 16;  // chunk (P 0, digit 0)
+#pragma unroll
+    for (int P = 0; P < 2; ++P) {
+        uint32_t col[4][4];  // [m][digit]
+#pragma unroll
+        for (int mm = 0; mm < 4; ++mm) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = prep_src<FMT>(P, mm, j);
+                const float v = raw_value(raw, r);
+                zs += v;
+                const int b = __float2int_rn(v * p1 * p2) * (1 << prep_shift<FMT>(r));
+                // balanced base-256 digits of b (|b| <= 2^30) are the bytes of
+                // (b + 0x808080) ^ 0x808080 (the xor is applied after the transpose)
+                w[j] = (uint32_t)b + 0x808080u;
             }
+            transpose_bytes(w[0], w[1], w[2], w[3], col[mm]);
         }
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-            const int bb = 2 * nt + hb;
-            float4* tabp = reinterpret_cast<float4*>(xt + kGroupsPerStage * 2 * LANES * 16) + G * 4 + 2 * hb;
-            if (bb >= p.batch) {
-                // zero digits (rows of a 32-lane tile) and zero table entries
-                if (LANES == 32) {
-                    const int ln0 = 4 * (4 * hb) + (lane & 3), pp = (lane >> 2) & 1, dd = lane >> 3;
-                    *reinterpret_cast<uint4*>(xt + ((G * 2 + pp) * LANES + ln0 + 4 * dd) * 16) = make_uint4(0u, 0u, 0u, 0u);
-                }
-                if (lane < 2) tabp[lane] = make_float4(0.0f, 0.0f, 0.0f, two ? 1.0f : 0.0f);
-                continue;
-            }
-            const int es = E[hb] - Fmt<FMT>::kQuantShift;  // x * 2^es -> Q / 2^shift
-            const int e1 = max(-126, min(127, es));
-            const float p1 = exp2i(e1), p2 = exp2i(es - e1);
-            long long sumq = 0;
-            // (k-slot of this lane's first value; the others differ by compile-time offsets)
-            uint8_t* xb = xt + (G * 2) * LANES * 16;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int kk = lane * 4 + i;
-                const int Q = __float2int_rn(xv[hb][i] * p1 * p2) << Fmt<FMT>::kQuantShift;
-                sumq += Q;
-                int b, t, q, h, j;
-                if (FMT == BQ_Q1G128) {
-                    b = Q >> (kk & 7);  // exact: Q is a multiple of 2^7
-                    t = kk >> 5; j = (kk >> 3) & 3; q = (kk >> 1) & 3; h = kk & 1;
-                } else if (FMT == BQ_T2G128) {
-                    b = Q >> (2 * (kk & 3));  // exact: Q is a multiple of 2^6
-                    t = kk >> 5; h = (kk >> 4) & 1; j = (kk >> 2) & 3; q = kk & 3;
-                } else {
-                    b = Q;
-                    int ri;  // A register of the thread
-                    if (kk < 120) {
-                        const int byte = kk / 5, d = kk - 5 * byte, ib = byte % 6;
-                        t = byte / 6;
-                        if (d < 4) { ri = ib; j = d; }
-                        else if (ib < 4) { ri = 6; j = ib; }
-                        else { ri = 7; j = ib - 4; }
-                    } else {
-                        const int e = kk - 120;
-                        t = e >> 1; ri = 7; j = 2 + (e & 1);
-                    }
-                    q = ri >> 1; h = ri & 1;
-                }
-                // balanced base-256 digits d0..d3 of b (|b| < 2^30): the bytes of
-                // (b + 0x808080) ^ 0x808080 (adding 128 to the three low digits
-                // keeps every byte in [0, 255], so no carry crosses a byte)
-                const uint32_t w = ((uint32_t)b + 0x808080u) ^ 0x808080u;
-                uint8_t* dst = xb + ((q >> 1) * LANES + 4 * (4 * hb) + t) * 16 + (q & 1) * 8 + h * 4 + j;
-#pragma unroll
-                for (int d = 0; d < 4; ++d) dst[d * 4 * 16] = (uint8_t)(w >> (8 * d));  // lane 4 (d + 4 hb) + t
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sumq += __shfl_xor_sync(0xffffffffu, sumq, off);
-            if (lane < 2) {
-                const int hh = lane;  // digit pair (0,1) or (2,3)
-                const int e = Fmt<FMT>::kCoefShift - E[hb] + 16 * hh;
-                const double z = (hh == 0) ? ldexp((double)sumq, -E[hb]) : 0.0;
-                const int a = two ? max(-60, min(60, e)) : e;
-                float4 tab;
-                tab.x = exp2i(a);
-                tab.y = exp2i(e - a);
-                tab.z = (float)z;
-                tab.w = two ? 1.0f : 0.0f;
-                tabp[hh] = tab;
-            }
+        for (int d = 0; d < 4; ++d) {
+            const uint32_t f = d < 3 ? 0x80808080u : 0u;
+            *reinterpret_cast<uint4*>(xb + (P * LANES + 4 * d) * 16) =
+                make_uint4(col[0][d] ^ f, col[1][d] ^ f, col[2][d] ^ f, col[3][d] ^ f);
         }
+    }
+    // z = the group's activation sum (FP32, fixed order)
+    zs += __shfl_xor_sync(0xffffffffu, zs, 1);
+    zs += __shfl_xor_sync(0xffffffffu, zs, 2);
+    if (t < 2) {
+        const int hh = t;  // digit pair (0,1) or (2,3)
+        const int e = Fmt<FMT>::kCoefShift - E + 16 * hh;
+        const bool two = Fmt<FMT>::kCoefShift - E < -126;
+        const int a = two ? max(-60, min(60, e)) : e;
+        float4* tabp = reinterpret_cast<float4*>(xt + kGroupsPerStage * 2 * LANES * 16) + G * 4 + 2 * hb + hh;
+        *tabp = make_float4(exp2i(a), exp2i(e - a), hh == 0 ? zs : 0.0f, two ? 1.0f : 0.0f);
     }
 }
 
@@ -316,19 +326,8 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     float yacc[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = 0.0f;
-    bool alive = true;
-    for (int st = 0; st < p.stages; ++st, rp.next()) {
-        const int slot = rp.slot;
-        if (!ptx::mbar_wait_bounded(&full[slot], rp.round & 1u, kWaitPolls)) {
-            record_status(p.status, BQ_ERR_TIMEOUT);
-            alive = false;
-            break;
-        }
-        if (!active) {
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&empty[slot]);
-            continue;
-        }
+    // this warp's GPW groups of stage st (ring slot `slot`), added into yacc
+    auto stage = [&](int st, int slot) {
         const uint8_t* sb = smem + slot * p.slot_bytes;
         const uint8_t* codes_t = sb + my_rt * 2048;  // column box 0 of this row tile
         const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + p.scales_off + my_rt * kTileScaleBytes);
@@ -382,7 +381,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                 }
             } else {
                 // words 2t, 2t+1 of the row's 32-byte group
-                const uint8_t* box = codes_t + (G >> 2) * kBoxColumnBytes;
+                const uint8_t* box = codes_t + (G >> 2) * (p.chunk_cap * 2048);  // column box 1 after chunk_cap tiles
                 const int chunk = 2 * (G & 3) + (t >> 1);
                 const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
                 const uint2 wr0 = *reinterpret_cast<const uint2*>(box + g * 128 + off);
@@ -415,8 +414,49 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                 yacc[nt][1] = fmaf(s1, u1, yacc[nt][1]);
             }
         }
+    };
+    // Binary format: where a warp has fewer than four groups (over all
+    // n-tiles) per stage, stages are taken U at a time, so that U independent
+    // MMA chains run between two barrier waits, if the ring holds 2 U slots.
+    // (The longer 2-bit and 5-trit stage bodies measured slower this way.)
+    constexpr int U = (FMT != BQ_Q1G128 || GPW * NT >= 4) ? 1 : 4 / (GPW * NT);
+    const int ustep = (U > 1 && p.slots >= 2 * U) ? U : 1;  // (the producer keeps U slots ahead)
+    bool alive = true;
+    for (int st = 0; st < p.stages; st += ustep) {
+        const int nst = min(ustep, p.stages - st);
+        const Ring r0 = rp;  // ring position of stage st
+        int su[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            su[u] = rp.slot;
+            if (u < nst && alive) {
+                if (!ptx::mbar_wait_bounded(&full[rp.slot], rp.round & 1u, kWaitPolls)) {
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+                    alive = false;
+                }
+                rp.next();
+            }
+        }
+        if (!alive) break;
+        if (active) {
+            if constexpr (U == 1) {
+                stage(st, su[0]);
+            } else if (nst == U) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) stage(st + u, su[u]);
+            } else {
+                // (tail, or a ring too shallow for U: one stage at a time)
+                Ring rs = r0;
+#pragma unroll 1
+                for (int u = 0; u < nst; ++u, rs.next()) stage(st + u, rs.slot);
+            }
+        }
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[slot]);
+        if (lane == 0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (u < nst) ptx::mbar_arrive(&empty[su[u]]);
+        }
     }
     // digit pairs (t, t^1) -> one value per (batch row, row) on even t
 #pragma unroll
@@ -477,7 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     uint64_t* empty = full + kMaxSlots;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = gridDim.x, c = blockIdx.x;
-    const int rt0 = (int)((int64_t)c * p.row_tiles / C), rt1 = (int)((int64_t)(c + 1) * p.row_tiles / C);
+    // row tiles [rt0, rt1): the first row_tiles % C CTAs take one extra
+    const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
+    const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.slots; ++i) {
@@ -491,67 +533,79 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ weight producer
+        // lane 0 waits for the slot and posts the byte count; the copies of a
+        // stage are then issued by several lanes at once (one row tile, or one
+        // 128-row box, each)
         if (lane == 0) {
             ptx::prefetch_tensormap(&tm.codes16);
             ptx::prefetch_tensormap(&tm.scales16);
             ptx::prefetch_tensormap(&tm.codes128);
             ptx::prefetch_tensormap(&tm.scales128);
-            constexpr int TCB = tile_code_bytes<FMT>();
-            int it = 0;
-            Ring rp;
-            rp.depth = p.slots;
-            bool alive = true;
-            for (int r = rt0; r < rt1 && alive;) {
-                const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
-                for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
-                    const int slot = rp.slot;
+        }
+        constexpr int TCB = tile_code_bytes<FMT>();
+        constexpr int KB = Fmt<FMT>::kBoxes;
+        int it = 0;
+        Ring rp;
+        rp.depth = p.slots;
+        bool alive = true;
+        for (int r = rt0; r < rt1 && alive;) {
+            const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
+            for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
+                const int slot = rp.slot;
+                int ok = 1;
+                if (lane == 0) {
                     if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
                         record_status(p.status, BQ_ERR_TIMEOUT);
-                        alive = false;
-                        break;
-                    }
-                    uint8_t* sb = smem + slot * p.slot_bytes;
-                    ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
-                    if (FMT == BQ_T5P8G128) {
-                        if (ct == kMaxChunkTiles) {
-                            ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + p.scales_off, &tm.scales128, st * kGroupsPerStage, r * 16,
-                                             &full[slot]);
-                        } else {
-                            for (int i = 0; i < ct; ++i) {
-                                ptx::tma_load_2d(sb + i * TCB, &tm.codes16, st * kT5RowBytes, (r + i) * 16, &full[slot]);
-                                ptx::tma_load_2d(sb + p.scales_off + i * kTileScaleBytes, &tm.scales16,
-                                                 st * kGroupsPerStage, (r + i) * 16, &full[slot]);
-                            }
-                        }
-                    } else if (ct >= kMaxChunkTiles) {
-                        // 128-row boxes: one per 128-byte column (2-bit) or per 8 row tiles (binary)
-                        for (int h8 = 0; h8 < ct / kMaxChunkTiles; ++h8) {
-#pragma unroll
-                            for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
-                                ptx::tma_load_2d(sb + b * kBoxColumnBytes + h8 * kBoxColumnBytes, &tm.codes128,
-                                                 st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + 8 * h8) * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes,
-                                             &tm.scales128, st * kGroupsPerStage, (r + 8 * h8) * 16, &full[slot]);
-                        }
+                        ok = 0;
                     } else {
-                        for (int i = 0; i < ct; ++i) {
-#pragma unroll
-                            for (int b = 0; b < Fmt<FMT>::kBoxes; ++b)
-                                ptx::tma_load_2d(sb + b * kBoxColumnBytes + i * 2048, &tm.codes16,
-                                                 st * (Fmt<FMT>::kBoxes * 128) + b * 128, (r + i) * 16, &full[slot]);
-                            ptx::tma_load_2d(sb + p.scales_off + i * kTileScaleBytes, &tm.scales16,
-                                             st * kGroupsPerStage, (r + i) * 16, &full[slot]);
-                        }
+                        ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
                     }
                 }
-                r += ct;
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    alive = false;
+                    break;
+                }
+                uint8_t* sb = smem + slot * p.slot_bytes;
+                if (FMT == BQ_T5P8G128) {
+                    if (ct == kMaxChunkTiles) {
+                        if (lane == 0) ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
+                        if (lane == 1)
+                            ptx::tma_load_2d(sb + p.scales_off, &tm.scales128, st * kGroupsPerStage, r * 16, &full[slot]);
+                    } else if (lane < ct) {
+                        ptx::tma_load_2d(sb + lane * TCB, &tm.codes16, st * kT5RowBytes, (r + lane) * 16, &full[slot]);
+                        ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16,
+                                         st * kGroupsPerStage, (r + lane) * 16, &full[slot]);
+                    }
+                } else if (ct >= kMaxChunkTiles) {
+                    // 128-row boxes: one per 128-byte column (2-bit) and 8 row tiles
+                    const int nbox = ct / kMaxChunkTiles;
+                    if (lane < nbox * KB) {
+                        const int h8 = lane / KB, b = lane - h8 * KB;
+                        ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + h8 * kBoxColumnBytes, &tm.codes128,
+                                         st * (KB * 128) + b * 128,
+                                         (r + 8 * h8) * 16, &full[slot]);
+                    } else if (lane >= 16 && lane < 16 + nbox) {
+                        const int h8 = lane - 16;
+                        ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes, &tm.scales128,
+                                         st * kGroupsPerStage, (r + 8 * h8) * 16, &full[slot]);
+                    }
+                } else if (lane < ct) {
+#pragma unroll
+                    for (int b = 0; b < KB; ++b)
+                        ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + lane * 2048, &tm.codes16,
+                                         st * (KB * 128) + b * 128,
+                                         (r + lane) * 16, &full[slot]);
+                    ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16, st * kGroupsPerStage,
+                                     (r + lane) * 16, &full[slot]);
+                }
             }
-            // every copy this CTA issued must land before it may exit
+            r += ct;
+        }
+        // every copy this CTA issued must land before it may exit
+        if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
                 if (!ptx::mbar_wait_bounded(&full[j % p.slots], (uint32_t)((j / p.slots) & 1), kWaitPolls))
                     record_status(p.status, BQ_ERR_TIMEOUT);
-        }
         return;
     }
 
@@ -566,24 +620,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     }
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
     {
-        // items (stage, group) i = warp + 16 j; the x loads of up to kPrepBatch
-        // items are issued before any of them is processed
-        constexpr int kPrepBatch = 4;
+        // items (stage, batch row) i = warp + 16 j: lane 4 G + t takes group G;
+        // rows up to the n-tiles' width (zero past the batch; one row at 16 lanes)
+        constexpr int kPrepBatch = 2;
         uint8_t* xres = smem + p.x_off;
-        const int items = p.stages * kGroupsPerStage;
+        const int rows = LANES == 16 ? 1 : 2 * NT;
+        const int items = p.stages * rows;
+        const int G = lane >> 2, t = lane & 3;
         for (int i0 = warp; i0 < items; i0 += kComputeWarps * kPrepBatch) {
-            uint2 raw[kPrepBatch][2 * NT];
+            uint32_t raw[kPrepBatch][16];
 #pragma unroll
             for (int j = 0; j < kPrepBatch; ++j) {
                 const int i = i0 + j * kComputeWarps;
-                if (i < items) load_group_x<NT>(p, i / kGroupsPerStage, i % kGroupsPerStage, lane, raw[j]);
+                const int st = i / rows, bb = i - st * rows;
+                if (i < items && bb < p.batch) {
+                    load_lane_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, raw[j]);
+                } else {
+#pragma unroll
+                    for (int w = 0; w < 16; ++w) raw[j][w] = 0u;
+                }
             }
 #pragma unroll
             for (int j = 0; j < kPrepBatch; ++j) {
                 const int i = i0 + j * kComputeWarps;
-                if (i < items)
-                    prep_group<FMT, NT, LANES>(p, xres + (size_t)(i / kGroupsPerStage) * NT * x_nt_bytes(LANES),
-                                               i % kGroupsPerStage, lane, raw[j]);
+                if (i < items) {  // (warp-uniform)
+                    const int st = i / rows, bb = i - st * rows;
+                    prep_lane<FMT, LANES>(xres + (size_t)(st * NT + (bb >> 1)) * x_nt_bytes(LANES), G, t, bb & 1,
+                                          raw[j]);
+                }
             }
         }
     }
@@ -655,10 +719,15 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     const int sms = sm_count();
     pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
     // 16-tile chunks (binary, batch <= 4) only where a CTA owns at least 16
-    // row tiles; otherwise 8-tile slots keep the ring deep
+    // row tiles; otherwise 8-tile slots keep the ring deep.  No chunk is larger
+    // than the most tiles a CTA owns (rounded down to a power of two), so
+    // slots are sized for that; a slot is a multiple of 1 KB (the swizzled
+    // copies land on 1 KB boundaries).
     const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + kTileScaleBytes;
     pl.chunk_cap = (fmt == BQ_Q1G128 && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
-    const int64_t slot = pl.chunk_cap * tile_bytes;
+    const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
+    while (pl.chunk_cap > 1 && pl.chunk_cap > most) pl.chunk_cap >>= 1;
+    const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
     pl.slot_bytes = (int)slot;
     pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
