@@ -383,6 +383,7 @@ def main():
     weight_bytes = sum(m["codes"].numel() + 2 * m["scales"].numel() for m in mats)
     algo_bytes = weight_bytes + sum(2 * m["k"] * batch + 2 * m["n"] * batch for m in mats)
     launches_per_step = sum(bq.bq_gemv_launches(f, m["n"], m["k"], batch) for m in mats)
+    calls_per_step = len(mats)
     # the arithmetic of the path bq_gemv takes for this format and batch
     int8_path = batch <= 4 and all(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) == 0 for m in mats)
     path_dtype = "s8xu8->s32 (warp MMA), f32 recombine" if int8_path else "f16 (tcgen05) -> f32"
@@ -509,7 +510,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": path_dtype, "data": "synthetic",
             "config": {"workload": workload_name(args.model, fmt, batch, args.layers), "fmt": fmt, "batch": batch,
-                       "weight_bytes_per_step": weight_bytes, "gemv_calls_per_step": len(mats),
+                       "weight_bytes_per_step": weight_bytes, "gemv_calls_per_step": calls_per_step,
                        "l2": f"inputs larger than L2 ({weight_bytes / 1e9:.2f} GB of weights per step, L2 126 MB), no flush",
                        "parallelism": f"replicas x{world}"},
             "hbm_roofline_pct": round(100.0 * value / world / peak, 2),
