@@ -246,8 +246,7 @@ def gemm_leg(fmt, dev, reps):
 # ------------------------------------------------------------------ reference
 def run_reference(args):
     """The CPU oracle as it stands, on a bounded sample of the workload."""
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if world_info()[1] != 0:
         return 0
     import numpy as np
     import oracle
@@ -315,6 +314,30 @@ def cpu_baseline(fmt, mats, batch):
                       f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s"}
 
 
+# ------------------------------------------------------------ ranks (host side)
+def world_info():
+    """(WORLD_SIZE, RANK, LOCAL_RANK) as torchrun sets them; one process alone is rank 0 of 1."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of each rank's timings (every rank calls it, in
+    the same order); without a process group the values themselves."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_value(bytes_per_rank_step, world, ms_per_step):
+    """Whole-job GB/s: the bytes all ranks processed in one step over the
+    slowest rank's step time (replicas: each rank runs the full step)."""
+    return bytes_per_rank_step * world / (ms_per_step / 1000.0) / 1e9
+
+
 # ----------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -327,9 +350,7 @@ def main():
     import synth
     import ternary_g128_weight_b200 as bq
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = world_info()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     torch.cuda.set_device(local)
@@ -346,6 +367,9 @@ def main():
         if rank == 0:
             print(json.dumps({"metric": "prefill GEMM TFLOP/s", "fmt": fmt,
                               "prefill_gemm": gemm_leg(fmt, dev, max(args.steps, 1))}), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
         return 0
     gen = synth.device_generator(synth.SEED_BASE + 1 + 1000 * rank, device=dev)
     shapes = step_shapes(args.model, args.layers)
@@ -478,16 +502,12 @@ def main():
                "h2d": sum(2 * batch * m["k"] for m in mats), "d2h": sum(2 * batch * m["n"] for m in mats)}
 
     # ---- max over ranks
-    ms_per_step = elapsed_ms / args.steps
-    if dist is not None:
-        t = torch.tensor([ms_per_step, e2e["ms_per_step"] if e2e else 0.0], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t[0])
-        if e2e:
-            e2e["ms_per_step"] = float(t[1])
+    ms_per_step, e2e_ms = max_over_ranks([elapsed_ms / args.steps, e2e["ms_per_step"] if e2e else 0.0], dist, dev)
+    if e2e:
+        e2e["ms_per_step"] = e2e_ms
 
     peak, peak_src = measured_peaks()
-    value = weight_bytes * world / (ms_per_step / 1000.0) / 1e9
+    value = job_value(weight_bytes, world, ms_per_step)
     achieved = algo_bytes / (ms_per_step / 1000.0) / 1e9
     traffic = recorded_traffic(args.model, fmt, batch, args.layers)
 
@@ -527,7 +547,7 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
         }
         if e2e:
-            line["e2e"] = {"value": round(weight_bytes * world / (e2e["ms_per_step"] / 1000.0) / 1e9, 2),
+            line["e2e"] = {"value": round(job_value(weight_bytes, world, e2e["ms_per_step"]), 2),
                            "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
                            "d2h_bytes_per_step": e2e["d2h"]}
         if cpu:
