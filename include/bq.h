@@ -128,11 +128,13 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
  * when that is 0), 256-byte aligned; its contents on entry do not matter.
  * Asynchronous on `stream`.
  * Kernel choice (the same for bq_gemv_noalloc and for bq_gemm with T <= 4):
- * batch <= 4 and K % 1024 == 0 run the row-owning tensor-core GEMV (no
- * workspace) when its activation operand fits in shared memory; otherwise
- * binary and 2-bit ternary run the split-K tensor-core GEMV, and the 5-trit
- * format and batch 5..16 the tcgen05 GEMM with T = batch (workspace for the
- * FP16 activations).  bq_gemv_workspace_bytes reports the chosen path's need. */
+ * batch <= 8 and K % 1024 == 0 run the row-owning tensor-core GEMV (all three
+ * formats, one launch, no workspace) when its activation operand and a ring
+ * of at least two weight slots fit in shared memory; otherwise binary and
+ * 2-bit ternary at batch <= 4 run the split-K tensor-core GEMV (workspace),
+ * and the rest (the 5-trit format there, batch 9..16, K % 1024 != 0) the
+ * tcgen05 GEMM with T = batch (workspace for the FP16 activations).
+ * bq_gemv_workspace_bytes and bq_gemv_launches report the chosen path. */
 bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                   const uint16_t* x, int batch, void* y, int y_dtype,
                   void* workspace, size_t workspace_bytes, void* stream);

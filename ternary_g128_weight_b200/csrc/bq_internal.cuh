@@ -61,7 +61,7 @@ int64_t gemv_tc_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_tc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                            const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s);
 
-// Row-owning decode GEMV (binary and 2-bit ternary, batch <= 4, K % 1024 == 0,
+// Row-owning decode GEMV (all three formats, batch <= 8, K % 1024 == 0,
 // activation operand resident in shared memory): no workspace.
 bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
