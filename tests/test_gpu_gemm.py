@@ -31,9 +31,9 @@ def test_gemm_shapes(fmt, n, k, t):
                 what=f"gemm {fmt} {n}x{k} T{t}")
 
 
-@pytest.mark.parametrize("fmt", ["q1g128", "t2g128"])
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
 @pytest.mark.parametrize("shape", synth.PREFILL_SHAPES)
-@pytest.mark.parametrize("t", [64, 512, 4096])
+@pytest.mark.parametrize("t", [1, 8, 64, 512, 4096])
 def test_gemm_prefill_config_sampled(fmt, shape, t):
     """W 17408 x 5120 and 5120 x 17408 at full size; sampled output rows."""
     import torch
