@@ -14,7 +14,9 @@ pages it cites:
 * "把 27B 模型压到 4GB 跑在手机上" section 2.4 (2-bit slots waste a code; five
   trits per byte since 3^5 = 243 <= 256);
 * "1-bit Bonsai 8B" notes section 4.1 (bits mapped to signed values times the
-  group scale, decoded inside the matmul) and Table 2 (package sizes).
+  group scale, decoded inside the matmul), Table 2 (package sizes) and Table 1
+  (SwiGLU feed-forward: ``swiglu`` / ``mlp_swiglu``, with the BF16 rounding of
+  the activation a reading, not a page fact).
 
 Parity status: the packing rules (mean-|w| scale, zero maps to +1, ternary
 threshold s/2, bit order, base-3 digit order) are readings of pages that do not
@@ -75,6 +77,8 @@ def lib():
         L.bqo_matmul_rows.argtypes = [ctypes.c_int, u8p, u16p, ctypes.c_int64, ctypes.c_int64, u16p,
                                       ctypes.c_int64, i64p, ctypes.c_int64, f64p, f64p, ctypes.c_int]
         L.bqo_matmul_rows.restype = ctypes.c_int
+        L.bqo_swiglu.argtypes = [f64p, ctypes.c_int64, ctypes.c_int64, u16p, f64p]
+        L.bqo_swiglu.restype = ctypes.c_int
         L.bqo_max_threads.argtypes = []
         L.bqo_max_threads.restype = ctypes.c_int
         _lib = L
@@ -206,6 +210,36 @@ def matmul_rows(fmt, codes, scales, n: int, k: int, x_bf16: np.ndarray, rows, nt
     if st != OK:
         raise OracleError(st, "matmul_rows")
     return y, bound
+
+
+def swiglu(h: np.ndarray):
+    """SwiGLU of h[b] = [gate | up] (FP64, length 2 * inter): act[b][j] =
+    BF16_RNE(silu(gate_j) * up_j), silu(v) = v / (1 + e^-v).  Returns the BF16
+    bits [b][inter] and the unrounded FP64 values."""
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    if h.ndim == 1:
+        h = h.reshape(1, -1)
+    batch, two_i = h.shape
+    if two_i % 2:
+        raise OracleError(ERR_SHAPE, "swiglu")
+    inter = two_i // 2
+    bits = np.zeros((batch, inter), dtype=np.uint16)
+    vals = np.zeros((batch, inter), dtype=np.float64)
+    st = lib().bqo_swiglu(_ptr(h, ctypes.c_double), batch, inter, _ptr(bits, ctypes.c_uint16),
+                          _ptr(vals, ctypes.c_double))
+    if st != OK:
+        raise OracleError(st, "swiglu")
+    return bits, vals
+
+
+def mlp_swiglu(fmt, gu_codes, gu_scales, d_codes, d_scales, hidden: int, inter: int, x_bf16: np.ndarray):
+    """A gated MLP block on low-bit weights: h = W_gate|up x ([2 inter][hidden]
+    weights), act = swiglu(h) in BF16, y = W_down act ([hidden][inter]
+    weights).  Returns y, its bound sum |s act| for the BF16 act, and act's bits."""
+    h, _ = matmul(fmt, gu_codes, gu_scales, 2 * inter, hidden, x_bf16)
+    act, _ = swiglu(h)
+    y, bound = matmul(fmt, d_codes, d_scales, hidden, inter, act)
+    return y, bound, act
 
 
 def max_threads() -> int:

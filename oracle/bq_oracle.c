@@ -350,3 +350,22 @@ int bqo_matmul(int fmt, const uint8_t* codes, const uint16_t* scales,
     (void)nthreads;
     return status;
 }
+
+/* ------------------------------------------------------------ SwiGLU */
+/* silu(v) = v * sigma(v), sigma(v) = 1 / (1 + e^-v); the gate value times the
+ * matching up value, rounded once to BF16. */
+int bqo_swiglu(const double* h, int64_t batch, int64_t inter, uint16_t* act_bf16, double* act_f64) {
+    if (batch < 0 || inter < 0) return BQO_ERR_SHAPE;
+    if (batch == 0 || inter == 0) return BQO_OK;
+    if (!h || !act_bf16) return BQO_ERR_NULL;
+    for (int64_t b = 0; b < batch; ++b) {
+        const double* hb = h + b * 2 * inter;
+        for (int64_t j = 0; j < inter; ++j) {
+            const double g = hb[j], u = hb[inter + j];
+            const double a = (g / (1.0 + exp(-g))) * u;
+            act_bf16[b * inter + j] = bqo_double_to_bf16(a);
+            if (act_f64) act_f64[b * inter + j] = a;
+        }
+    }
+    return BQO_OK;
+}

@@ -69,6 +69,14 @@ int bqo_matmul_rows(int fmt, const uint8_t* codes, const uint16_t* scales,
                     const int64_t* rows, int64_t nrows,
                     double* y, double* bound, int nthreads);
 
+/* SwiGLU activation of a gated MLP block (the 8B whitepaper notes, Table 1:
+ * SwiGLU feed-forward): for h[b] = [gate | up] of length 2 * inter (the FP64
+ * product of the concatenated gate and up matrices),
+ *   act[b][j] = BF16_RNE( silu(h[b][j]) * h[b][inter + j] ),
+ *   silu(v) = v / (1 + exp(-v)),
+ * computed in FP64; act_f64 (may be NULL) receives the unrounded values. */
+int bqo_swiglu(const double* h, int64_t batch, int64_t inter, uint16_t* act_bf16, double* act_f64);
+
 /* Number of OpenMP threads a call with nthreads <= 0 would use. */
 int bqo_max_threads(void);
 

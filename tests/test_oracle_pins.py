@@ -383,3 +383,39 @@ def test_rows_variant_matches_full():
     rows = np.array([49, 0, 17, 17, 3])
     yr, br = oracle.matmul_rows("t5p8", codes, scales, n, k, x, rows)
     assert np.array_equal(yr, y[:, rows]) and np.array_equal(br, b[:, rows])
+
+
+def test_swiglu_pins():
+    """SwiGLU activation of a gated MLP block (8B notes, Table 1), pinned to
+    values its definition takes rather than to a retyped formula: sigma(1) =
+    e / (1 + e); the BF16 bits of silu(+-1), of a zero gate and of a large
+    negative gate (underflow to -0); the odd-part identity silu(v) - silu(-v) = v;
+    and the MLP composition on all-plus-one weights."""
+    e = 2.718281828459045
+    bits, vals = oracle.swiglu(np.array([[1.0, -1.0, 0.0, -100.0, 1.0, 1.0, 5.0, 2.0]]))
+    assert vals[0, 0] == pytest.approx(e / (1.0 + e), rel=1e-15)    # 0.7310585786300049
+    assert vals[0, 1] == pytest.approx(-1.0 / (1.0 + e), rel=1e-15)  # -0.2689414213699951
+    assert list(bits[0]) == [0x3F3B, 0xBE8A, 0x0000, 0x8000]          # 0.73046875, -0.26953125, 0, -0
+    # gate 2, up 3: 3 * 2 * sigma(2), sigma(2) = e^2 / (1 + e^2) (a dropped up factor,
+    # or gate and up swapped, gives another value)
+    bits, vals = oracle.swiglu(np.array([[2.0, 3.0]]))
+    assert vals[0, 0] == pytest.approx(6.0 * e * e / (1.0 + e * e), rel=1e-15)  # 5.284782467867294
+    assert bits[0, 0] == 0x40A9                                                # 5.28125
+    # odd part: gate = [v, -v], up = 1  ->  act[j] - act[inter + j] = v_j
+    v = synth.rng(7).normal(0.0, 4.0, 64)
+    _, a = oracle.swiglu(np.concatenate([v, -v, np.ones(128)]).reshape(1, -1))
+    np.testing.assert_allclose(a[0, :64] - a[0, 64:], v, rtol=1e-13, atol=1e-13)
+    # composition: every weight +1 with scale 1 and x one-hot (x_0 = 1) make every
+    # gate and up value 1, so act = BF16(silu(1)) = 0.73046875 and each output is
+    # inter * 0.73046875 exactly
+    hidden, inter = 256, 384
+    gu = np.full(oracle.codes_bytes("q1g128", 2 * inter, hidden), 0xFF, dtype=np.uint8)
+    gs = np.full(2 * inter * hidden // 128, 0x3C00, dtype=np.uint16)
+    dn = np.full(oracle.codes_bytes("q1g128", hidden, inter), 0xFF, dtype=np.uint8)
+    ds = np.full(hidden * inter // 128, 0x3C00, dtype=np.uint16)
+    x = np.zeros((1, hidden), dtype=np.uint16)
+    x[0, 0] = 0x3F80  # BF16 1.0
+    y, bound, act = oracle.mlp_swiglu("q1g128", gu, gs, dn, ds, hidden, inter, x)
+    assert np.all(act == 0x3F3B)
+    assert np.all(y == inter * 0.73046875)
+    assert np.all(bound == inter * 0.73046875)
