@@ -17,27 +17,32 @@
 // into four signed base-256 digits, one MMA column each; the k-slot of class
 // p (i) carries Q / 2^p (Q / 4^i), so every product is bit * Q or c * Q
 // exactly.  Per group and row the int32 column sums are recombined in FP32:
-//   binary : y += s * (2 * 2^-E * sum bit Q - 2^-E * sum Q)
-//   ternary: y += s * (    2^-E * sum c   Q - 2^-E * sum Q)
-// ("Bonsai-27B ... Binary g128": 0 -> -scale, 1 -> +scale; "1-bit Bonsai 8B"
-// notes, section 4.1: one FP16 scale per 128 weights).
+//   binary : y += s * (2 * 2^-E * sum bit Q - z)
+//   ternary: y += s * (    2^-E * sum c   Q - z)
+// with z the group's activation sum in FP32 (it stands in for 2^-E sum Q,
+// which differs by the rounding of Q) ("Bonsai-27B ... Binary g128": 0 ->
+// -scale, 1 -> +scale; "1-bit Bonsai 8B" notes, section 4.1: one FP16 scale
+// per 128 weights).
 //
 // CTA (one per SM): 16 compute warps and one producer warp.
-//   * The producer streams the CTA's weights -- per (chunk of up to 8 row
-//     tiles of 16 rows, stage of 1024 K) TMA boxes of codes (128-byte
-//     swizzle) and scales -- into a ring of shared-memory slots, starting
-//     before the wait on the previous kernel in the stream (programmatic
-//     dependent launch): the weights do not depend on it.  A full chunk is
-//     one 128-row box per 128-byte column (one TMA instruction per 16 KB:
-//     with one box per 16-row tile the TMA issue, not HBM, limited the
-//     stream to ~43% of the HBM bandwidth); a partial chunk uses 16-row boxes.
+//   * The producer streams the CTA's weights -- per (chunk of up to 16 row
+//     tiles of 16 rows for binary, 8 otherwise; stage of 1024 K) TMA boxes of
+//     codes (128-byte swizzle) and scales -- into a ring of shared-memory
+//     slots sized for the largest chunk the CTA owns, starting before the
+//     wait on the previous kernel in the stream (programmatic dependent
+//     launch): the weights do not depend on it.  A full chunk is one 128-row
+//     box per 128-byte column (one TMA instruction per 16 KB: with one box per
+//     16-row tile the TMA issue, not HBM, limited the stream to ~43% of the
+//     HBM bandwidth); a partial chunk uses 16-row boxes, one lane per tile.
 //   * After that wait the compute warps turn x into the MMA B fragments and
 //     the per-group recombination table for all of K, once per CTA, into
-//     shared memory.
-//   * A chunk of CT row tiles (CT = 8, 4, 2 or 1) gives each row tile
+//     shared memory: each lane builds the fragment chunks of 32 activations
+//     in registers.
+//   * A chunk of CT row tiles (CT = 16, 8, 4, 2 or 1) gives each row tile
 //     16/CT warps (at most 8), each taking an equal share of the stage's 8
 //     groups; the warps sharing a row tile add their partial sums through
-//     shared memory in warp order (deterministic).
+//     shared memory in warp order (deterministic).  Binary chunks of at most
+//     two tiles take four stages per barrier wait (independent MMA chains).
 #include <cuda.h>
 
 #include "bq_internal.cuh"
