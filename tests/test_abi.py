@@ -112,6 +112,27 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_debug_wait_timeout(-1, None) == bq.BQ_ERR_SHAPE
 
 
+def test_gemv_path_choice_host_only(lib):
+    """Which kernel a bq_gemv call takes is decided on the host (shared memory
+    plan at 148 SMs when no device is visible): the row-owning kernel needs no
+    workspace and one launch; split-K and the GEMM need workspace."""
+    ws, nl = bq.bq_gemv_workspace_bytes, bq.bq_gemv_launches
+    for fmt in ("q1g128", "t2g128", "t5p8"):
+        for n, k, b in ((4096, 4096, 1), (151936, 4096, 1), (4096, 12288, 1), (777, 1024, 2)):
+            assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)   # row-owning
+    for fmt in ("q1g128", "t2g128"):
+        assert ws(fmt, 24576, 4096, 8) == 0 and nl(fmt, 24576, 4096, 8) == 1
+    # 5-trit at batch 8: its 32 KB digit table, the operand of four n-tiles and two
+    # slots exceed shared memory -> GEMM with T = batch
+    assert ws("t5p8", 24576, 4096, 8) >= 8 * 4096 * 2
+        assert ws(fmt, 4096, 1152, 1) >= 1152 * 2                                 # K % 1024 != 0: GEMM
+        assert ws(fmt, 4096, 4096, 9) >= 9 * 4096 * 2                             # batch > 8: GEMM
+    for fmt in ("q1g128", "t2g128"):
+        assert ws(fmt, 4096, 12288, 4) == 0              # ring sized to the chunks: operand and slots fit
+        assert ws(fmt, 4096, 17408, 4) > 0 and nl(fmt, 4096, 17408, 4) == 2  # operand too large: split-K
+    assert ws("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2   # 5-trit has no split-K kernel: GEMM
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     import importlib
     mod = importlib.import_module("ternary_g128_weight_b200")
