@@ -120,17 +120,19 @@ def test_gemv_path_choice_host_only(lib):
     for fmt in ("q1g128", "t2g128", "t5p8"):
         for n, k, b in ((4096, 4096, 1), (151936, 4096, 1), (4096, 12288, 1), (777, 1024, 2)):
             assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)   # row-owning
-    for fmt in ("q1g128", "t2g128"):
-        assert ws(fmt, 24576, 4096, 8) == 0 and nl(fmt, 24576, 4096, 8) == 1
-    # 5-trit at batch 8: its 32 KB digit table, the operand of four n-tiles and two
-    # slots exceed shared memory -> GEMM with T = batch
-    assert ws("t5p8", 24576, 4096, 8) >= 8 * 4096 * 2
         assert ws(fmt, 4096, 1152, 1) >= 1152 * 2                                 # K % 1024 != 0: GEMM
         assert ws(fmt, 4096, 4096, 9) >= 9 * 4096 * 2                             # batch > 8: GEMM
     for fmt in ("q1g128", "t2g128"):
-        assert ws(fmt, 4096, 12288, 4) == 0              # ring sized to the chunks: operand and slots fit
+        assert ws(fmt, 24576, 4096, 8) == 0 and nl(fmt, 24576, 4096, 8) == 1
         assert ws(fmt, 4096, 17408, 4) > 0 and nl(fmt, 4096, 17408, 4) == 2  # operand too large: split-K
-    assert ws("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2   # 5-trit has no split-K kernel: GEMM
+    # batch 4 at K = 12288: the operand takes 209 KB; two 5 KB binary slots still fit
+    # beside it (row-owning), one 9 KB 2-bit slot does not (split-K)
+    assert ws("q1g128", 4096, 12288, 4) == 0 and nl("q1g128", 4096, 12288, 4) == 1
+    assert ws("t2g128", 4096, 12288, 4) > 0 and nl("t2g128", 4096, 12288, 4) == 2
+    # 5-trit: its 32 KB digit table leaves less room -> GEMM with T = batch where the
+    # operand of four n-tiles (batch 8) or of 17 stages at batch 4 does not fit
+    assert ws("t5p8", 24576, 4096, 8) >= 8 * 4096 * 2
+    assert ws("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
