@@ -80,15 +80,30 @@ typedef enum { BQ_BF16 = 0, BQ_F32 = 1 } bq_dtype;
 
 /* ------------------------------------------------------------------ sizes */
 /* Bytes of the code array for an N x K matrix; -1 for an invalid format or
- * shape (negative size or K % 128 != 0). */
+ * shape (negative size or K % 128 != 0).  Binary: one bit per weight, packed
+ * ("1-bit Bonsai 8B" notes, section 4.1: the {0,1} bits are stored packed,
+ * 1 bit per weight).  2-bit slots: one 2-bit code per trit; 5 trits per byte:
+ * 3^5 = 243 <= 256 ("把 27B 模型压到 4GB" section 2.4 on both ternary
+ * storages). */
 int64_t bq_codes_bytes(int fmt, int64_t n, int64_t k);
-/* Bytes of the FP16 scale array, N * (K/128) * 2; -1 for an invalid shape. */
+/* Bytes of the FP16 scale array, N * (K/128) * 2; -1 for an invalid shape.
+ * One FP16 scale per 128 consecutive weights ("Bonsai-27B-mlx-1bit ...
+ * Binary g128", section "Binary g128权重表示原理"). */
 int64_t bq_scales_bytes(int64_t n, int64_t k);
-/* Storage bits per weight including the scale: 1.125, 2.125, 1.75; -1 if invalid. */
+/* Storage bits per weight including the scale: 1.125, 2.125, 1.75; -1 if
+ * invalid.  1.125 = 1 + 16/128 is the binary g128 figure of the "1-bit Bonsai
+ * 8B" notes (section 4.1, Table 2); the ternary page's 1.71 bits ("Ternary
+ * Bonsai", section "什么是Ternary Bonsai技术") is the entropy log2(3) + 16/128,
+ * which no byte-addressed storage here reaches. */
 double bq_effective_bits(int fmt);
 
 /* ---------------------------------------------------------------- packers */
 /* Float weights -> codes + FP16 scales (one thread per 128-weight group).
+ * The codes: bq_pack_q1g128 writes bit 1 for +scale and bit 0 for -scale
+ * ("Bonsai-27B-mlx-1bit ... Binary g128", section "Binary g128权重表示原理");
+ * bq_pack_t2g128 / bq_pack_t5p8 write trits {-1, 0, +1} in 2-bit slots / five
+ * per byte ("Ternary Bonsai", section "什么是Ternary Bonsai技术"; "把 27B 模型压到
+ * 4GB" section 2.4).
  * Reading of the pages, which do not state the rule for trained weights:
  *   s = FP16 round-to-nearest-even of (sum of |w| over the group, summed in
  *       order in FP64) / 128, unless `scales_in` gives the scales;
@@ -133,8 +148,10 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
  * of at least two weight slots fit in shared memory; otherwise binary and
  * 2-bit ternary at batch <= 4 run the split-K tensor-core GEMV (workspace),
  * and the rest (the 5-trit format there, batch 9..16, K % 1024 != 0) the
- * tcgen05 GEMM with T = batch (workspace for the FP16 activations).
- * bq_gemv_workspace_bytes and bq_gemv_launches report the chosen path. */
+ * tcgen05 GEMM with T = batch (workspace for the FP16 activations).  A shape
+ * no kernel takes (K > 2^28, or N >= 2^31) returns BQ_ERR_SHAPE.
+ * bq_gemv_workspace_bytes and bq_gemv_launches report the chosen path (-1 for
+ * such a shape). */
 bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                   const uint16_t* x, int batch, void* y, int y_dtype,
                   void* workspace, size_t workspace_bytes, void* stream);
@@ -171,7 +188,7 @@ int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t);
  * a dense contraction).  For T <= 16 this is bq_gemv with batch = T.  Larger T
  * runs a tensor-core (tcgen05) kernel that dequantises W tiles on chip to FP16
  * s*q (exact) and multiplies by X converted to FP16 with a per-token
- * power-of-two pre-scale (exact for every BF16 value within 2^-32 of the
+ * power-of-two pre-scale (exact for every BF16 value within 2^-31 of the
  * token's largest magnitude), accumulating in FP32.
  * X BF16 [T][K] 16-byte aligned; Y BF16 [T][N] 16-byte aligned; workspace as
  * bq_gemm_workspace_bytes, 256-byte aligned.  Asynchronous on `stream`. */

@@ -83,7 +83,7 @@ GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
     if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
     if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
     if (gemm_tc_eligible(fmt, n, k, batch)) return GemvPath::Gemm;
-    return GemvPath::Simt;
+    return GemvPath::None;
 }
 
 int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
@@ -100,7 +100,7 @@ cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, i
         case GemvPath::Rows: return launch_gemv_rows(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
         case GemvPath::SplitK: return launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
         case GemvPath::Gemm: return launch_gemm_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
-        default: return launch_gemv_simt(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 }  // namespace bq
@@ -148,13 +148,14 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch) {
         case GemvPath::Rows: return 1;
         case GemvPath::SplitK: return 2;  // activation prep + split-K kernel
         case GemvPath::Gemm: return gemm_tc_launches(n, k, batch);
-        default: return 1;
+        default: return -1;  // no kernel takes the shape (bq_gemv returns BQ_ERR_SHAPE)
     }
 }
 
 int64_t bq_gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || batch < 1 || batch > BQ_MAX_BATCH) return -1;
     if (n == 0 || k == 0) return 0;
+    if (gemv_path(fmt, n, k, batch) == GemvPath::None) return -1;
     return gemv_workspace_bytes(fmt, n, k, batch);
 }
 
@@ -169,6 +170,7 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     if (!y || (k > 0 && !x)) return BQ_ERR_NULL;
     if (!aligned(y, 16) || (x && !aligned(x, 16))) return BQ_ERR_ALIGN;
     const int64_t need = bq_gemv_workspace_bytes(fmt, n, k, batch);
+    if (need < 0) return BQ_ERR_SHAPE;
     if (need > 0 && (!workspace || workspace_bytes < (size_t)need)) return BQ_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 256)) return BQ_ERR_ALIGN;
     if (k == 0) {
@@ -181,8 +183,8 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
 
 // Prefill dispatch: up to 4 tokens run the tensor-core GEMV paths (the weight
 // stream dominates and the result is bit-identical with bq_gemv); more tokens
-// run the tcgen05 GEMM; shapes neither takes run the CUDA-core GEMV in chunks
-// of 16.
+// run the tcgen05 GEMM.  A shape neither takes (K > 2^28, N >= 2^31) is
+// rejected with BQ_ERR_SHAPE.
 static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
     if (t > 4) return false;
     const GemvPath p = gemv_path(fmt, n, k, (int)t);
@@ -194,7 +196,7 @@ int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
     if (t == 0 || n == 0 || k == 0) return 0;
     if (gemm_uses_gemv(fmt, n, k, t)) return gemv_workspace_bytes(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_workspace_bytes(n, k, t);
-    return 0;
+    return -1;
 }
 
 int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t) {
@@ -202,7 +204,7 @@ int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t) {
     if (t == 0 || n == 0 || k == 0) return 0;
     if (gemm_uses_gemv(fmt, n, k, t)) return bq_gemv_launches(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_launches(n, k, t);
-    return (int)((t + BQ_MAX_BATCH - 1) / BQ_MAX_BATCH);
+    return -1;
 }
 
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
@@ -215,22 +217,17 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     if (!y || (k > 0 && !x)) return BQ_ERR_NULL;
     if (!aligned(y, 16) || (x && !aligned(x, 16))) return BQ_ERR_ALIGN;
     const int64_t need = bq_gemm_workspace_bytes(fmt, n, k, t);
+    if (need < 0) return BQ_ERR_SHAPE;
     if (need > 0 && (!workspace || workspace_bytes < (size_t)need)) return BQ_ERR_WORKSPACE;
     if (workspace && !aligned(workspace, 256)) return BQ_ERR_ALIGN;
     cudaStream_t s = as_stream(stream);
     if (k == 0)
         return cudaMemsetAsync(y, 0, (size_t)t * n * 2, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     cudaError_t e = cudaSuccess;
-    if (gemm_uses_gemv(fmt, n, k, t)) {
+    if (gemm_uses_gemv(fmt, n, k, t))
         e = launch_gemv(fmt, codes, scales, n, k, x, (int)t, y, BQ_BF16, workspace, s);
-    } else if (gemm_tc_eligible(fmt, n, k, t)) {
+    else
         e = launch_gemm_tc(fmt, codes, scales, n, k, x, t, y, BQ_BF16, workspace, s);
-    } else {
-        for (int64_t t0 = 0; t0 < t && e == cudaSuccess; t0 += BQ_MAX_BATCH) {
-            const int b = (int)((t - t0) < BQ_MAX_BATCH ? (t - t0) : BQ_MAX_BATCH);
-            e = launch_gemv_simt(fmt, codes, scales, n, k, x + t0 * k, b, y + t0 * n, BQ_BF16, s);
-        }
-    }
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 

@@ -100,7 +100,8 @@ __device__ __forceinline__ void permute_stage(const uint32_t (&in)[32], uint32_t
 
 // ----------------------------------------------------------------- X prep
 // One CTA per token: X' = FP16(x * 2^e) in the permuted K order,
-// inv_scale = 2^-e with e = 14 - floor(log2 max|x|) (0 for an all-zero row).
+// inv_scale = 2^-e with e = 14 - floor(log2 max|x|) (0 for an all-zero row):
+// exact for every BF16 value within 2^-31 of the row's largest magnitude.
 template <int FMT>
 __global__ void __launch_bounds__(128) xprep_f16_kernel(const uint16_t* __restrict__ x, int64_t k,
                                                         uint16_t* __restrict__ xh, float* __restrict__ inv_scale) {
@@ -121,8 +122,9 @@ __global__ void __launch_bounds__(128) xprep_f16_kernel(const uint16_t* __restri
     if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
     __syncthreads();
     m = fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3]));
-    int e = (m > 0.f) ? 14 - ilogbf(m) : 0;
-    e = max(-126, min(126, e));
+    // e is in [-113, 147] for any finite BF16 maximum (2^-133 .. 2^128); 2^-e
+    // is then a normal or subnormal float, both exact
+    const int e = (m > 0.f) ? 14 - ilogbf(m) : 0;
     if (threadIdx.x == 0) inv_scale[t] = ldexpf(1.0f, -e);
     const int64_t stages = k / kStageK;
     for (int64_t st = threadIdx.x; st < stages; st += blockDim.x) {
@@ -522,32 +524,6 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float* __restr
 }
 
 // ----------------------------------------------------------------- host
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-int sm_count() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    return sms;
-}
 
 // Tile shape, K split and grid of one call.
 struct Plan {
@@ -581,11 +557,9 @@ template <int FMT>
 cudaError_t launch_typed(Params prm, const Plan& pl, const uint16_t* x, uint16_t* xh, float* inv_scale, cudaStream_t s) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    {
+        const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemm_tc_kernel<FMT>), kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     CUtensorMap tm_x;
     {

@@ -678,32 +678,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
 }
 
 // ----------------------------------------------------------------- host
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-int sm_count() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    return sms;
-}
 
 struct Plan {
     int nt = 0, lanes = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0, chunk_cap = 8, slot_bytes = 0, scales_off = 0;
@@ -757,12 +731,9 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
                          int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_rows_kernel<FMT, NT, LANES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmemLimit);
+    {
+        const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_rows_kernel<FMT, NT, LANES>), kSmemLimit);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : (FMT == BQ_T2G128) ? k / 4 : (k / 128) * 26;
     const int64_t G = k / 128;

@@ -498,21 +498,6 @@ __global__ void __launch_bounds__(kThreads, 2) gemv_tc_kernel(const __grid_const
 }
 
 // ----------------------------------------------------------------- host
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
 
 struct Plan {
     int nt = 0, stages_total = 0, row_blocks = 0, grid = 0;
@@ -522,17 +507,6 @@ struct Plan {
 bool eligible(int fmt, int64_t n, int64_t k, int batch) {
     return (fmt == BQ_Q1G128 || fmt == BQ_T2G128) && batch >= 1 && batch <= 4 && k > 0 && k % 1024 == 0 &&
            n > 0 && n <= (int64_t)INT32_MAX && k / 8 <= (int64_t)INT32_MAX / 4;
-}
-
-int sm_count() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    return sms;
 }
 
 Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
@@ -557,12 +531,9 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     using L = Layout<FMT, NT>;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_tc_kernel<FMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::kSmemBytes);
+    {
+        const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_tc_kernel<FMT, NT>), L::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : k / 4;
     const int64_t G = k / 128;

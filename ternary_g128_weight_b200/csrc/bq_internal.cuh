@@ -1,5 +1,6 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -29,6 +30,17 @@ __device__ __forceinline__ void record_pack_error(unsigned long long* first, int
 // Address of the device status word of the current device.
 int* device_status_ptr();
 
+// Per-device launcher state (bq_device.cu): the current device's SM count,
+// raising a kernel's opt-in dynamic shared memory on the current device (once
+// per kernel and device), and the driver's cuTensorMapEncodeTiled (NULL if the
+// driver lacks it).  Safe to call from several host threads.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+int sm_count();
+cudaError_t ensure_dynamic_smem(const void* func, int bytes);
+EncodeTiledFn encode_fn();
+
 // BF16 bit pattern -> float (exact).
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
     return __uint_as_float(b << 16);
@@ -50,9 +62,6 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
 cudaError_t launch_pack(int fmt, const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
                         uint8_t* codes, uint16_t* scales, unsigned long long* first_error,
                         cudaStream_t s);
-cudaError_t launch_gemv_simt(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n,
-                             int64_t k, const uint16_t* x, int batch, void* y, int y_dtype,
-                             cudaStream_t s);
 cudaError_t launch_wait_timeout(int64_t spin_limit, cudaStream_t s);
 
 // Tensor-core decode GEMV (binary and 2-bit ternary, batch <= 4, K % 1024 == 0).
@@ -69,9 +78,10 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
 
 // GEMV path choice shared by bq_gemv, bq_gemm (T <= 4) and bq_gemv_noalloc:
 // the row-owning kernel where eligible, else the split-K tensor-core kernel,
-// else the tcgen05 GEMM with T = batch (5-trit format, batch 5..16), else the
-// CUDA-core kernel.  gemv_workspace_bytes reports the workspace of the choice.
-enum class GemvPath { Rows, SplitK, Gemm, Simt };
+// else the tcgen05 GEMM with T = batch; None when no kernel takes the shape
+// (K > 2^28 or N >= 2^31).  gemv_workspace_bytes reports the workspace of the
+// choice.
+enum class GemvPath { Rows, SplitK, Gemm, None };
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch);
 int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,

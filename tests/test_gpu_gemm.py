@@ -5,7 +5,7 @@ import pytest
 import oracle
 import synth
 import ternary_g128_weight_b200 as bq
-from gpu_util import check_close, to_dev, x_to_dev
+from gpu_util import check_close, to_dev, x_to_dev, y_to_f64
 from test_gpu_gemv import host_weights
 
 pytestmark = pytest.mark.gpu
@@ -74,3 +74,68 @@ def test_gemm_t1_matches_gemv():
     y2 = bq.bq_gemv("q1g128", c, s, n, k, xd)
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+def _edge_tokens(g, t, k):
+    """T tokens of BF16 activations at the edges of the per-token FP16
+    pre-scale: an all-zero token, magnitudes spread over 1e-30 .. 1e30 with
+    zeros, one large value with the rest at and below 2^-31 of it (rounded or
+    flushed by the pre-scale), a token whose largest magnitude is ~1e-36 (the
+    pre-scale exponent past 126), BF16 subnormals only, and N(0,1) tokens."""
+    x = np.empty((t, k), dtype=np.float32)
+    for i in range(t):
+        kind = i % 7
+        sign = g.choice([-1.0, 1.0], size=k)
+        if kind == 0:
+            x[i] = 0.0
+        elif kind == 1:
+            x[i] = sign * 10.0 ** g.uniform(-30, 30, size=k)
+            x[i, ::5] = 0.0
+        elif kind == 2:
+            x[i] = sign * 2.0 ** (100 - g.uniform(20, 60, size=k))
+            x[i, g.integers(0, k)] = 2.0 ** 100
+        elif kind == 3:
+            x[i] = sign * 1e-36 * g.uniform(0.0, 1.0, size=k)
+        elif kind == 4:
+            x[i] = sign * 2.0 ** -133 * g.integers(0, 128, size=k)
+        else:
+            x[i] = g.standard_normal(k)
+    return synth.float32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+@pytest.mark.parametrize("n,k,batch", [(300, 2048, 9), (257, 4096, 16), (200, 1152, 5), (129, 1152, 8)])
+def test_gemm_path_activation_edges_f32(fmt, n, k, batch):
+    """The tcgen05 GEMM (bq_gemv routes batch 9..16, and K % 1024 != 0, to it
+    with T = batch) with F32 output on edge-case activations: the per-token
+    FP16 pre-scale must keep every output within 2e-3 sum|s x| (plus the F32
+    rounding of y)."""
+    import torch
+    assert bq.bq_gemv_launches(fmt, n, k, batch) in (2, 3)  # activation prep + GEMM (+ split-K reduce)
+    codes, scales = host_weights(fmt, n, k, synth.SEED_BASE + 95 + n)
+    x = _edge_tokens(synth.rng(96 + batch), batch, k)
+    yref, bound = oracle.matmul(fmt, codes, scales, n, k, x)
+    y = bq.bq_gemv(fmt, to_dev(codes), to_dev(scales.astype(np.int16)), n, k, x_to_dev(x), y_dtype=bq.BQ_F32)
+    torch.cuda.synchronize()
+    assert bq.bq_check() == bq.BQ_OK
+    check_close(y, yref, bound, "f32", strict=False, what=f"gemm edges {fmt} {n}x{k} T{batch}")
+    assert np.all(y_to_f64(y)[0] == 0.0)  # the all-zero token
+
+
+@pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
+@pytest.mark.parametrize("t", [5, 17, 64])
+def test_gemm_activation_edges_bf16(fmt, t):
+    """bq_gemm (BF16 output) on the same edge-case tokens; outputs whose exact
+    value is a BF16 subnormal are compared against the oracle rounded to BF16."""
+    import torch
+    n, k = 256, 2048
+    codes, scales = host_weights(fmt, n, k, synth.SEED_BASE + 97)
+    x = _edge_tokens(synth.rng(98 + t), t, k)
+    yref, bound = oracle.matmul(fmt, codes, scales, n, k, x)
+    y = run_gemm(fmt, codes, scales, n, k, x)
+    yv = y_to_f64(y)
+    # the BF16 output grid near zero is 2^-133: allow half of it on top of the stated bound
+    err = np.abs(yv - yref)
+    allow = 2e-3 * bound + 2.0 ** -8 * (np.abs(yref) + 2e-3 * bound) + 2.0 ** -134
+    assert np.all(err <= allow), float((err / allow).max())
+    assert np.all(yv[0] == 0.0)
