@@ -1,5 +1,6 @@
 // Per-device host state of the launchers: the SM count, the opt-in dynamic
-// shared-memory size of each kernel, and the driver's tensor-map encoder.
+// shared-memory size and carveout of each kernel, and the driver's tensor-map
+// encoder.
 // A process may drive several GPUs, from several host threads: the SM count
 // and the kernel attribute are kept per device (a function attribute set with
 // one device current does not carry over to another), under one mutex.
@@ -57,6 +58,12 @@ cudaError_t ensure_dynamic_smem(const void* func, int bytes) {
     for (int i = 0; i < g_nattrs; ++i)
         if (g_attrs[i].func == func && g_attrs[i].device == dev && g_attrs[i].bytes >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    // Every kernel of the library asks for the largest shared-memory carveout,
+    // so that an SM never has to change its L1 / shared split between two of
+    // them (it can only do so when idle): a call's CTAs can then start on an
+    // SM while the previous call's CTAs still run there.
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     for (int i = 0; i < g_nattrs; ++i)
         if (g_attrs[i].func == func && g_attrs[i].device == dev) {

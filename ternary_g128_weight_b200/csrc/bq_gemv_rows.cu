@@ -4,45 +4,46 @@
 // 5-trits-per-byte ternary g128, batch 1..8, K % 1024 == 0, while the
 // activation operand of all of K fits in shared memory).
 //
-// Arithmetic (as in the split-K tensor-core GEMV): the codes are expanded with
-// one LOP3 per four weights into int8 operands of the warp MMA m16n8k32,
+// Arithmetic: the codes are expanded with one LOP3 per four weights into int8
+// operands of the warp MMA m16n8k32,
 //   binary : byte j of (w & (0x01010101 << p)) = 2^p * bit(8j+p),
 //   2-bit  : byte j of (w & (0x03030303 << 2i)) = 4^i * c(4j+i), c = q+1,
 //   5-trit : a byte v = sum c_i 3^i ("把 27B 模型压到 4GB" section 2.4: 3^5 <= 256)
 //            gives c0..c3 as the four bytes of a 256-entry table word (one
 //            copy per lane in shared memory, so lookups never conflict) and
 //            c4 = (810 v) >> 16 (exact for v < 243),
-// against activations in per-(batch row, group) fixed point Q (largest |x| of
-// the group mapped into [2^29, 2^30), Q a multiple of 2^7 resp. 2^6), split
-// into four signed base-256 digits, one MMA column each; the k-slot of class
-// p (i) carries Q / 2^p (Q / 4^i), so every product is bit * Q or c * Q
-// exactly.  Per group and row the int32 column sums are recombined in FP32:
-//   binary : y += s * (2 * 2^-E * sum bit Q - z)
-//   ternary: y += s * (    2^-E * sum c   Q - z)
-// with z the group's activation sum in FP32 (it stands in for 2^-E sum Q,
-// which differs by the rounding of Q) ("Bonsai-27B ... Binary g128": 0 ->
-// -scale, 1 -> +scale; "1-bit Bonsai 8B" notes, section 4.1: one FP16 scale
-// per 128 weights).
+// against activations in per-(batch row, group) fixed point: with 2^E mapping
+// the group's largest |x| into [2^29, 2^30), the k-slot of class p (binary) or
+// i (2-bit) carries B = round(x 2^(E-p)) resp. round(x 2^(E-2i)), so that the
+// product A * B = bit * x * 2^E (resp. c * x * 2^E) up to 2^(p-1) units of
+// 2^-E (at most 2^-23 of the group's largest |x| per element).  B is split
+// into four signed base-256 digits, one MMA column each.  Per group and row the
+// int32 column sums are recombined in FP32:
+//   binary : y += s * (2 * 2^-E * sum bit B 2^p - z)
+//   ternary: y += s * (    2^-E * sum c   B 4^i - z)
+// with z the group's activation sum in FP32 ("Bonsai-27B ... Binary g128":
+// 0 -> -scale, 1 -> +scale; "1-bit Bonsai 8B" notes, section 4.1: one FP16
+// scale per 128 weights).
 //
-// CTA (one per SM): 16 compute warps and one producer warp.
-//   * The producer streams the CTA's weights -- per (chunk of up to 16 row
-//     tiles of 16 rows for binary, 8 otherwise; stage of 1024 K) TMA boxes of
-//     codes (128-byte swizzle) and scales -- into a ring of shared-memory
-//     slots sized for the largest chunk the CTA owns, starting before the
-//     wait on the previous kernel in the stream (programmatic dependent
-//     launch): the weights do not depend on it.  A full chunk is one 128-row
-//     box per 128-byte column (one TMA instruction per 16 KB: with one box per
-//     16-row tile the TMA issue, not HBM, limited the stream to ~43% of the
-//     HBM bandwidth); a partial chunk uses 16-row boxes, one lane per tile.
-//   * After that wait the compute warps turn x into the MMA B fragments and
-//     the per-group recombination table for all of K, once per CTA, into
-//     shared memory: each lane builds the fragment chunks of 32 activations
-//     in registers.
-//   * A chunk of CT row tiles (CT = 16, 8, 4, 2 or 1) gives each row tile
-//     16/CT warps (at most 8), each taking an equal share of the stage's 8
-//     groups; the warps sharing a row tile add their partial sums through
-//     shared memory in warp order (deterministic).  Binary chunks of at most
-//     two tiles take four stages per barrier wait (independent MMA chains).
+// CTA: NW compute warps and one producer warp, in one of two shapes.
+//   * NW = 8, at most half of an SM's shared memory and registers, two CTAs
+//     per SM: the largest matrices (LM heads) at batch 1-2, where each warp
+//     takes two row tiles of a 16-tile chunk and reuses the activation
+//     fragments of a group for both.
+//   * NW = 16, one CTA per SM: everything else.
+//   The producer streams the CTA's weights -- per (chunk of row tiles of 16
+//   rows; stage of 1024 K) TMA boxes of codes (128-byte swizzle) and scales --
+//   into a ring of shared-memory slots, starting before the wait on the
+//   previous kernel in the stream (the weights do not depend on it).  A full
+//   chunk is one 128-row box per 128-byte column (one TMA instruction per
+//   16 KB); a partial chunk uses 16-row boxes, one lane per tile.
+//   After that wait the compute warps turn x into the MMA B fragments and the
+//   per-group recombination table for all of K, into shared memory; the work
+//   is spread over every compute lane (one lane per 16 activations).
+//   A chunk of CT row tiles gives each warp TPW = CT / NW row tiles (CT >= NW)
+//   or gives each row tile NW / CT warps, each taking a contiguous share of the
+//   stage's 8 groups; the warps sharing a row tile add their partial sums
+//   through shared memory in warp order (deterministic).
 #include <cuda.h>
 
 #include "bq_internal.cuh"
@@ -52,51 +53,46 @@ namespace bq {
 namespace rows {
 
 constexpr int kGroupsPerStage = 8;  // 1024 K per stage
-constexpr int kComputeWarps = 16;
-constexpr int kProducerWarp = kComputeWarps;
-constexpr int kThreads = (kComputeWarps + 1) * 32;
-constexpr int kMaxChunkTiles = 8;  // chunk bound of the 2-bit and 5-trit formats
+constexpr int kMaxChunkTiles = 8;   // chunk bound of the 2-bit and 5-trit formats
 constexpr int kTileScaleBytes = 16 * kGroupsPerStage * 2;  // 256
 constexpr int kMaxSlots = 8;
-constexpr int kSmemLimit = 232448;  // opt-in shared memory per block on sm_100
+constexpr int kSmemFull = 232448;  // opt-in shared memory per block on sm_100 (one CTA per SM)
+constexpr int kSmemHalf = 115712;  // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2
 constexpr uint32_t kWaitPolls = 1u << 23;
+
+template <int NW>
+constexpr int threads_of() { return (NW + 1) * 32; }
 
 template <int FMT>
 struct Fmt;
 template <>
 struct Fmt<BQ_Q1G128> {
-    static constexpr int kBoxes = 1;         // 128-byte columns per row tile and stage
-    static constexpr int kCoefShift = 1;     // 2 * sum(bit * x) - sum(x)
-    static constexpr int kQuantShift = 7;    // Q multiple of 2^7
+    static constexpr int kBoxes = 1;      // 128-byte columns per row tile and stage
+    static constexpr int kCoefShift = 1;  // 2 * sum(bit * x) - sum(x)
 };
 template <>
 struct Fmt<BQ_T2G128> {
     static constexpr int kBoxes = 2;
-    static constexpr int kCoefShift = 0;     // sum(c * x) - sum(x)
-    static constexpr int kQuantShift = 6;    // Q multiple of 2^6
+    static constexpr int kCoefShift = 0;  // sum(c * x) - sum(x)
 };
 template <>
 struct Fmt<BQ_T5P8G128> {
-    static constexpr int kBoxes = 1;         // one unswizzled 208-byte column (8 groups x 26 bytes)
-    static constexpr int kCoefShift = 0;     // sum(c * x) - sum(x)
-    static constexpr int kQuantShift = 0;    // plain bytes c, operand Q
+    static constexpr int kBoxes = 1;      // one unswizzled 208-byte column (8 groups x 26 bytes)
+    static constexpr int kCoefShift = 0;  // sum(c * x) - sum(x)
 };
 constexpr int kT5RowBytes = kGroupsPerStage * 26;  // 208
 constexpr int kLutBytes = 256 * 32 * 4;           // byte -> c0..c3, one copy per lane
 // Slot layout: codes [column box b][row tile i][16 rows][128 B] (so that a
-// 128-row box of column b lands on all 8 row tiles at once; 5-trit format:
+// 128-row box of column b lands on 8 row tiles at once; 5-trit format:
 // [row tile i][16 rows][208 B]), then scales [row tile i][16 rows][8 groups]
 // FP16.
 template <int FMT>
 constexpr int tile_code_bytes() { return FMT == BQ_T5P8G128 ? 16 * kT5RowBytes : Fmt<FMT>::kBoxes * 16 * 128; }
 constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
-// Row tiles per chunk the kernel is built for: 16 for the binary format up
-// to batch 4 (each of the 16 compute warps then owns one row tile and all 8
-// groups of a stage), else 8; a call uses 16 only where a CTA owns at least
-// 16 row tiles (see make_plan).
+// Largest chunk (row tiles) a kernel is built for: 16 for the binary format
+// up to batch 4 (two row tiles per warp at NW = 8, one at NW = 16), else 8.
 template <int FMT, int NT>
 constexpr int mct() { return (FMT == BQ_Q1G128 && NT <= 2) ? 16 : kMaxChunkTiles; }
-
 
 struct Params {
     const uint16_t* x;  // [batch][K] BF16
@@ -108,8 +104,8 @@ struct Params {
     int slots;          // ring slots
     int slot_bytes;     // bytes per slot (chunk_cap row tiles)
     int scales_off;     // offset of the scale tiles within a slot
-    int chunk_cap;      // row tiles per chunk, at most (1 .. 8, or 16 for binary); column boxes
-                        // of 2-bit codes are chunk_cap * 2 KB apart in a slot
+    int chunk_cap;      // row tiles per chunk, at most; column boxes of 2-bit
+                        // codes are chunk_cap * 2 KB apart in a slot
     uint32_t x_off, red_off, lut_off, bar_off;  // shared-memory offsets
     int* status;
 };
@@ -126,7 +122,8 @@ struct Ring {
     }
 };
 
-__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kComputeWarps * 32) : "memory"); }
+template <int NW>
+__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory"); }
 
 __device__ __forceinline__ int chunk_tiles(int remaining, int cap) {
     const int c = remaining < cap ? remaining : cap;
@@ -158,23 +155,24 @@ __device__ __forceinline__ int ilog2f(float m) {
 //           bytes 6t+4, 6t+5 and trits 120+2t, 121+2t (the group's last
 //           eight trits, in bytes 24 and 25)
 // Table entry (G, t) of an n-tile, t = 2 (bb & 1) + hh for digit pair hh, with
-// e = coef - E + 16 hh and z = [hh == 0] times the group's activation sum
-// (FP32; it stands in for 2^-E sum Q, which differs by the rounding of Q):
+// e = coef - E + 16 hh and z = [hh == 0] times the group's activation sum:
 //   one factor  : {2^e, 1, z, 0}, u = (D0 + 256 D1) 2^e - z;
 //   two factors : {2^a, 2^(e-a), z, 1} when 2^e is not a normal float,
 //                 u = (D0 + 256 D1) 2^a 2^(e-a) - z.
 // Rows past the batch are prepared as zero activations (zero digits, z = 0).
 //
-// Work split: lane 4 G + t of a warp prepares group G of one stage and one
-// batch row for B-fragment thread t, i.e. the 32 activations that land in the
-// slots of thread t: k = 32 t .. 32 t + 31 (binary, 2-bit), or k = 30 t ..
-// 30 t + 29 and 120 + 2 t, 121 + 2 t (5-trit); r numbers them in that order.
-// Byte 4 m + j of the 16-byte chunk (pair P, digit d) is digit d of value
-// prep_src(P, m, j), so the lane assembles all eight of its chunks in
-// registers (a 4 x 4 byte transpose per (P, m)) and stores them whole.
+// Work split: a task is (group G, B-fragment thread t, MMA pair P) of one
+// stage and batch row: the 16 activations that land in pair P of thread t's
+// slots.  Byte 4 m + j of the 16-byte chunk (pair P, digit d) is digit d of
+// activation prep_src(P, m, j) of the thread's 32 (k = 32 t + r for binary
+// and 2-bit; k = 30 t + r, r < 30, and 120 + 2 t + (r - 30) for 5-trit), so a
+// lane assembles its four chunks in registers (a 4 x 4 byte transpose per m)
+// and stores them whole.  Lane 8 g + 2 t + P of a warp takes group 4 h + g of
+// half h of a stage; the group's eight lanes share the maximum and the sum
+// through shuffles.
 template <int FMT>
 __device__ __forceinline__ constexpr int prep_src(int P, int m, int j) {
-    if (FMT == BQ_Q1G128) return 8 * j + 4 * P + m;                    // k = 32t + 8j + 2q + h
+    if (FMT == BQ_Q1G128) return 8 * j + 4 * P + m;                        // k = 32t + 8j + 2q + h
     if (FMT == BQ_T2G128) return 16 * (m & 1) + 4 * j + 2 * P + (m >> 1);  // k = 32t + 16h + 4j + q
     if (P == 0) return 5 * m + j;                 // digits 0..3 of bytes 6t .. 6t+3
     if (m < 2) return 20 + 5 * m + j;             // digits 0..3 of bytes 6t+4, 6t+5
@@ -182,35 +180,54 @@ __device__ __forceinline__ constexpr int prep_src(int P, int m, int j) {
     return j == 0 ? 24 : j == 1 ? 29 : 28 + j;    // digit 4 of 6t+4, 6t+5; trits 120+2t, 121+2t
 }
 
-// Left shift taking the rounded value to the operand byte stream b:
-// Q = round(x 2^es) 2^kQuantShift, and the class of value r divides Q by
-// 2^(r mod 8) (binary) or 4^(r mod 4) (2-bit).
+// Class of activation (P, m, j) as a left shift: the operand's power of two
+// (binary: the bit's weight 2^class; 2-bit: 4^class).
 template <int FMT>
-__device__ __forceinline__ constexpr int prep_shift(int r) {
-    return FMT == BQ_Q1G128 ? 7 - (r & 7) : FMT == BQ_T2G128 ? 6 - 2 * (r & 3) : 0;
+__device__ __forceinline__ int prep_class_shift(int P, int m) {
+    if (FMT == BQ_Q1G128) return 4 * P + m;               // (8j + 4P + m) mod 8
+    if (FMT == BQ_T2G128) return 2 * (2 * P + (m >> 1));  // 2 * ((16(m&1) + 4j + 2P + (m>>1)) mod 4)
+    return 0;
 }
 
-// The lane's 32 activations as 16 words of two BF16 values (value r in half
-// r & 1 of word r >> 1); xg is the group's first activation (16-byte aligned).
+// The task's activations.  Binary: the four runs k = 32t + 8j + 4P + {0..3}
+// (value 4j + m of raw); 2-bit: the pairs k = 32t + 4j + 2P + {0,1} and
+// 32t + 16 + 4j + 2P + {0,1} (words 2j and 2j + 1 of raw); 5-trit: all 32
+// activations of thread t (value r of raw, both pairs).  xg is the group's
+// first activation (16-byte aligned).
 template <int FMT>
-__device__ __forceinline__ void load_lane_x(const uint16_t* xg, int t, uint32_t (&raw)[16]) {
-    if (FMT == BQ_T5P8G128) {
+__device__ __forceinline__ void load_task_x(const uint16_t* xg, int t, int P, uint32_t (&raw)[16]) {
+    if (FMT == BQ_Q1G128) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
+            raw[2 * j] = v.x;
+            raw[2 * j + 1] = v.y;
+        }
+    } else if (FMT == BQ_T2G128) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            raw[2 * j] = __ldg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 4 * j + 2 * P));
+            raw[2 * j + 1] = __ldg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 16 + 4 * j + 2 * P));
+        }
+    } else {
         const uint32_t* src = reinterpret_cast<const uint32_t*>(xg + 30 * t);  // 60 t bytes: 4-byte aligned
 #pragma unroll
         for (int i = 0; i < 15; ++i) raw[i] = __ldg(src + i);
         raw[15] = __ldg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
-    } else {
-        const uint4* src = reinterpret_cast<const uint4*>(xg + 32 * t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint4 v = __ldg(src + i);
-            raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
-        }
     }
 }
 
 __device__ __forceinline__ float raw_value(const uint32_t (&raw)[16], int r) {
     return __uint_as_float((r & 1) ? (raw[r >> 1] & 0xFFFF0000u) : (raw[r >> 1] << 16));
+}
+
+// Activation (P, m, j) of the task (see load_task_x).
+template <int FMT>
+__device__ __forceinline__ float task_value(const uint32_t (&raw)[16], int P, int m, int j) {
+    if (FMT == BQ_Q1G128) return raw_value(raw, 4 * j + m);
+    if (FMT == BQ_T2G128) return raw_value(raw, 2 * (2 * j + (m & 1)) + (m >> 1));
+    const float v0 = raw_value(raw, prep_src<FMT>(0, m, j)), v1 = raw_value(raw, prep_src<FMT>(1, m, j));
+    return P ? v1 : v0;
 }
 
 // Rows 0 .. 3 of a 4 x 4 byte matrix given as rows a, b, c, e, returned as
@@ -224,60 +241,67 @@ __device__ __forceinline__ void transpose_bytes(uint32_t a, uint32_t b, uint32_t
     out[3] = __byte_perm(ab_hi, ce_hi, 0x7632);
 }
 
-// One lane's share (group G, thread t, batch row parity hb of the n-tile at
-// xt): its eight B-fragment chunks and, on t = 0 / 1, the table entry of digit
-// pair t.  All four lanes of the group run it together (shuffles).
+// One lane's task (group G, thread t, pair P, batch row parity hb of the
+// n-tile at xt): its four B-fragment chunks and, on P = 0, t < 2, the table
+// entry of digit pair t.  All eight lanes of the group run it together
+// (shuffles).
 template <int FMT, int LANES>
-__device__ __forceinline__ void prep_lane(uint8_t* xt, int G, int t, int hb, const uint32_t (&raw)[16]) {
+__device__ __forceinline__ void prep_task(uint8_t* xt, int G, int t, int P, int hb, const uint32_t (&raw)[16]) {
     // group maximum of |x| on the BF16 bits (a larger magnitude has larger bits)
+    constexpr int kWords = FMT == BQ_T5P8G128 ? 16 : 8;
     uint32_t mx = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, raw[i] & 0x7FFF7FFFu);
+    for (int i = 0; i < kWords; ++i) mx = __vmaxu2(mx, raw[i] & 0x7FFF7FFFu);
     mx = max(mx & 0xFFFFu, mx >> 16);
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     const float m = __uint_as_float(mx << 16);
-    const int E = (m > 0.f) ? 29 - ilog2f(m) : 0;
-    const int es = E - Fmt<FMT>::kQuantShift;  // x * 2^es -> Q / 2^shift
-    const int e1 = max(-126, min(127, es));
-    const float p1 = exp2i(e1), p2 = exp2i(es - e1);
+    const int E = (m > 0.f) ? 29 - ilog2f(m) : 0;  // in [-98, 162]
+    // operand multipliers 2^(E - class): one factor unless 2^E leaves the
+    // normal range (largest |x| below ~2^-97), then 2^(E-127) * 2^(127-class)
+    const bool two = E > 127;
+    const float pa = exp2i(two ? E - 127 : 0);
+    const int Eb = two ? 127 : E;
+    float mul[4];
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) mul[mm] = exp2i(Eb - prep_class_shift<FMT>(P, mm));
+    const bool any_two = __any_sync(0xffffffffu, two);
     float zs = 0.0f;
-    uint8_t* xb = xt + ((G * 2) * LANES + 16 * hb + t) * 16;  // chunk (P 0, digit 0)
+    uint32_t col[4][4];  // [m][digit]
 #pragma unroll
-    for (int P = 0; P < 2; ++P) {
-        uint32_t col[4][4];  // [m][digit]
+    for (int mm = 0; mm < 4; ++mm) {
+        uint32_t w[4];
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = prep_src<FMT>(P, mm, j);
-                const float v = raw_value(raw, r);
-                zs += v;
-                const int b = __float2int_rn(v * p1 * p2) * (1 << prep_shift<FMT>(r));
-                // balanced base-256 digits of b (|b| <= 2^30) are the bytes of
-                // (b + 0x808080) ^ 0x808080 (the xor is applied after the transpose)
-                w[j] = (uint32_t)b + 0x808080u;
-            }
-            transpose_bytes(w[0], w[1], w[2], w[3], col[mm]);
+        for (int j = 0; j < 4; ++j) {
+            const float v = task_value<FMT>(raw, P, mm, j);
+            zs += v;
+            const int b = __float2int_rn(any_two ? (v * pa) * mul[mm] : v * mul[mm]);
+            // balanced base-256 digits of b (|b| <= 2^30) are the bytes of
+            // (b + 0x808080) ^ 0x808080 (the xor is applied after the transpose)
+            w[j] = (uint32_t)b + 0x808080u;
         }
-#pragma unroll
-        for (int d = 0; d < 4; ++d) {
-            const uint32_t f = d < 3 ? 0x80808080u : 0u;
-            *reinterpret_cast<uint4*>(xb + (P * LANES + 4 * d) * 16) =
-                make_uint4(col[0][d] ^ f, col[1][d] ^ f, col[2][d] ^ f, col[3][d] ^ f);
-        }
+        transpose_bytes(w[0], w[1], w[2], w[3], col[mm]);
     }
-    // z = the group's activation sum (FP32, fixed order)
+    uint8_t* xb = xt + ((G * 2 + P) * LANES + 16 * hb + t) * 16;  // chunk (P, digit 0)
+#pragma unroll
+    for (int d = 0; d < 4; ++d) {
+        const uint32_t f = d < 3 ? 0x80808080u : 0u;
+        *reinterpret_cast<uint4*>(xb + 4 * d * 16) =
+            make_uint4(col[0][d] ^ f, col[1][d] ^ f, col[2][d] ^ f, col[3][d] ^ f);
+    }
+    // z = the group's activation sum (FP32, fixed order: each lane's 16 in
+    // order, then pairs of lanes by xor 1, 2, 4)
     zs += __shfl_xor_sync(0xffffffffu, zs, 1);
     zs += __shfl_xor_sync(0xffffffffu, zs, 2);
-    if (t < 2) {
+    zs += __shfl_xor_sync(0xffffffffu, zs, 4);
+    if (P == 0 && t < 2) {
         const int hh = t;  // digit pair (0,1) or (2,3)
         const int e = Fmt<FMT>::kCoefShift - E + 16 * hh;
-        const bool two = Fmt<FMT>::kCoefShift - E < -126;
-        const int a = two ? max(-60, min(60, e)) : e;
+        const bool tf = Fmt<FMT>::kCoefShift - E < -126;
+        const int a = tf ? max(-60, min(60, e)) : e;
         float4* tabp = reinterpret_cast<float4*>(xt + kGroupsPerStage * 2 * LANES * 16) + G * 4 + 2 * hb + hh;
-        *tabp = make_float4(exp2i(a), exp2i(e - a), hh == 0 ? zs : 0.0f, two ? 1.0f : 0.0f);
+        *tabp = make_float4(exp2i(a), exp2i(e - a), hh == 0 ? zs : 0.0f, tf ? 1.0f : 0.0f);
     }
 }
 
@@ -307,19 +331,44 @@ __device__ __forceinline__ void t5_row(const uint8_t* p, const uint32_t* lut, in
     R[7] = c4[4] | (c4[5] << 8) | (x01 << 16);
 }
 
+// GPW consecutive FP16 scales (the warp's groups of one row and stage) as
+// packed pairs.
+template <int GPW>
+__device__ __forceinline__ void load_scales(const uint8_t* p, uint32_t (&s)[(GPW + 1) / 2]) {
+    if constexpr (GPW == 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
+    } else if constexpr (GPW == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        s[0] = v.x; s[1] = v.y;
+    } else if constexpr (GPW == 2) {
+        s[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else {
+        s[0] = *reinterpret_cast<const uint16_t*>(p);
+    }
+}
+
+__device__ __forceinline__ float scale_of(const uint32_t* s, int i) {
+    return __half2float(__ushort_as_half((uint16_t)((i & 1) ? (s[i >> 1] >> 16) : (s[i >> 1] & 0xFFFFu))));
+}
+
 // ------------------------------------------------------------ one chunk
-// CT row tiles (16 rows each) starting at row tile rt, all stages.  Warp w
-// takes row tile w / WPR and groups G = w % WPR + WPR i (i < 8 / WPR), with
-// WPR = min(16 / CT, 8) warps per row tile; warps past CT row tiles only
-// keep the stage barriers going.
-template <int FMT, int NT, int LANES, int CT>
+// CT row tiles (16 rows each) starting at row tile rt, all stages.
+//   CT >= NW: warp w takes row tiles w + NW i (i < TPW = CT / NW), all groups;
+//   CT <  NW: warp w takes row tile w / WPR (WPR = NW / CT warps per row tile,
+//             at most 8; warps past CT row tiles only keep the stage barriers
+//             going) and the GPW = 8 / WPR groups G = GPW (w % WPR) + i.
+template <int FMT, int NT, int LANES, int NW, int CT>
 __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, Ring& rp,
                           int warp, int lane) {
-    constexpr int WPR = (kComputeWarps / CT) < kGroupsPerStage ? (kComputeWarps / CT) : kGroupsPerStage;
+    constexpr int TPW = CT >= NW ? CT / NW : 1;
+    constexpr int WPR = CT >= NW ? 1 : ((NW / CT) < kGroupsPerStage ? (NW / CT) : kGroupsPerStage);
     constexpr int GPW = kGroupsPerStage / WPR;  // groups per warp and stage
     constexpr int TCB = tile_code_bytes<FMT>();
+    constexpr int TSTRIDE = FMT == BQ_T5P8G128 ? TCB : 2048;  // code bytes between row tiles of a column box
     constexpr int X_NT = x_nt_bytes(LANES);
-    const int my_rt = warp / WPR, gsub = warp % WPR;
+    const int my_rt = CT >= NW ? warp : warp / WPR;
+    const int gsub = CT >= NW ? 0 : warp % WPR;
     const bool active = my_rt < CT;
     const int g = lane >> 2, t = lane & 3;
     // at batch 1 the upper 16 lanes (columns of a second batch row) read the
@@ -328,18 +377,25 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     const uint8_t* xres = smem + p.x_off;
     const uint32_t* lut = reinterpret_cast<const uint32_t*>(smem + p.lut_off);
     const uint32_t t5sel = (uint32_t)(2 * t) | ((uint32_t)(2 * t + 1) << 4);
-    float yacc[NT][2];
+    float yacc[TPW][NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) yacc[nt][0] = yacc[nt][1] = 0.0f;
+    for (int tp = 0; tp < TPW; ++tp)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) yacc[tp][nt][0] = yacc[tp][nt][1] = 0.0f;
     // this warp's GPW groups of stage st (ring slot `slot`), added into yacc
     auto stage = [&](int st, int slot) {
         const uint8_t* sb = smem + slot * p.slot_bytes;
-        const uint8_t* codes_t = sb + my_rt * 2048;  // column box 0 of this row tile
-        const uint16_t* scales_t = reinterpret_cast<const uint16_t*>(sb + p.scales_off + my_rt * kTileScaleBytes);
         const uint8_t* xs = xres + (size_t)st * NT * X_NT;
+        uint32_t sc[TPW][2][(GPW + 1) / 2];
+#pragma unroll
+        for (int tp = 0; tp < TPW; ++tp) {
+            const uint8_t* srow = sb + p.scales_off + (my_rt + NW * tp) * kTileScaleBytes + gsub * GPW * 2;
+            load_scales<GPW>(srow + g * 16, sc[tp][0]);
+            load_scales<GPW>(srow + (g + 8) * 16, sc[tp][1]);
+        }
 #pragma unroll
         for (int gi = 0; gi < GPW; ++gi) {
-            const int G = gsub + WPR * gi;
+            const int G = gsub * GPW + gi;
             uint4 bf[NT][2];
             float4 tab[NT];
 #pragma unroll
@@ -349,82 +405,85 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                 for (int h = 0; h < 2; ++h) bf[nt][h] = *reinterpret_cast<const uint4*>(xt + ((G * 2 + h) * LANES + blane) * 16);
                 tab[nt] = *reinterpret_cast<const float4*>(xt + kGroupsPerStage * 2 * LANES * 16 + (G * 4 + t) * 16);
             }
-            int acc[NT][4];
-            if (FMT == BQ_Q1G128) {
-                const int off = ((G ^ g) << 4) + 4 * t;
-                const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_t + g * 128 + off);
-                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_t + (g + 8) * 128 + off);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
+            for (int tp = 0; tp < TPW; ++tp) {
+                const uint8_t* codes_t = sb + (my_rt + NW * tp) * TSTRIDE;  // column box 0 of this row tile
+                int acc[NT][4];
+                if (FMT == BQ_Q1G128) {
+                    const int off = ((G ^ g) << 4) + 4 * t;
+                    const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_t + g * 128 + off);
+                    const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_t + (g + 8) * 128 + off);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
-                        const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
-                        if (q == 0)
-                            ptx::mma_u8s8_init(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1, 0);
-                        else
-                            ptx::mma_u8s8(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t m0 = 0x01010101u << (2 * q), m1 = 0x01010101u << (2 * q + 1);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            if (q == 0)
+                                ptx::mma_u8s8_init(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1, 0);
+                            else
+                                ptx::mma_u8s8(acc[nt], w0 & m0, w1 & m0, w0 & m1, w1 & m1, b0, b1);
+                        }
+                    }
+                } else if (FMT == BQ_T5P8G128) {
+                    const uint8_t* g0 = codes_t + g * kT5RowBytes + 26 * G;
+                    uint32_t R0[8], R1[8];
+                    t5_row(g0, lut, t, lane, t5sel, R0);
+                    t5_row(g0 + 8 * kT5RowBytes, lut, t, lane, t5sel, R1);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            if (q == 0)
+                                ptx::mma_u8s8_init(acc[nt], R0[0], R1[0], R0[1], R1[1], b0, b1, 0);
+                            else
+                                ptx::mma_u8s8(acc[nt], R0[2 * q], R1[2 * q], R0[2 * q + 1], R1[2 * q + 1], b0, b1);
+                        }
+                    }
+                } else {
+                    // words 2t, 2t+1 of the row's 32-byte group
+                    const uint8_t* box = codes_t + (G >> 2) * (p.chunk_cap * 2048);  // column box 1 after chunk_cap tiles
+                    const int chunk = 2 * (G & 3) + (t >> 1);
+                    const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
+                    const uint2 wr0 = *reinterpret_cast<const uint2*>(box + g * 128 + off);
+                    const uint2 wr1 = *reinterpret_cast<const uint2*>(box + (g + 8) * 128 + off);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t m = 0x03030303u << (2 * q);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
+                            const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
+                            if (q == 0)
+                                ptx::mma_u8s8_init(acc[nt], wr0.x & m, wr1.x & m, wr0.y & m, wr1.y & m, b0, b1, 0);
+                            else
+                                ptx::mma_u8s8(acc[nt], wr0.x & m, wr1.x & m, wr0.y & m, wr1.y & m, b0, b1);
+                        }
                     }
                 }
-            } else if (FMT == BQ_T5P8G128) {
-                const uint8_t* g0 = sb + my_rt * TCB + g * kT5RowBytes + 26 * G;
-                uint32_t R0[8], R1[8];
-                t5_row(g0, lut, t, lane, t5sel, R0);
-                t5_row(g0 + 8 * kT5RowBytes, lut, t, lane, t5sel, R1);
+                const float s0 = scale_of(sc[tp][0], gi), s1 = scale_of(sc[tp][1], gi);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
-                        const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
-                        if (q == 0)
-                            ptx::mma_u8s8_init(acc[nt], R0[0], R1[0], R0[1], R1[1], b0, b1, 0);
-                        else
-                            ptx::mma_u8s8(acc[nt], R0[2 * q], R1[2 * q], R0[2 * q + 1], R1[2 * q + 1], b0, b1);
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    // D0 + 256 D1 is exact in int32 (|D0|, |D1| <= 2^21)
+                    const float v0 = (float)(acc[nt][0] + (acc[nt][1] << 8));
+                    const float v1 = (float)(acc[nt][2] + (acc[nt][3] << 8));
+                    // (with one factor tab.y = 1: the same rounding as fmaf(v, 2^e, -z))
+                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                    yacc[tp][nt][0] = fmaf(s0, u0, yacc[tp][nt][0]);
+                    yacc[tp][nt][1] = fmaf(s1, u1, yacc[tp][nt][1]);
                 }
-            } else {
-                // words 2t, 2t+1 of the row's 32-byte group
-                const uint8_t* box = codes_t + (G >> 2) * (p.chunk_cap * 2048);  // column box 1 after chunk_cap tiles
-                const int chunk = 2 * (G & 3) + (t >> 1);
-                const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
-                const uint2 wr0 = *reinterpret_cast<const uint2*>(box + g * 128 + off);
-                const uint2 wr1 = *reinterpret_cast<const uint2*>(box + (g + 8) * 128 + off);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t m = 0x03030303u << (2 * q);
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const uint32_t b0 = (q & 1) ? bf[nt][q >> 1].z : bf[nt][q >> 1].x;
-                        const uint32_t b1 = (q & 1) ? bf[nt][q >> 1].w : bf[nt][q >> 1].y;
-                        if (q == 0)
-                            ptx::mma_u8s8_init(acc[nt], wr0.x & m, wr1.x & m, wr0.y & m, wr1.y & m, b0, b1, 0);
-                        else
-                            ptx::mma_u8s8(acc[nt], wr0.x & m, wr1.x & m, wr0.y & m, wr1.y & m, b0, b1);
-                    }
-                }
-            }
-            const float s0 = half_bits_to_float(scales_t[g * kGroupsPerStage + G]);
-            const float s1 = half_bits_to_float(scales_t[(g + 8) * kGroupsPerStage + G]);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                // D0 + 256 D1 is exact in int32 (|D0|, |D1| <= 2^21)
-                const float v0 = (float)(acc[nt][0] + (acc[nt][1] << 8));
-                const float v1 = (float)(acc[nt][2] + (acc[nt][3] << 8));
-                // (with one factor tab.y = 1: the same rounding as fmaf(v, 2^e, -z))
-                const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                yacc[nt][0] = fmaf(s0, u0, yacc[nt][0]);
-                yacc[nt][1] = fmaf(s1, u1, yacc[nt][1]);
             }
         }
     };
-    // Binary format: where a warp has fewer than four groups (over all
-    // n-tiles) per stage, stages are taken U at a time, so that U independent
-    // MMA chains run between two barrier waits, if the ring holds 2 U slots.
-    // (The longer 2-bit and 5-trit stage bodies measured slower this way.)
-    constexpr int U = (FMT != BQ_Q1G128 || GPW * NT >= 4) ? 1 : 4 / (GPW * NT);
+    // Binary format: where a warp has fewer than four (group, n-tile) pairs per
+    // stage, stages are taken U at a time, so that U independent MMA chains run
+    // between two barrier waits, if the ring holds 2 U slots.  (The longer
+    // 2-bit and 5-trit stage bodies measured slower this way.)
+    constexpr int U = (FMT != BQ_Q1G128 || GPW * NT * TPW >= 4) ? 1 : 4 / (GPW * NT * TPW);
     const int ustep = (U > 1 && p.slots >= 2 * U) ? U : 1;  // (the producer keeps U slots ahead)
     bool alive = true;
     for (int st = 0; st < p.stages; st += ustep) {
@@ -465,17 +524,19 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     }
     // digit pairs (t, t^1) -> one value per (batch row, row) on even t
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int tp = 0; tp < TPW; ++tp)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) yacc[nt][r] += __shfl_xor_sync(0xffffffffu, yacc[nt][r], 1);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) yacc[tp][nt][r] += __shfl_xor_sync(0xffffffffu, yacc[tp][nt][r], 1);
     if (WPR > 1) {
         // partial sums of the warps sharing a row tile, added in warp order
         float* red = reinterpret_cast<float*>(smem + p.red_off);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int r = 0; r < 2; ++r) red[((warp * 32 + lane) * NT + nt) * 2 + r] = yacc[nt][r];
-        bar_compute();
+            for (int r = 0; r < 2; ++r) red[((warp * 32 + lane) * NT + nt) * 2 + r] = yacc[0][nt][r];
+        bar_compute<NW>();
         if (active && gsub == 0) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
@@ -484,25 +545,27 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                     float s = 0.0f;
 #pragma unroll
                     for (int j = 0; j < WPR; ++j) s += red[(((warp + j) * 32 + lane) * NT + nt) * 2 + r];
-                    yacc[nt][r] = s;
+                    yacc[0][nt][r] = s;
                 }
         }
-        bar_compute();  // red is reused by the next chunk
+        bar_compute<NW>();  // red is reused by the next chunk
     }
     if (active && gsub == 0 && (t & 1) == 0) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int tp = 0; tp < TPW; ++tp)
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int bb = nt * 2 + (t >> 1);
-                const int64_t row = (int64_t)(rt + my_rt) * 16 + g + 8 * r;
-                if (bb < p.batch && row < p.n) {
-                    if (p.y_dtype == BQ_F32)
-                        static_cast<float*>(p.y)[bb * p.n + row] = yacc[nt][r];
-                    else
-                        static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[nt][r]);
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int bb = nt * 2 + (t >> 1);
+                    const int64_t row = (int64_t)(rt + my_rt + NW * tp) * 16 + g + 8 * r;
+                    if (bb < p.batch && row < p.n) {
+                        if (p.y_dtype == BQ_F32)
+                            static_cast<float*>(p.y)[bb * p.n + row] = yacc[tp][nt][r];
+                        else
+                            static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(yacc[tp][nt][r]);
+                    }
                 }
-            }
     }
     return alive;
 }
@@ -514,29 +577,31 @@ struct Maps {
     CUtensorMap codes16, scales16, codes128, scales128;
 };
 
-template <int FMT, int NT, int LANES>
-__global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_constant__ Maps tm, const Params p) {
+template <int FMT, int NT, int LANES, int NW>
+__global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
+    gemv_rows_kernel(const __grid_constant__ Maps tm, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = ptx::align_smem<1024>(smem_raw);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+    const uint32_t bar_off = p.bar_off;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + bar_off);
     uint64_t* empty = full + kMaxSlots;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = gridDim.x, c = blockIdx.x;
-    // row tiles [rt0, rt1): the first row_tiles % C CTAs take one extra
-    const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
-    const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.slots; ++i) {
             ptx::mbar_init(&full[i], 1);
-            ptx::mbar_init(&empty[i], kComputeWarps);
+            ptx::mbar_init(&empty[i], NW);
         }
         ptx::fence_barrier_init();
     }
     __syncthreads();
+    // row tiles [rt0, rt1): the first row_tiles % C CTAs take one extra
+    const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
+    const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
     ptx::pdl_launch_dependents();
 
-    if (warp == kProducerWarp) {
+    if (warp == NW) {
         // ------------------------------------------------ weight producer
         // lane 0 waits for the slot and posts the byte count; the copies of a
         // stage are then issued by several lanes at once (one row tile, or one
@@ -618,28 +683,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
     if (FMT == BQ_T5P8G128) {
         // digit table: lut[32 v + l] = c0 | c1 << 8 | c2 << 16 | c3 << 24 of byte v
         uint32_t* lut = reinterpret_cast<uint32_t*>(smem + p.lut_off);
-        for (int i = threadIdx.x; i < 256 * 32; i += kComputeWarps * 32) {
+        for (int i = threadIdx.x; i < 256 * 32; i += NW * 32) {
             const uint32_t v = (uint32_t)i >> 5;
             lut[i] = (v % 3u) | ((v / 3u % 3u) << 8) | ((v / 9u % 3u) << 16) | ((v / 27u % 3u) << 24);
         }
     }
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
     {
-        // items (stage, batch row) i = warp + 16 j: lane 4 G + t takes group G;
-        // rows up to the n-tiles' width (zero past the batch; one row at 16 lanes)
+        // warp items (stage, batch row, half h of the stage's groups), item i
+        // on warp i % NW; lane 8 gq + 2 t + P takes group 4 h + gq.  Rows go up
+        // to the n-tiles' width (zero past the batch; one row at 16 lanes).
         constexpr int kPrepBatch = 2;
         uint8_t* xres = smem + p.x_off;
         const int rows = LANES == 16 ? 1 : 2 * NT;
-        const int items = p.stages * rows;
-        const int G = lane >> 2, t = lane & 3;
-        for (int i0 = warp; i0 < items; i0 += kComputeWarps * kPrepBatch) {
+        const int items = p.stages * rows * 2;
+        const int gq = lane >> 3, t = (lane >> 1) & 3, P = lane & 1;
+        for (int i0 = warp; i0 < items; i0 += NW * kPrepBatch) {
             uint32_t raw[kPrepBatch][16];
 #pragma unroll
             for (int j = 0; j < kPrepBatch; ++j) {
-                const int i = i0 + j * kComputeWarps;
-                const int st = i / rows, bb = i - st * rows;
+                const int i = i0 + j * NW;
+                const int sr = i >> 1, G = 4 * (i & 1) + gq;
+                const int st = sr / rows, bb = sr - st * rows;
                 if (i < items && bb < p.batch) {
-                    load_lane_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, raw[j]);
+                    load_task_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, P, raw[j]);
                 } else {
 #pragma unroll
                     for (int w = 0; w < 16; ++w) raw[j][w] = 0u;
@@ -647,56 +714,52 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(const __grid_con
             }
 #pragma unroll
             for (int j = 0; j < kPrepBatch; ++j) {
-                const int i = i0 + j * kComputeWarps;
+                const int i = i0 + j * NW;
                 if (i < items) {  // (warp-uniform)
-                    const int st = i / rows, bb = i - st * rows;
-                    prep_lane<FMT, LANES>(xres + (size_t)(st * NT + (bb >> 1)) * x_nt_bytes(LANES), G, t, bb & 1,
+                    const int sr = i >> 1, G = 4 * (i & 1) + gq;
+                    const int st = sr / rows, bb = sr - st * rows;
+                    prep_task<FMT, LANES>(xres + (size_t)(st * NT + (bb >> 1)) * x_nt_bytes(LANES), G, t, P, bb & 1,
                                           raw[j]);
                 }
             }
         }
     }
-    bar_compute();
+    bar_compute<NW>();
     Ring rp;
     rp.depth = p.slots;
     for (int r = rt0; r < rt1;) {
         const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
         bool ok;
         if (mct<FMT, NT>() >= 16 && ct == 16)
-            ok = run_chunk<FMT, NT, LANES, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 8)
-            ok = run_chunk<FMT, NT, LANES, 8>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 4)
-            ok = run_chunk<FMT, NT, LANES, 4>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
         else if (ct == 2)
-            ok = run_chunk<FMT, NT, LANES, 2>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
         else
-            ok = run_chunk<FMT, NT, LANES, 1>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
         if (!ok) break;
         r += ct;
     }
 }
 
 // ----------------------------------------------------------------- host
-
 struct Plan {
-    int nt = 0, lanes = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0, chunk_cap = 8, slot_bytes = 0, scales_off = 0;
+    int nt = 0, lanes = 0, nw = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0, chunk_cap = 8, slot_bytes = 0,
+        scales_off = 0;
     uint32_t x_off = 0, red_off = 0, lut_off = 0, bar_off = 0, smem = 0;
     bool ok = false;
 };
 
-Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
-    Plan pl;
-    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 8 && k > 0 &&
-          k % 1024 == 0 && n > 0 &&
-          n <= (int64_t)INT32_MAX - 16 && k / 4 <= (int64_t)INT32_MAX / 4 && k <= (int64_t)1 << 20))
-        return pl;
-    pl.nt = batch <= 2 ? 1 : batch <= 4 ? 2 : 4;  // n-tiles of two batch rows (5..8 -> 4)
-    pl.lanes = batch == 1 ? 16 : 32;
-    pl.stages = (int)(k / 1024);
-    pl.row_tiles = (int)((n + 15) / 16);
-    const int sms = sm_count();
-    pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
+// Shared-memory layout for NW compute warps within `limit` bytes; false if a
+// ring of two slots does not fit.
+bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
+    const int ctas_per_sm = nw == 8 ? 2 : 1;
+    const int cap_grid = sms * ctas_per_sm;
+    pl.nw = nw;
+    pl.grid = pl.row_tiles < cap_grid ? pl.row_tiles : cap_grid;
     // 16-tile chunks (binary, batch <= 4) only where a CTA owns at least 16
     // row tiles; otherwise 8-tile slots keep the ring deep.  No chunk is larger
     // than the most tiles a CTA owns (rounded down to a power of two), so
@@ -711,28 +774,54 @@ Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
-    const int64_t red = (int64_t)kComputeWarps * 32 * pl.nt * 2 * 4;
+    const int64_t red = (int64_t)nw * 32 * pl.nt * 2 * 4;
     const int64_t fixed = 1024 + x_area + red + lut + 2 * kMaxSlots * 8;
-    int64_t slots = (kSmemLimit - fixed) / slot;
+    int64_t slots = (limit - fixed) / slot;
     if (slots > kMaxSlots) slots = kMaxSlots;
-    if (slots < 2) return pl;
+    if (slots < 2) return false;
     pl.slots = (int)slots;
     pl.x_off = (uint32_t)(slots * slot);
     pl.red_off = (uint32_t)(pl.x_off + x_area);
     pl.lut_off = (uint32_t)(pl.red_off + red);
     pl.bar_off = (uint32_t)(pl.lut_off + lut);
     pl.smem = (uint32_t)(1024 + pl.bar_off + 2 * kMaxSlots * 8);
-    pl.ok = true;
+    return true;
+}
+
+Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
+    Plan pl;
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 8 && k > 0 &&
+          k % 1024 == 0 && n > 0 &&
+          n <= (int64_t)INT32_MAX - 16 && k / 4 <= (int64_t)INT32_MAX / 4 && k <= (int64_t)1 << 20))
+        return pl;
+    pl.nt = batch <= 2 ? 1 : batch <= 4 ? 2 : 4;  // n-tiles of two batch rows (5..8 -> 4)
+    pl.lanes = batch == 1 ? 16 : 32;
+    pl.stages = (int)(k / 1024);
+    pl.row_tiles = (int)((n + 15) / 16);
+    const int sms = sm_count();
+    // Two CTAs per SM (8 compute warps, half the shared memory each) for the
+    // largest matrices (at least 32 row tiles per SM), where the activation
+    // operand leaves room for a ring; else one CTA of 16 compute warps per SM.
+    // (Measured on B200: the half-SM shape on every call let each call's CTAs
+    // prefetch under the previous call, but the 8-warp compute of the small
+    // and medium matrices lost more than that gained; on the largest matrices
+    // two 8-warp CTAs per SM, each with two row tiles per warp, are faster.)
+    if (pl.nt == 1 && pl.row_tiles >= 32 * sms && layout(pl, fmt, 8, kSmemHalf, sms)) {
+        pl.ok = true;
+        return pl;
+    }
+    pl.ok = layout(pl, fmt, 16, kSmemFull, sms);
     return pl;
 }
 
-template <int FMT, int NT, int LANES>
+template <int FMT, int NT, int LANES, int NW>
 cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
                          int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     {
-        const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_rows_kernel<FMT, NT, LANES>), kSmemLimit);
+        const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_rows_kernel<FMT, NT, LANES, NW>),
+                                                  NW == 8 ? kSmemHalf : kSmemFull);
         if (e != cudaSuccess) return e;
     }
     const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : (FMT == BQ_T2G128) ? k / 4 : (k / 128) * 26;
@@ -788,14 +877,27 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     attr.val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads_of<NW>());
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = s;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<FMT, NT, LANES>, tm, prm);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<FMT, NT, LANES, NW>, tm, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
+                       int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
+    if (pl.nw == 8) {
+        if (batch == 1) return launch_typed<FMT, 1, 16, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        return launch_typed<FMT, 1, 32, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    }
+    if (batch == 1) return launch_typed<FMT, 1, 16, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.nt == 1) return launch_typed<FMT, 1, 32, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.nt == 2) return launch_typed<FMT, 2, 32, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return launch_typed<FMT, 4, 32, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 }  // namespace rows
@@ -806,22 +908,9 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s) {
     const rows::Plan pl = rows::make_plan(fmt, n, k, batch);
     if (!pl.ok) return cudaErrorInvalidValue;
-    if (fmt == BQ_Q1G128) {
-        if (batch == 1) return rows::launch_typed<BQ_Q1G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        if (pl.nt == 1) return rows::launch_typed<BQ_Q1G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        if (pl.nt == 2) return rows::launch_typed<BQ_Q1G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        return rows::launch_typed<BQ_Q1G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    }
-    if (fmt == BQ_T2G128) {
-        if (batch == 1) return rows::launch_typed<BQ_T2G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        if (pl.nt == 1) return rows::launch_typed<BQ_T2G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        if (pl.nt == 2) return rows::launch_typed<BQ_T2G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-        return rows::launch_typed<BQ_T2G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    }
-    if (batch == 1) return rows::launch_typed<BQ_T5P8G128, 1, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    if (pl.nt == 1) return rows::launch_typed<BQ_T5P8G128, 1, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    if (pl.nt == 2) return rows::launch_typed<BQ_T5P8G128, 2, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    return rows::launch_typed<BQ_T5P8G128, 4, 32>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (fmt == BQ_Q1G128) return rows::launch_fmt<BQ_Q1G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (fmt == BQ_T2G128) return rows::launch_fmt<BQ_T2G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return rows::launch_fmt<BQ_T5P8G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 }  // namespace bq
