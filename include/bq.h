@@ -175,6 +175,50 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
 bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                           const uint16_t* x, int batch, void* y, int y_dtype, void* stream);
 
+/* --------------------------------------------------------- layer chains */
+/* One product of a chain (see bq_gemv_chain).  All pointers are device
+ * pointers; codes/scales/x 16-byte aligned as for bq_gemv. */
+typedef struct {
+    const uint8_t* codes;   /* W, N x K, the chain's format */
+    const uint16_t* scales; /* FP16 [N][K/128] */
+    int64_t n, k;           /* K % 1024 == 0 */
+    const uint16_t* x;      /* BF16 [batch][K]; may be an earlier step's y */
+    void* y;                /* swiglu == 0: [batch][N] of y_dtype; swiglu == 1: BF16 [batch][N/2] */
+    int y_dtype;            /* BQ_BF16 or BQ_F32 (swiglu == 0); a y that a later step
+                               reads as its x must be BQ_BF16 */
+    int swiglu;             /* 0: y = W x.  1: W = [gate; up] (N = 2 I, I % 16 == 0):
+                               y[b][j] = BF16_RNE(silu(g_j) * u_j), g = W_gate x,
+                               u = W_up x, silu(v) = v / (1 + e^-v) */
+} bq_chain_step;
+
+#define BQ_MAX_CHAIN_STEPS 8
+
+/* Workspace bytes of bq_gemv_chain: its grid-barrier counters (256). */
+int64_t bq_gemv_chain_workspace_bytes(void);
+
+/* The products of one decoder layer, in order, in ONE persistent launch ("1-bit
+ * Bonsai 8B" notes, Table 1: the attention projections and the SwiGLU
+ * feed-forward of each block; section 2: decode is bound by streaming the
+ * weights).  steps[0..nsteps) (HOST array, read during the call) run one
+ * after another with a device-wide barrier between them: every step sees all
+ * outputs of the steps before it, so a step's x may be an earlier step's y (for
+ * example the gated MLP: gate|up with swiglu = 1 writing act, then down with
+ * x = act).  Each product is the bq_gemv product (same tolerance); a SwiGLU
+ * step rounds its output once, to BF16.  One CTA per SM streams every step's
+ * weights back to back, so the weights of the next step arrive while the
+ * current one computes.
+ * fmt for all steps; 1 <= nsteps <= BQ_MAX_CHAIN_STEPS; batch 1..8 (limited by
+ * shared memory: the activation operand of the largest K must fit, else
+ * BQ_ERR_SHAPE).
+ * workspace: >= bq_gemv_chain_workspace_bytes() device bytes, 16-byte aligned,
+ * ZERO-FILLED before its first use; every call leaves it zero.  Calls that
+ * share a workspace must not overlap on the GPU.  After bq_check() reports
+ * BQ_ERR_TIMEOUT, zero it again.
+ * The launch is cooperative: it fails (BQ_ERR_CUDA) where one CTA per SM
+ * cannot be resident.  Asynchronous on `stream`. */
+bq_status bq_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------- GEMM */
 /* Workspace bytes bq_gemm needs for T tokens (0 if none); -1 if invalid. */
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t);

@@ -29,10 +29,19 @@ EXPORTED = [
     "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8",
     "bq_gemv_workspace_bytes", "bq_gemv_launches", "bq_gemv", "bq_gemv_noalloc",
     "bq_gemm_workspace_bytes", "bq_gemm_launches", "bq_gemm",
+    "bq_gemv_chain_workspace_bytes", "bq_gemv_chain",
     "bq_check", "bq_debug_wait_timeout", "bq_status_string", "bq_version",
 ]
 
 _lib = None
+BQ_MAX_CHAIN_STEPS = 8
+
+
+class ChainStep(ctypes.Structure):
+    """bq_chain_step of bq.h (device pointers)."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("n", ctypes.c_int64),
+                ("k", ctypes.c_int64), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int),
+                ("swiglu", ctypes.c_int)]
 
 
 class BQError(RuntimeError):
@@ -65,6 +74,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]; L.bq_gemm_workspace_bytes.restype = i64
     L.bq_gemm_launches.argtypes = [i32, i64, i64, i64]; L.bq_gemm_launches.restype = i32
     L.bq_gemm.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]; L.bq_gemm.restype = i32
+    L.bq_gemv_chain_workspace_bytes.argtypes = []; L.bq_gemv_chain_workspace_bytes.restype = i64
+    L.bq_gemv_chain.argtypes = [i32, ctypes.POINTER(ChainStep), i32, i32, vp, sz, vp]
+    L.bq_gemv_chain.restype = i32
     L.bq_check.argtypes = [vp]; L.bq_check.restype = i32
     L.bq_debug_wait_timeout.argtypes = [i64, vp]; L.bq_debug_wait_timeout.restype = i32
     L.bq_status_string.argtypes = [i32]; L.bq_status_string.restype = ctypes.c_char_p
@@ -222,6 +234,37 @@ def bq_gemm(fmt, codes, scales, n: int, k: int, x, y=None, workspace=None, strea
                         _ptr(workspace), wsb, _stream(stream))
     _check(st, "bq_gemm")
     return y
+
+
+# ------------------------------------------------------------------ chains
+def bq_gemv_chain_workspace_bytes() -> int:
+    return int(load().bq_gemv_chain_workspace_bytes())
+
+
+def bq_gemv_chain(fmt, steps, workspace=None, stream=None):
+    """Run the products of `steps` in order in one persistent launch (see bq.h).
+    steps: list of dicts with keys codes, scales, n, k, x (BF16 [batch][K] CUDA
+    tensor), y (output tensor: float32 for F32 output, else BF16) and optionally
+    swiglu (bool).  workspace: a zero-filled CUDA uint8 tensor of >=
+    bq_gemv_chain_workspace_bytes() bytes, reused across calls (a fresh zeroed
+    one is made when None)."""
+    import torch
+    f = _fmt(fmt)
+    arr = (ChainStep * len(steps))()
+    batch = None
+    for i, st in enumerate(steps):
+        x = st["x"]
+        b = x.shape[0] if x.dim() == 2 else 1
+        batch = b if batch is None else batch
+        ydt = BQ_F32 if st["y"].dtype == torch.float32 else BQ_BF16
+        arr[i] = ChainStep(st["codes"].data_ptr(), st["scales"].data_ptr(), int(st["n"]), int(st["k"]),
+                           x.data_ptr(), st["y"].data_ptr(), ydt, 1 if st.get("swiglu") else 0)
+    if workspace is None:
+        workspace = torch.zeros(bq_gemv_chain_workspace_bytes(), dtype=torch.uint8, device=steps[0]["x"].device)
+    wsb = workspace.numel() * workspace.element_size()
+    st = load().bq_gemv_chain(f, arr, len(steps), int(batch or 0), _ptr(workspace), wsb, _stream(stream))
+    _check(st, "bq_gemv_chain")
+    return workspace
 
 
 # ------------------------------------------------------------------ errors

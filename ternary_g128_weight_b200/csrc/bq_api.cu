@@ -231,6 +231,31 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
+int64_t bq_gemv_chain_workspace_bytes(void) { return 256; }
+
+bq_status bq_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!fmt_ok(fmt)) return BQ_ERR_FORMAT;
+    if (!steps) return BQ_ERR_NULL;
+    if (nsteps < 1 || nsteps > BQ_MAX_CHAIN_STEPS || batch < 1 || batch > BQ_MAX_BATCH) return BQ_ERR_SHAPE;
+    for (int i = 0; i < nsteps; ++i) {
+        const bq_chain_step& st = steps[i];
+        const bq_status v = validate_matrix(fmt, st.codes, st.scales, st.n, st.k);
+        if (v != BQ_OK) return v;
+        if (st.swiglu != 0 && st.swiglu != 1) return BQ_ERR_FORMAT;
+        if (!st.swiglu && st.y_dtype != BQ_BF16 && st.y_dtype != BQ_F32) return BQ_ERR_FORMAT;
+        if (st.n == 0 || st.k == 0) return BQ_ERR_SHAPE;
+        if (!st.x || !st.y) return BQ_ERR_NULL;
+        if (!aligned(st.x, 16) || !aligned(st.y, 16)) return BQ_ERR_ALIGN;
+    }
+    if (!gemv_chain_eligible(fmt, steps, nsteps, batch)) return BQ_ERR_SHAPE;
+    if (!workspace || workspace_bytes < (size_t)bq_gemv_chain_workspace_bytes()) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return BQ_ERR_ALIGN;
+    const cudaError_t e =
+        launch_gemv_chain(fmt, steps, nsteps, batch, static_cast<unsigned int*>(workspace), as_stream(stream));
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 bq_status bq_check(void* stream) {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return BQ_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;

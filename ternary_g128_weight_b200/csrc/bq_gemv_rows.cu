@@ -108,6 +108,11 @@ struct Params {
                         // codes are chunk_cap * 2 KB apart in a slot
     uint32_t x_off, red_off, lut_off, bar_off;  // shared-memory offsets
     int* status;
+    // SwiGLU epilogue (persistent chain kernel only; 0 otherwise): the W rows
+    // are [gate; up], a CTA's row tiles are gate tiles paired with the up
+    // tiles pair_tiles further on, and y receives BF16(silu(gate) * up)
+    int pair_tiles;
+    uint32_t stg_off;  // staging of a chunk's sums for that epilogue
 };
 
 // Position in the slot ring (the ring depth is a runtime value: no divisions).
@@ -193,27 +198,29 @@ __device__ __forceinline__ int prep_class_shift(int P, int m) {
 // (value 4j + m of raw); 2-bit: the pairs k = 32t + 4j + 2P + {0,1} and
 // 32t + 16 + 4j + 2P + {0,1} (words 2j and 2j + 1 of raw); 5-trit: all 32
 // activations of thread t (value r of raw, both pairs).  xg is the group's
-// first activation (16-byte aligned).
+// first activation (16-byte aligned).  The loads go through L2 (not the
+// non-coherent path): in the chain kernel x may have been written by other
+// CTAs of the same launch.
 template <int FMT>
 __device__ __forceinline__ void load_task_x(const uint16_t* xg, int t, int P, uint32_t (&raw)[16]) {
     if (FMT == BQ_Q1G128) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
+            const uint2 v = __ldcg(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
             raw[2 * j] = v.x;
             raw[2 * j + 1] = v.y;
         }
     } else if (FMT == BQ_T2G128) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            raw[2 * j] = __ldg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 4 * j + 2 * P));
-            raw[2 * j + 1] = __ldg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 16 + 4 * j + 2 * P));
+            raw[2 * j] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 4 * j + 2 * P));
+            raw[2 * j + 1] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 16 + 4 * j + 2 * P));
         }
     } else {
         const uint32_t* src = reinterpret_cast<const uint32_t*>(xg + 30 * t);  // 60 t bytes: 4-byte aligned
 #pragma unroll
-        for (int i = 0; i < 15; ++i) raw[i] = __ldg(src + i);
-        raw[15] = __ldg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
+        for (int i = 0; i < 15; ++i) raw[i] = __ldcg(src + i);
+        raw[15] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
     }
 }
 
@@ -550,7 +557,17 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
         }
         bar_compute<NW>();  // red is reused by the next chunk
     }
-    if (active && gsub == 0 && (t & 1) == 0) {
+    if (active && gsub == 0 && (t & 1) == 0 && p.pair_tiles > 0) {
+        // SwiGLU step: the chunk's sums go to the staging area [tile][row][batch]
+        float* stg = reinterpret_cast<float*>(smem + p.stg_off);
+#pragma unroll
+        for (int tp = 0; tp < TPW; ++tp)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                    stg[((my_rt + NW * tp) * 16 + g + 8 * r) * 8 + nt * 2 + (t >> 1)] = yacc[tp][nt][r];
+    } else if (active && gsub == 0 && (t & 1) == 0) {
 #pragma unroll
         for (int tp = 0; tp < TPW; ++tp)
 #pragma unroll
@@ -576,6 +593,172 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
 struct Maps {
     CUtensorMap codes16, scales16, codes128, scales128;
 };
+
+// Row tile of W that tile i of a chunk of ct tiles starting at r holds: r + i,
+// or, for a SwiGLU step, gate tiles r .. r + ct/2 - 1 then the up tiles
+// pair_tiles further on.
+__device__ __forceinline__ int chunk_row_tile(const Params& p, int r, int ct, int i) {
+    if (p.pair_tiles == 0) return r + i;
+    const int c = ct >> 1;
+    return i < c ? r + i : p.pair_tiles + r + (i - c);
+}
+
+// The producer's copies of one (chunk, stage) into ring slot `slot`; lane 0
+// has posted the byte count on full[slot].  A full chunk is one 128-row box per
+// 128-byte column and 8 row tiles whose rows are contiguous; otherwise 16-row
+// boxes, one lane per row tile.
+template <int FMT>
+__device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, int slot,
+                                            int st, int r, int ct, int lane) {
+    constexpr int TCB = tile_code_bytes<FMT>();
+    constexpr int KB = Fmt<FMT>::kBoxes;
+    uint8_t* sb = smem + slot * p.slot_bytes;
+    const bool box128 = FMT == BQ_T5P8G128 ? (ct == kMaxChunkTiles && p.pair_tiles == 0)
+                                           : (ct >= kMaxChunkTiles && (p.pair_tiles == 0 || ct >= 2 * kMaxChunkTiles));
+    if (FMT == BQ_T5P8G128) {
+        if (box128) {
+            if (lane == 0) ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
+            if (lane == 1)
+                ptx::tma_load_2d(sb + p.scales_off, &tm.scales128, st * kGroupsPerStage, r * 16, &full[slot]);
+        } else if (lane < ct) {
+            const int rt = chunk_row_tile(p, r, ct, lane);
+            ptx::tma_load_2d(sb + lane * TCB, &tm.codes16, st * kT5RowBytes, rt * 16, &full[slot]);
+            ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16, st * kGroupsPerStage, rt * 16,
+                             &full[slot]);
+        }
+    } else if (box128) {
+        // 128-row boxes: one per 128-byte column (2-bit) and 8 row tiles
+        const int nbox = ct / kMaxChunkTiles;
+        if (lane < nbox * KB) {
+            const int h8 = lane / KB, b = lane - h8 * KB;
+            ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + h8 * kBoxColumnBytes, &tm.codes128,
+                             st * (KB * 128) + b * 128, chunk_row_tile(p, r, ct, 8 * h8) * 16, &full[slot]);
+        } else if (lane >= 16 && lane < 16 + nbox) {
+            const int h8 = lane - 16;
+            ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes, &tm.scales128,
+                             st * kGroupsPerStage, chunk_row_tile(p, r, ct, 8 * h8) * 16, &full[slot]);
+        }
+    } else if (lane < ct) {
+        const int rt = chunk_row_tile(p, r, ct, lane);
+#pragma unroll
+        for (int b = 0; b < KB; ++b)
+            ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + lane * 2048, &tm.codes16, st * (KB * 128) + b * 128,
+                             rt * 16, &full[slot]);
+        ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16, st * kGroupsPerStage, rt * 16,
+                         &full[slot]);
+    }
+}
+
+// Producer warp: streams the weights of row tiles [rt0, rt1) (pair tiles for
+// a SwiGLU step), chunk by chunk and stage by stage, through the ring.  rp and
+// it (copies issued) carry over from one call to the next.  False if a slot
+// wait timed out.
+template <int FMT>
+__device__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0,
+                        int rt1, Ring& rp, int& it, int lane) {
+    constexpr int TCB = tile_code_bytes<FMT>();
+    const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
+    for (int r = rt0; r < rt1;) {
+        const int c = chunk_tiles(rt1 - r, cap);
+        const int ct = p.pair_tiles > 0 ? 2 * c : c;
+        for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
+            const int slot = rp.slot;
+            int ok = 1;
+            if (lane == 0) {
+                if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+                    ok = 0;
+                } else {
+                    ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+            issue_stage<FMT>(tm, p, smem, full, slot, st, r, ct, lane);
+        }
+        r += c;
+    }
+    return true;
+}
+
+// Compute warps: x -> the resident activation operand (B fragments and table
+// of all of K).  Warp items (stage, batch row, half h of the stage's groups),
+// item i on warp i % NW; lane 8 gq + 2 t + P takes group 4 h + gq.  Rows go up
+// to the n-tiles' width (zero past the batch; one row at 16 lanes).
+template <int FMT, int NT, int LANES, int NW>
+__device__ void prep_x(const Params& p, uint8_t* smem, int warp, int lane) {
+    constexpr int kPrepBatch = 2;
+    uint8_t* xres = smem + p.x_off;
+    const int rows = LANES == 16 ? 1 : 2 * NT;
+    const int items = p.stages * rows * 2;
+    const int gq = lane >> 3, t = (lane >> 1) & 3, P = lane & 1;
+    for (int i0 = warp; i0 < items; i0 += NW * kPrepBatch) {
+        uint32_t raw[kPrepBatch][16];
+#pragma unroll
+        for (int j = 0; j < kPrepBatch; ++j) {
+            const int i = i0 + j * NW;
+            const int sr = i >> 1, G = 4 * (i & 1) + gq;
+            const int st = sr / rows, bb = sr - st * rows;
+            if (i < items && bb < p.batch) {
+                load_task_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, P, raw[j]);
+            } else {
+#pragma unroll
+                for (int w = 0; w < 16; ++w) raw[j][w] = 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kPrepBatch; ++j) {
+            const int i = i0 + j * NW;
+            if (i < items) {  // (warp-uniform)
+                const int sr = i >> 1, G = 4 * (i & 1) + gq;
+                const int st = sr / rows, bb = sr - st * rows;
+                prep_task<FMT, LANES>(xres + (size_t)(st * NT + (bb >> 1)) * x_nt_bytes(LANES), G, t, P, bb & 1,
+                                      raw[j]);
+            }
+        }
+    }
+}
+
+// Compute warps: every chunk of row tiles [rt0, rt1) (pair tiles for a SwiGLU
+// step, whose chunks hold c gate and c up tiles and end with the SwiGLU
+// epilogue).  False if a wait timed out.
+template <int FMT, int NT, int LANES, int NW>
+__device__ bool run_chunks(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0, int rt1,
+                           Ring& rp, int warp, int lane) {
+    const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
+    for (int r = rt0; r < rt1;) {
+        const int c = chunk_tiles(rt1 - r, cap);
+        const int ct = p.pair_tiles > 0 ? 2 * c : c;
+        bool ok;
+        if (mct<FMT, NT>() >= 16 && ct == 16)
+            ok = run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 8)
+            ok = run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 4)
+            ok = run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 2)
+            ok = run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
+        else
+            ok = run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+        if (!ok) return false;
+        if (p.pair_tiles > 0) {
+            // act = BF16(silu(gate) * up) of the chunk's c pair tiles
+            bar_compute<NW>();
+            const float* stg = reinterpret_cast<const float*>(smem + p.stg_off);
+            uint16_t* act = static_cast<uint16_t*>(p.y);
+            for (int i = threadIdx.x; i < c * 16 * p.batch; i += NW * 32) {
+                const int bb = i / (c * 16), rr = i - bb * (c * 16);
+                const int64_t row = (int64_t)r * 16 + rr;
+                if (row < p.n) {
+                    const float gv = stg[rr * 8 + bb], uv = stg[(c * 16 + rr) * 8 + bb];
+                    act[bb * p.n + row] = float_to_bf16_bits(gv / (1.0f + expf(-gv)) * uv);
+                }
+            }
+            bar_compute<NW>();  // the staging area is reused by the next chunk
+        }
+        r += c;
+    }
+    return true;
+}
 
 template <int FMT, int NT, int LANES, int NW>
 __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
@@ -612,65 +795,10 @@ __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
             ptx::prefetch_tensormap(&tm.codes128);
             ptx::prefetch_tensormap(&tm.scales128);
         }
-        constexpr int TCB = tile_code_bytes<FMT>();
-        constexpr int KB = Fmt<FMT>::kBoxes;
         int it = 0;
         Ring rp;
         rp.depth = p.slots;
-        bool alive = true;
-        for (int r = rt0; r < rt1 && alive;) {
-            const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
-            for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
-                const int slot = rp.slot;
-                int ok = 1;
-                if (lane == 0) {
-                    if (rp.round > 0 && !ptx::mbar_wait_bounded(&empty[slot], (rp.round - 1) & 1u, kWaitPolls)) {
-                        record_status(p.status, BQ_ERR_TIMEOUT);
-                        ok = 0;
-                    } else {
-                        ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
-                    }
-                }
-                if (!__shfl_sync(0xffffffffu, ok, 0)) {
-                    alive = false;
-                    break;
-                }
-                uint8_t* sb = smem + slot * p.slot_bytes;
-                if (FMT == BQ_T5P8G128) {
-                    if (ct == kMaxChunkTiles) {
-                        if (lane == 0) ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
-                        if (lane == 1)
-                            ptx::tma_load_2d(sb + p.scales_off, &tm.scales128, st * kGroupsPerStage, r * 16, &full[slot]);
-                    } else if (lane < ct) {
-                        ptx::tma_load_2d(sb + lane * TCB, &tm.codes16, st * kT5RowBytes, (r + lane) * 16, &full[slot]);
-                        ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16,
-                                         st * kGroupsPerStage, (r + lane) * 16, &full[slot]);
-                    }
-                } else if (ct >= kMaxChunkTiles) {
-                    // 128-row boxes: one per 128-byte column (2-bit) and 8 row tiles
-                    const int nbox = ct / kMaxChunkTiles;
-                    if (lane < nbox * KB) {
-                        const int h8 = lane / KB, b = lane - h8 * KB;
-                        ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + h8 * kBoxColumnBytes, &tm.codes128,
-                                         st * (KB * 128) + b * 128,
-                                         (r + 8 * h8) * 16, &full[slot]);
-                    } else if (lane >= 16 && lane < 16 + nbox) {
-                        const int h8 = lane - 16;
-                        ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes, &tm.scales128,
-                                         st * kGroupsPerStage, (r + 8 * h8) * 16, &full[slot]);
-                    }
-                } else if (lane < ct) {
-#pragma unroll
-                    for (int b = 0; b < KB; ++b)
-                        ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + lane * 2048, &tm.codes16,
-                                         st * (KB * 128) + b * 128,
-                                         (r + lane) * 16, &full[slot]);
-                    ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16, st * kGroupsPerStage,
-                                     (r + lane) * 16, &full[slot]);
-                }
-            }
-            r += ct;
-        }
+        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
         // every copy this CTA issued must land before it may exit
         if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
@@ -689,59 +817,158 @@ __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
         }
     }
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
-    {
-        // warp items (stage, batch row, half h of the stage's groups), item i
-        // on warp i % NW; lane 8 gq + 2 t + P takes group 4 h + gq.  Rows go up
-        // to the n-tiles' width (zero past the batch; one row at 16 lanes).
-        constexpr int kPrepBatch = 2;
-        uint8_t* xres = smem + p.x_off;
-        const int rows = LANES == 16 ? 1 : 2 * NT;
-        const int items = p.stages * rows * 2;
-        const int gq = lane >> 3, t = (lane >> 1) & 3, P = lane & 1;
-        for (int i0 = warp; i0 < items; i0 += NW * kPrepBatch) {
-            uint32_t raw[kPrepBatch][16];
-#pragma unroll
-            for (int j = 0; j < kPrepBatch; ++j) {
-                const int i = i0 + j * NW;
-                const int sr = i >> 1, G = 4 * (i & 1) + gq;
-                const int st = sr / rows, bb = sr - st * rows;
-                if (i < items && bb < p.batch) {
-                    load_task_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, P, raw[j]);
-                } else {
-#pragma unroll
-                    for (int w = 0; w < 16; ++w) raw[j][w] = 0u;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kPrepBatch; ++j) {
-                const int i = i0 + j * NW;
-                if (i < items) {  // (warp-uniform)
-                    const int sr = i >> 1, G = 4 * (i & 1) + gq;
-                    const int st = sr / rows, bb = sr - st * rows;
-                    prep_task<FMT, LANES>(xres + (size_t)(st * NT + (bb >> 1)) * x_nt_bytes(LANES), G, t, P, bb & 1,
-                                          raw[j]);
-                }
-            }
-        }
-    }
+    prep_x<FMT, NT, LANES, NW>(p, smem, warp, lane);
     bar_compute<NW>();
     Ring rp;
     rp.depth = p.slots;
-    for (int r = rt0; r < rt1;) {
-        const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
-        bool ok;
-        if (mct<FMT, NT>() >= 16 && ct == 16)
-            ok = run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
-        else if (ct == 8)
-            ok = run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
-        else if (ct == 4)
-            ok = run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
-        else if (ct == 2)
-            ok = run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
-        else
-            ok = run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+    run_chunks<FMT, NT, LANES, NW>(p, smem, full, empty, rt0, rt1, rp, warp, lane);
+}
+
+// ------------------------------------------------------------ chain kernel
+// A persistent grid (one CTA of 16 compute warps per SM) that runs a short
+// list of dependent products in order -- the projections of one decoder
+// layer ("1-bit Bonsai 8B" notes, Table 1: GQA attention projections and the
+// SwiGLU feed-forward).  The producer warp streams every step's weights back
+// to back through one ring, so the next product's weights arrive while the
+// current one computes; the compute warps finish step s, publish it with a
+// grid-wide barrier (a counter in global memory, bounded waits), and only then
+// read step s+1's activations, which may be step s's output.  A SwiGLU step
+// (W = [gate; up]) writes BF16(silu(gate) * up) instead of the raw products.
+constexpr int kMaxChainSteps = 8;
+constexpr int kChainStgBytes = 16 * 16 * 8 * 4;  // [16 tiles][16 rows][8 batch] floats
+
+struct ChainMaps {
+    Maps m[kMaxChainSteps];
+};
+struct ChainParams {
+    Params step[kMaxChainSteps];  // shared-memory layout fields are the same in every step
+    int nsteps;
+    unsigned int* bar;            // [0] barrier arrivals, [1] exits; zero on entry, left zero
+};
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* a) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+    return v;
+}
+
+// Compute warps of every CTA: publish this CTA's outputs of the current step
+// (arrive), or wait until every CTA has published (target arrivals).  Only
+// thread 0 touches the counter; the other threads wait at the compute-warp
+// barrier.  A wait that gives up records BQ_ERR_TIMEOUT; the return value is
+// the same in every compute thread.
+template <int NW>
+__device__ void grid_arrive(unsigned int* bar) {
+    bar_compute<NW>();  // every compute thread's stores of the step are done
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(&bar[0], 1u);
+    }
+}
+
+template <int NW>
+__device__ bool grid_wait(unsigned int* bar, unsigned int target, int* status, int* flag_smem) {
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        if (ld_acquire_gpu(&bar[0]) < target) {
+            const uint64_t t0 = ptx::globaltimer_ns();
+            for (uint32_t i = 1;; ++i) {
+                __nanosleep(64);
+                if (ld_acquire_gpu(&bar[0]) >= target) break;
+                if (i >= kWaitPolls || ((i & 255u) == 0 && ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs)) {
+                    record_status(status, BQ_ERR_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        *flag_smem = ok;
+    }
+    bar_compute<NW>();
+    return *flag_smem != 0;
+}
+
+template <int FMT, int NT, int LANES>
+__global__ void __launch_bounds__(threads_of<16>(), 1)
+    gemv_chain_kernel(const __grid_constant__ ChainMaps tm, const __grid_constant__ ChainParams cp) {
+    constexpr int NW = 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = ptx::align_smem<1024>(smem_raw);
+    const Params& p0 = cp.step[0];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p0.bar_off);
+    uint64_t* empty = full + kMaxSlots;
+    int* flag = reinterpret_cast<int*>(smem + p0.bar_off + 2 * kMaxSlots * 8);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = gridDim.x, c = blockIdx.x;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p0.slots; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], NW);
+        }
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    // (every CTA of this grid is resident once all of them have executed
+    // this, so a later kernel cannot take an SM one of them still needs)
+    ptx::pdl_launch_dependents();
+    const int nsteps = cp.nsteps;
+
+    if (warp == NW) {
+        // ------------------------------------------------ weight producer
+        if (lane < 4 * nsteps) {
+            const Maps& m = tm.m[lane >> 2];
+            const CUtensorMap* mp[4] = {&m.codes16, &m.scales16, &m.codes128, &m.scales128};
+            ptx::prefetch_tensormap(mp[lane & 3]);
+        }
+        int it = 0;
+        Ring rp;
+        rp.depth = p0.slots;
+        for (int s = 0; s < nsteps; ++s) {
+            const Params& p = cp.step[s];
+            const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
+            const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
+            if (!produce<FMT>(tm.m[s], p, smem, full, empty, rt0, rt1, rp, it, lane)) break;
+        }
+        if (lane == 0)
+            for (int j = (it > p0.slots ? it - p0.slots : 0); j < it; ++j)
+                if (!ptx::mbar_wait_bounded(&full[j % p0.slots], (uint32_t)((j / p0.slots) & 1), kWaitPolls))
+                    record_status(p0.status, BQ_ERR_TIMEOUT);
+        return;
+    }
+
+    // ---------------------------------------------------- compute warps
+    if (FMT == BQ_T5P8G128) {
+        uint32_t* lut = reinterpret_cast<uint32_t*>(smem + p0.lut_off);
+        for (int i = threadIdx.x; i < 256 * 32; i += NW * 32) {
+            const uint32_t v = (uint32_t)i >> 5;
+            lut[i] = (v % 3u) | ((v / 3u % 3u) << 8) | ((v / 9u % 3u) << 16) | ((v / 27u % 3u) << 24);
+        }
+    }
+    ptx::pdl_wait();  // the first step's x is produced, the outputs may still be read, by the previous kernel
+    Ring rp;
+    rp.depth = p0.slots;
+    bool ok = true;
+    for (int s = 0; s < nsteps && ok; ++s) {
+        const Params& p = cp.step[s];
+        if (s > 0) ok = grid_wait<NW>(cp.bar, (unsigned int)(s * C), p0.status, flag);
         if (!ok) break;
-        r += ct;
+        prep_x<FMT, NT, LANES, NW>(p, smem, warp, lane);
+        bar_compute<NW>();
+        const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
+        const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
+        ok = run_chunks<FMT, NT, LANES, NW>(p, smem, full, empty, rt0, rt1, rp, warp, lane);
+        if (s + 1 < nsteps) grid_arrive<NW>(cp.bar);
+    }
+    // The last CTA out leaves the counters zero for the next launch (every CTA
+    // has passed its last wait by then).
+    bar_compute<NW>();
+    if (threadIdx.x == 0 && ok) {
+        __threadfence();
+        if (atomicAdd(&cp.bar[1], 1u) == (unsigned int)C - 1) {
+            atomicExch(&cp.bar[0], 0u);
+            atomicExch(&cp.bar[1], 0u);
+        }
     }
 }
 
@@ -870,6 +1097,8 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
     prm.red_off = pl.red_off;
     prm.lut_off = pl.lut_off;
     prm.bar_off = pl.bar_off;
+    prm.pair_tiles = 0;
+    prm.stg_off = 0;
     prm.status = device_status_ptr();
     if (!prm.status) return cudaErrorUnknown;
     cudaLaunchAttribute attr;
@@ -903,6 +1132,158 @@ cudaError_t launch_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, 
 }  // namespace rows
 
 bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch) { return rows::make_plan(fmt, n, k, batch).ok; }
+
+namespace rows {
+
+// One shared-memory layout for every step: x area for the largest K, 16
+// compute warps, one CTA per SM, chunk bound and slot size as a single call
+// of the format and batch would use them at one CTA per SM.
+bool chain_plan(Plan& pl, int fmt, const bq_chain_step* steps, int nsteps, int batch) {
+    int64_t kmax = 0;
+    for (int i = 0; i < nsteps; ++i) kmax = steps[i].k > kmax ? steps[i].k : kmax;
+    pl.nt = batch <= 2 ? 1 : batch <= 4 ? 2 : 4;
+    pl.lanes = batch == 1 ? 16 : 32;
+    pl.stages = (int)(kmax / 1024);
+    pl.nw = 16;
+    const int sms = sm_count();
+    pl.grid = sms;
+    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + kTileScaleBytes;
+    pl.chunk_cap = kMaxChunkTiles;
+    const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+    pl.slot_bytes = (int)slot;
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
+    const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
+    const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
+    const int64_t red = (int64_t)16 * 32 * pl.nt * 2 * 4;
+    const int64_t fixed = 1024 + x_area + red + kChainStgBytes + lut + 2 * kMaxSlots * 8 + 16;
+    int64_t slots = (kSmemFull - fixed) / slot;
+    if (slots > kMaxSlots) slots = kMaxSlots;
+    if (slots < 2) return false;
+    pl.slots = (int)slots;
+    pl.x_off = (uint32_t)(slots * slot);
+    pl.red_off = (uint32_t)(pl.x_off + x_area);
+    pl.lut_off = (uint32_t)(pl.red_off + red + kChainStgBytes);  // staging after red
+    pl.bar_off = (uint32_t)(pl.lut_off + lut);
+    pl.smem = (uint32_t)(1024 + pl.bar_off + 2 * kMaxSlots * 8 + 16);
+    pl.ok = true;
+    return true;
+}
+
+cudaError_t encode_maps(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, Maps& tm) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const int64_t row_bytes = (fmt == BQ_Q1G128) ? k / 8 : (fmt == BQ_T2G128) ? k / 4 : (k / 128) * 26;
+    const int64_t G = k / 128;
+    for (int v = 0; v < 2; ++v) {
+        const cuuint32_t rows = v == 0 ? 16u : 128u;
+        cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)n};
+        cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+        cuuint32_t box[2] = {fmt == BQ_T5P8G128 ? (cuuint32_t)kT5RowBytes : 128u, rows};
+        cuuint32_t es[2] = {1, 1};
+        if (enc(v == 0 ? &tm.codes16 : &tm.codes128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+                strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                fmt == BQ_T5P8G128 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        cuuint64_t sdims[2] = {(cuuint64_t)G, (cuuint64_t)n};
+        cuuint64_t sstrides[1] = {(cuuint64_t)(G * 2)};
+        cuuint32_t sbox[2] = {(cuuint32_t)kGroupsPerStage, rows};
+        if (enc(v == 0 ? &tm.scales16 : &tm.scales128, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales),
+                sdims, sstrides, sbox, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
+template <int FMT, int NT, int LANES>
+cudaError_t launch_chain_typed(const bq_chain_step* steps, int nsteps, int batch, unsigned int* bar, const Plan& pl,
+                               cudaStream_t s) {
+    {
+        const cudaError_t e =
+            ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_chain_kernel<FMT, NT, LANES>), kSmemFull);
+        if (e != cudaSuccess) return e;
+    }
+    ChainMaps tm;
+    ChainParams cp;
+    cp.nsteps = nsteps;
+    cp.bar = bar;
+    int* status = device_status_ptr();
+    if (!status) return cudaErrorUnknown;
+    for (int i = 0; i < nsteps; ++i) {
+        const bq_chain_step& st = steps[i];
+        const cudaError_t e = encode_maps(FMT, st.codes, st.scales, st.n, st.k, tm.m[i]);
+        if (e != cudaSuccess) return e;
+        Params& p = cp.step[i];
+        p.x = st.x;
+        p.y = st.y;
+        p.k = st.k;
+        p.batch = batch;
+        p.y_dtype = st.swiglu ? BQ_BF16 : st.y_dtype;
+        p.stages = (int)(st.k / 1024);
+        p.pair_tiles = st.swiglu ? (int)(st.n / 2 / 16) : 0;
+        p.n = st.swiglu ? st.n / 2 : st.n;  // outputs per batch row
+        p.row_tiles = st.swiglu ? p.pair_tiles : (int)((st.n + 15) / 16);
+        p.slots = pl.slots;
+        p.slot_bytes = pl.slot_bytes;
+        p.scales_off = pl.scales_off;
+        p.chunk_cap = pl.chunk_cap;
+        p.x_off = pl.x_off;
+        p.red_off = pl.red_off;
+        p.stg_off = pl.red_off + (uint32_t)(16 * 32 * pl.nt * 2 * 4);
+        p.lut_off = pl.lut_off;
+        p.bar_off = pl.bar_off;
+        p.status = status;
+    }
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(threads_of<16>());
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_chain_kernel<FMT, NT, LANES>, tm, cp);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <int FMT>
+cudaError_t launch_chain_fmt(const bq_chain_step* steps, int nsteps, int batch, unsigned int* bar, const Plan& pl,
+                             cudaStream_t s) {
+    if (batch == 1) return launch_chain_typed<FMT, 1, 16>(steps, nsteps, batch, bar, pl, s);
+    if (pl.nt == 1) return launch_chain_typed<FMT, 1, 32>(steps, nsteps, batch, bar, pl, s);
+    if (pl.nt == 2) return launch_chain_typed<FMT, 2, 32>(steps, nsteps, batch, bar, pl, s);
+    return launch_chain_typed<FMT, 4, 32>(steps, nsteps, batch, bar, pl, s);
+}
+
+}  // namespace rows
+
+bool gemv_chain_eligible(int fmt, const bq_chain_step* steps, int nsteps, int batch) {
+    if (nsteps < 1 || nsteps > rows::kMaxChainSteps || batch < 1 || batch > 8) return false;
+    for (int i = 0; i < nsteps; ++i) {
+        const bq_chain_step& st = steps[i];
+        if (st.k <= 0 || st.k % 1024 != 0 || st.k > ((int64_t)1 << 20) || st.n <= 0 || st.n > (int64_t)INT32_MAX - 16)
+            return false;
+        if (st.swiglu && (st.n % 32 != 0)) return false;  // whole gate and up row tiles
+    }
+    rows::Plan pl;
+    return rows::chain_plan(pl, fmt, steps, nsteps, batch);
+}
+
+cudaError_t launch_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch, unsigned int* bar,
+                              cudaStream_t s) {
+    rows::Plan pl;
+    if (!rows::chain_plan(pl, fmt, steps, nsteps, batch)) return cudaErrorInvalidValue;
+    if (fmt == BQ_Q1G128) return rows::launch_chain_fmt<BQ_Q1G128>(steps, nsteps, batch, bar, pl, s);
+    if (fmt == BQ_T2G128) return rows::launch_chain_fmt<BQ_T2G128>(steps, nsteps, batch, bar, pl, s);
+    return rows::launch_chain_fmt<BQ_T5P8G128>(steps, nsteps, batch, bar, pl, s);
+}
+
 
 cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s) {

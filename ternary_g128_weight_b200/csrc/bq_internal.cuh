@@ -76,6 +76,12 @@ bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
 
+// Persistent layer chain (bq_gemv_chain): eligibility of the step list and
+// its launch; bar = the two zeroed barrier counters.
+bool gemv_chain_eligible(int fmt, const bq_chain_step* steps, int nsteps, int batch);
+cudaError_t launch_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch, unsigned int* bar,
+                              cudaStream_t s);
+
 // GEMV path choice shared by bq_gemv, bq_gemm (T <= 4) and bq_gemv_noalloc:
 // the row-owning kernel where eligible, else the split-K tensor-core kernel,
 // else the tcgen05 GEMM with T = batch; None when no kernel takes the shape

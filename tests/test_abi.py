@@ -145,3 +145,33 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         mod._lib = saved
+
+
+def test_chain_argument_errors_without_device(lib):
+    """bq_gemv_chain rejects bad arguments before touching a device (fake,
+    aligned device addresses are never dereferenced on these paths)."""
+    S = bq.ChainStep
+    A = 0x100000
+
+    def call(steps, nsteps=None, batch=1, ws=A, wsb=256, fmt=bq.BQ_Q1G128):
+        arr = (S * max(1, len(steps)))(*steps)
+        return lib.bq_gemv_chain(fmt, arr, len(steps) if nsteps is None else nsteps, batch,
+                                 ctypes.c_void_p(ws) if ws else None, wsb, None)
+
+    ok = S(A, A, 64, 1024, A, A, bq.BQ_BF16, 0)
+    assert call([ok], nsteps=0) == bq.BQ_ERR_SHAPE
+    assert call([ok] * 9) == bq.BQ_ERR_SHAPE
+    assert call([ok], fmt=9) == bq.BQ_ERR_FORMAT
+    assert call([ok], batch=0) == bq.BQ_ERR_SHAPE
+    assert call([ok], batch=17) == bq.BQ_ERR_SHAPE
+    assert call([S(A, A, 64, 1152, A, A, bq.BQ_BF16, 0)]) == bq.BQ_ERR_SHAPE      # K % 1024 != 0
+    assert call([S(A, A, 64, 1000, A, A, bq.BQ_BF16, 0)]) == bq.BQ_ERR_SHAPE      # K % 128 != 0
+    assert call([S(A, A, 48, 1024, A, A, bq.BQ_BF16, 1)]) == bq.BQ_ERR_SHAPE      # gate|up not in whole tiles
+    assert call([S(A, A, 64, 1024, A, A, 7, 0)]) == bq.BQ_ERR_FORMAT              # output dtype
+    assert call([S(A, A, 64, 1024, A, A, bq.BQ_BF16, 2)]) == bq.BQ_ERR_FORMAT     # swiglu flag
+    assert call([S(A, A, 64, 1024, 0, A, bq.BQ_BF16, 0)]) == bq.BQ_ERR_NULL       # x
+    assert call([S(A, A, 64, 1024, A, A + 2, bq.BQ_BF16, 0)]) == bq.BQ_ERR_ALIGN  # y
+    assert call([S(A + 8, A, 64, 1024, A, A, bq.BQ_BF16, 0)]) == bq.BQ_ERR_ALIGN  # codes
+    assert call([ok], ws=0) == bq.BQ_ERR_WORKSPACE
+    assert call([ok], wsb=16) == bq.BQ_ERR_WORKSPACE
+    assert lib.bq_gemv_chain(bq.BQ_Q1G128, None, 1, 1, ctypes.c_void_p(A), 256, None) == bq.BQ_ERR_NULL
