@@ -861,8 +861,9 @@ template <int NW>
 __device__ void grid_arrive(unsigned int* bar) {
     bar_compute<NW>();  // every compute thread's stores of the step are done
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(&bar[0], 1u);
+        // release: the CTA's stores (ordered before this thread by the barrier)
+        // become visible no later than the arrival
+        asm volatile("fence.acq_rel.gpu;\n\tred.relaxed.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
     }
 }
 
@@ -873,7 +874,7 @@ __device__ bool grid_wait(unsigned int* bar, unsigned int target, int* status, i
         if (ld_acquire_gpu(&bar[0]) < target) {
             const uint64_t t0 = ptx::globaltimer_ns();
             for (uint32_t i = 1;; ++i) {
-                __nanosleep(64);
+                if (i > 64) __nanosleep(32);  // poll tightly first: the release is usually close
                 if (ld_acquire_gpu(&bar[0]) >= target) break;
                 if (i >= kWaitPolls || ((i & 255u) == 0 && ptx::globaltimer_ns() - t0 > ptx::kWaitLimitNs)) {
                     record_status(status, BQ_ERR_TIMEOUT);
@@ -882,7 +883,6 @@ __device__ bool grid_wait(unsigned int* bar, unsigned int target, int* status, i
                 }
             }
         }
-        __threadfence();
         *flag_smem = ok;
     }
     bar_compute<NW>();
