@@ -48,7 +48,12 @@ def parse():
     p.add_argument("--layers", type=int, default=None, help="blocks per pass (default: the model's)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM leg")
+    p.add_argument("--no-gemm", action="store_true", help="skip the prefill GEMM legs")
+    p.add_argument("--no-legs", action="store_true", help="skip the secondary configurations (the other formats, "
+                   "batches and the 27B class)")
+    p.add_argument("--leg-steps", type=int, default=10, help="timed steps of each secondary configuration")
+    p.add_argument("--mode", choices=["calls", "chain"], default="calls",
+                   help="one bq_gemv per product (calls) or one bq_gemv_chain per layer (chain)")
     p.add_argument("--gemm-only", action="store_true",
                    help="run only the prefill GEMM leg (a diagnostic line, e.g. for a profiler)")
     return p.parse_args()
@@ -192,54 +197,54 @@ def measured_tensor_peak():
 
 # ---------------------------------------------------------------- prefill GEMM
 GEMM_SHAPES = [(17408, 5120), (5120, 17408)]
-GEMM_TOKENS = 4096
 
 
 def gemm_leg(fmt, dev, reps):
-    """Prefill GEMM Y = X W^T at T = 4096 on the pages' two prefill shapes
-    (tensor-bound); each launch timed alone with CUDA events, L2 flushed by a
-    256 MB write before every timed launch."""
+    """Prefill GEMM Y = X W^T on the pages' two prefill shapes at T = 1, 8, 64,
+    512 and 4096 tokens; each launch timed alone with CUDA events, L2 flushed by
+    a 256 MB write before every timed launch.  Reported as TFLOP/s against the
+    dense 16-bit tensor peak and, for the weight-bound small T, as weight GB/s
+    against HBM."""
     import torch
     import synth
     import ternary_g128_weight_b200 as bq
     peak, src = measured_tensor_peak()
+    hbm, _ = measured_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     out = []
     for (n, k) in GEMM_SHAPES:
         gen = synth.device_generator(synth.SEED_BASE + 4, device=dev)
-        if fmt == "q1g128":
-            codes, scales = bq.bq_pack(fmt, synth.device_weights_normal(gen, n, k, device=dev))
-        else:
-            t = synth.device_trits(gen, n, k, device=dev)
-            s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
-            w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
-            codes, scales = bq.bq_pack(fmt, w, scales_in=s)
-            del w
-        x = synth.device_x_bf16(gen, GEMM_TOKENS, k, device=dev)
-        y = torch.empty((GEMM_TOKENS, n), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(bq.bq_gemm_workspace_bytes(fmt, n, k, GEMM_TOKENS), 256), dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
-        torch.cuda.synchronize()
-        times = []
-        for _ in range(reps):
-            flush.fill_(1)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
-            e1.record()
+        codes, scales = make_weights(fmt, n, k, gen, dev, False)
+        wbytes = codes.numel() + 2 * scales.numel()
+        for T in synth.PREFILL_TOKENS:
+            x = synth.device_x_bf16(gen, T, k, device=dev)
+            y = torch.empty((T, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(bq.bq_gemm_workspace_bytes(fmt, n, k, T), 256), dtype=torch.uint8, device=dev)
+            for _ in range(3):
+                bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
             torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1))
-        assert bq.bq_check() == bq.BQ_OK
-        ms = statistics.median(times)
-        tf = 2.0 * GEMM_TOKENS * n * k / (ms / 1000.0) / 1e12
-        out.append({"shape": f"{n}x{k}", "tokens": GEMM_TOKENS, "us": round(ms * 1000, 1),
-                    "tflops": round(tf, 1), "frac": round(tf / peak, 4),
-                    "launches": bq.bq_gemm_launches(fmt, n, k, GEMM_TOKENS)})
-        del codes, scales, x, y, ws
-    return {"bound": "tensor", "peak": peak, "unit": "TFLOP/s",
+            times = []
+            for _ in range(reps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                bq.bq_gemm(fmt, codes, scales, n, k, x, y=y, workspace=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1))
+            assert bq.bq_check() == bq.BQ_OK
+            ms = statistics.median(times)
+            tf = 2.0 * T * n * k / (ms / 1000.0) / 1e12
+            gbs = wbytes / (ms / 1000.0) / 1e9
+            out.append({"shape": f"{n}x{k}", "tokens": T, "us": round(ms * 1000, 1),
+                        "tflops": round(tf, 2), "frac": round(tf / peak, 4),
+                        "weight_GB_s": round(gbs, 1), "hbm_frac": round(gbs / hbm, 4),
+                        "launches": bq.bq_gemm_launches(fmt, n, k, T)})
+            del x, y, ws
+        del codes, scales
+    return {"bound": "tensor (T >= 64), hbm (T <= 8)", "peak": peak, "unit": "TFLOP/s",
             "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst; FP16 operands at the same rate)",
-            "kernel": "xprep_f16_kernel + gemm_tc_kernel (tcgen05 kind::f16, TMEM accumulators)",
+            "kernel": "xprep_f16_kernel + gemm_tc_kernel (tcgen05 kind::f16, TMEM accumulators); T <= 4: the GEMV",
             "dtype": "f16 operands (exact s*q and pre-scaled x), f32 accumulate", "cases": out}
 
 
@@ -338,6 +343,200 @@ def job_value(bytes_per_rank_step, world, ms_per_step):
     return bytes_per_rank_step * world / (ms_per_step / 1000.0) / 1e9
 
 
+# --------------------------------------------------------------- the passes
+def make_weights(fmt, n, k, gen, dev, direct_codes):
+    """Weights of one matrix: binary by packing N(0, 0.02) floats (or, for the
+    27B class, uniform code bytes with uniform FP16 scales, no float pass);
+    ternary by packing trits (P(-1) = P(+1) = 0.35) times uniform FP16 scales
+    with the scales given."""
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+    if fmt == "q1g128":
+        if direct_codes:
+            return (synth.device_code_bytes(gen, bq.bq_codes_bytes(fmt, n, k), device=dev),
+                    synth.device_scales_uniform(gen, n, k // 128, device=dev).view(-1))
+        return bq.bq_pack(fmt, synth.device_weights_normal(gen, n, k, device=dev))
+    t = synth.device_trits(gen, n, k, device=dev)
+    s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
+    w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
+    del t
+    return bq.bq_pack(fmt, w, scales_in=s)
+
+
+class Pass:
+    """One decode weight pass on the device: per layer q|k|v, o, gate|up, down,
+    then the LM head, each with its own weights; every activation and output
+    in one contiguous buffer (one copy per step for the end-to-end timing).
+    mode "calls": one bq_gemv per product, each a programmatic dependent of the
+    previous one; mode "chain": one bq_gemv_chain per layer (q|k|v, o,
+    gate|up with the SwiGLU epilogue, down on that output), then the head."""
+
+    def __init__(self, model, fmt, batch, layers, seed, dev, mode="calls"):
+        import torch
+        import synth
+        import ternary_g128_weight_b200 as bq
+        self.model, self.fmt, self.batch, self.layers, self.mode = model, fmt, batch, layers, mode
+        self.f = FMT_NAMES[fmt]
+        gen = synth.device_generator(seed, device=dev)
+        shapes = step_shapes(model, layers)
+        direct = model == "27b"
+
+        def offsets(sizes):
+            offs, tot = [], 0
+            for sz in sizes:
+                offs.append(tot)
+                tot += (sz + 127) // 128 * 128
+            return offs, tot
+        L = model_shapes(model)[0]
+        inter = L["gate"][0]
+        x_sizes, y_sizes = [], []
+        for name, n, k in shapes:
+            x_sizes.append(batch * k)
+            y_sizes.append(batch * (inter if (mode == "chain" and name.endswith("gate_up")) else n))
+        x_offs, x_tot = offsets(x_sizes)
+        y_offs, y_tot = offsets(y_sizes)
+        self.X = synth.device_x_bf16(gen, 1, x_tot, device=dev).view(-1)
+        self.Y = torch.zeros(y_tot, dtype=torch.bfloat16, device=dev)
+        self.mats = []
+        for i, (name, n, k) in enumerate(shapes):
+            codes, scales = make_weights(fmt, n, k, gen, dev, direct)
+            yn = y_sizes[i] // batch
+            self.mats.append({"name": name, "n": n, "k": k, "codes": codes, "scales": scales,
+                              "x": self.X[x_offs[i]:x_offs[i] + batch * k].view(batch, k),
+                              "y": self.Y[y_offs[i]:y_offs[i] + batch * yn].view(batch, yn)})
+        torch.cuda.synchronize()
+        self.weight_bytes = sum(m["codes"].numel() + 2 * m["scales"].numel() for m in self.mats)
+        self.algo_bytes = self.weight_bytes + sum(2 * m["k"] * batch + 2 * m["y"].shape[1] * batch
+                                                  for m in self.mats)
+        ws_need = max(bq.bq_gemv_workspace_bytes(self.f, m["n"], m["k"], batch) for m in self.mats)
+        self.workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
+        self.chains = []
+        if mode == "chain":
+            for l in range(layers):
+                q, o, gu, dn = self.mats[4 * l:4 * l + 4]
+                steps = [dict(codes=q["codes"], scales=q["scales"], n=q["n"], k=q["k"], x=q["x"], y=q["y"]),
+                         dict(codes=o["codes"], scales=o["scales"], n=o["n"], k=o["k"], x=o["x"], y=o["y"]),
+                         dict(codes=gu["codes"], scales=gu["scales"], n=gu["n"], k=gu["k"], x=gu["x"], y=gu["y"],
+                              swiglu=True),
+                         dict(codes=dn["codes"], scales=dn["scales"], n=dn["n"], k=dn["k"], x=gu["y"], y=dn["y"])]
+                self.chains.append((steps, torch.zeros(bq.bq_gemv_chain_workspace_bytes(), dtype=torch.uint8,
+                                                       device=dev)))
+        self.launches = (sum(bq.bq_gemv_launches(self.f, m["n"], m["k"], batch) for m in self.mats)
+                         if mode == "calls" else layers + bq.bq_gemv_launches(self.f, *shapes[-1][1:], batch))
+        self.graph = None
+
+    def step(self):
+        import ternary_g128_weight_b200 as bq
+        if self.mode == "chain":
+            for steps, ws in self.chains:
+                bq.bq_gemv_chain(self.f, steps, workspace=ws)
+            m = self.mats[-1]
+            bq.bq_gemv(self.f, m["codes"], m["scales"], m["n"], m["k"], m["x"], y=m["y"], workspace=self.workspace)
+            return
+        for m in self.mats:
+            bq.bq_gemv(self.f, m["codes"], m["scales"], m["n"], m["k"], m["x"], y=m["y"], workspace=self.workspace)
+
+    def capture(self):
+        """Warm up eagerly (lazy initialisation), then capture one step in a CUDA graph."""
+        import torch
+        import ternary_g128_weight_b200 as bq
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.step()
+            self.step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        assert bq.bq_check() == bq.BQ_OK
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+
+    def time_steps(self, steps, warmup, barrier):
+        """Device time of `steps` graph replays (ms per step), CUDA events on the
+        replaying stream, barrier + synchronize on both sides."""
+        import torch
+        import ternary_g128_weight_b200 as bq
+        for _ in range(warmup):
+            self.graph.replay()
+        barrier()
+        stream = torch.cuda.current_stream()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            self.graph.replay()
+        t1.record(stream)
+        barrier()
+        assert bq.bq_check() == bq.BQ_OK
+        return t0.elapsed_time(t1) / steps
+
+    def time_e2e(self, steps, barrier):
+        """The same step through the public API with the step's activations
+        copied from pinned host memory and every output copied back, inside the
+        timed region."""
+        import torch
+        x_host = torch.empty_like(self.X, device="cpu").pin_memory()
+        x_host.copy_(self.X)
+        y_host = torch.empty_like(self.Y, device="cpu").pin_memory()
+        stream = torch.cuda.current_stream()
+
+        def e2e_step():
+            self.X.copy_(x_host, non_blocking=True)
+            self.graph.replay()
+            y_host.copy_(self.Y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        return {"ms_per_step": e0.elapsed_time(e1) / steps, "h2d": self.X.numel() * 2, "d2h": self.Y.numel() * 2}
+
+    def free(self):
+        import torch
+        self.graph = None
+        self.mats.clear()
+        self.chains.clear()
+        self.X = self.Y = self.workspace = None
+        torch.cuda.empty_cache()
+
+
+def leg(model, fmt, batch, mode, dev, steps, warmup, peak, seed):
+    """One secondary configuration: a whole pass, its GB/s, roofline fraction,
+    tokens/s-equivalent and end-to-end figure."""
+    layers = model_shapes(model)[2]
+    ps = Pass(model, fmt, batch, layers, seed, dev, mode)
+    ps.capture()
+    import torch
+    ms = ps.time_steps(steps, warmup, torch.cuda.synchronize)
+    e2e = ps.time_e2e(max(2, steps // 2), torch.cuda.synchronize)
+    out = {"workload": workload_name(model, fmt, batch, layers) + ("" if mode == "calls" else ", one chain per layer"),
+           "model": model, "fmt": fmt, "batch": batch, "mode": mode, "steps": steps,
+           "ms_per_step": round(ms, 4), "value": round(ps.weight_bytes / (ms / 1000.0) / 1e9, 2), "unit": "GB/s",
+           "roofline_frac": round(ps.algo_bytes / (ms / 1000.0) / 1e9 / peak, 4),
+           "tokens_per_s_equiv": round(1000.0 / ms, 2),
+           "e2e": {"value": round(ps.weight_bytes / (e2e["ms_per_step"] / 1000.0) / 1e9, 2), "unit": "GB/s",
+                   "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+           "launches_per_step": ps.launches}
+    ps.free()
+    return out
+
+
+# The secondary configurations: the Qwen3-8B shapes in both ternary formats
+# at batch 1 and 16 and in binary at batch 8, the 27B class in all three
+# formats at batch 1 and 16, and the binary Qwen3-8B pass as per-layer chains.
+LEGS = [("qwen3-8b", "t2g128", 1, "calls"), ("qwen3-8b", "t5p8", 1, "calls"), ("qwen3-8b", "q1g128", 8, "calls"),
+        ("qwen3-8b", "t2g128", 16, "calls"), ("qwen3-8b", "t5p8", 16, "calls"),
+        ("27b", "q1g128", 1, "calls"), ("27b", "t2g128", 1, "calls"), ("27b", "t5p8", 1, "calls"),
+        ("27b", "q1g128", 16, "calls"), ("27b", "t2g128", 16, "calls"), ("27b", "t5p8", 16, "calls"),
+        ("qwen3-8b", "q1g128", 1, "chain")]
+
+
 # ----------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -347,7 +546,6 @@ def main():
         return run_reference(args)
 
     import torch
-    import synth
     import ternary_g128_weight_b200 as bq
 
     world, rank, local = world_info()
@@ -371,66 +569,16 @@ def main():
             dist.barrier()
             dist.destroy_process_group()
         return 0
-    gen = synth.device_generator(synth.SEED_BASE + 1 + 1000 * rank, device=dev)
-    shapes = step_shapes(args.model, args.layers)
-
-    # ---- activations and outputs: one contiguous buffer each (one copy per step for e2e)
-    def offsets(sizes):
-        offs, tot = [], 0
-        for sz in sizes:
-            offs.append(tot)
-            tot += (sz + 127) // 128 * 128
-        return offs, tot
-    x_offs, x_tot = offsets([batch * k for _, _, k in shapes])
-    y_offs, y_tot = offsets([batch * n for _, n, _ in shapes])
-    X_all = synth.device_x_bf16(gen, 1, x_tot, device=dev).view(-1)
-    Y_all = torch.zeros(y_tot, dtype=torch.bfloat16, device=dev)
-
-    # ---- weights: distinct per launch, packed on the GPU
-    mats = []
-    for i, (name, n, k) in enumerate(shapes):
-        if fmt == "q1g128":
-            w = synth.device_weights_normal(gen, n, k, device=dev)
-            codes, scales = bq.bq_pack(fmt, w)
-        else:
-            t = synth.device_trits(gen, n, k, device=dev)
-            s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
-            w = t.to(torch.float32) * s.view(torch.float16).to(torch.float32).repeat_interleave(128, dim=1)
-            codes, scales = bq.bq_pack(fmt, w, scales_in=s)
-        del w
-        mats.append({"name": name, "n": n, "k": k, "codes": codes, "scales": scales,
-                     "x": X_all[x_offs[i]:x_offs[i] + batch * k].view(batch, k),
-                     "y": Y_all[y_offs[i]:y_offs[i] + batch * n].view(batch, n)})
-    torch.cuda.synchronize()
-    ws_need = max(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) for m in mats)
-    workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=dev)
-    weight_bytes = sum(m["codes"].numel() + 2 * m["scales"].numel() for m in mats)
-    algo_bytes = weight_bytes + sum(2 * m["k"] * batch + 2 * m["n"] * batch for m in mats)
-    launches_per_step = sum(bq.bq_gemv_launches(f, m["n"], m["k"], batch) for m in mats)
+    ps = Pass(args.model, fmt, batch, args.layers, synth_seed(rank), dev, args.mode)
+    mats = ps.mats
+    ps.capture()
     calls_per_step = len(mats)
     # the arithmetic of the path bq_gemv takes for this format and batch
-    int8_path = batch <= 4 and all(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) == 0 for m in mats)
+    int8_path = batch <= 8 and all(bq.bq_gemv_workspace_bytes(f, m["n"], m["k"], batch) == 0 for m in mats)
     path_dtype = "s8xu8->s32 (warp MMA), f32 recombine" if int8_path else "f16 (tcgen05) -> f32"
-    path_kernel = ("gemv_rows_kernel (row-owning tensor-core GEMV)" if int8_path
+    path_kernel = (("gemv_rows_kernel (row-owning tensor-core GEMV)" if args.mode == "calls" else
+                    "gemv_chain_kernel (persistent layer chain) + gemv_rows_kernel (head)") if int8_path
                    else "xprep_f16_kernel + gemm_tc_kernel (tcgen05 GEMM with T = batch)")
-
-    def step():
-        for m in mats:
-            bq.bq_gemv(f, m["codes"], m["scales"], m["n"], m["k"], m["x"], y=m["y"], workspace=workspace)
-
-    # warm up eagerly (lazy initialisation), then capture one step in a CUDA graph
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        step()
-        step()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    assert bq.bq_check() == bq.BQ_OK
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    stream = torch.cuda.current_stream()
 
     def barrier():
         if dist is not None:
@@ -438,7 +586,7 @@ def main():
         torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
-        graph.replay()
+        ps.graph.replay()
     barrier()
     assert bq.bq_check() == bq.BQ_OK
 
@@ -446,29 +594,22 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    barrier()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for _ in range(args.steps):
-        graph.replay()
-    t_end.record(stream)
-    barrier()
+    elapsed_ms = ps.time_steps(args.steps, 0, barrier) * args.steps
     clocks = sampler.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    assert bq.bq_check() == bq.BQ_OK
 
     # ---- LM head alone (largest launch): per-launch time with events around it
     head = mats[-1]
+    stream = torch.cuda.current_stream()
     hg = torch.cuda.CUDAGraph()
     with torch.cuda.graph(hg):
         bq.bq_gemv(f, head["codes"], head["scales"], head["n"], head["k"], head["x"], y=head["y"],
-                   workspace=workspace)
+                   workspace=ps.workspace)
     hg.replay()
     torch.cuda.synchronize()
     h_times = []
     for _ in range(max(3, args.steps)):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        graph.replay()  # evicts the head's weights from L2 (1 GB streamed)
+        ps.graph.replay()  # evicts the head's weights from L2 (1 GB streamed)
         e0.record(stream)
         hg.replay()
         e1.record(stream)
@@ -478,28 +619,7 @@ def main():
     head_ms = statistics.median(h_times)
 
     # ---- end-to-end through the public API: pinned host inputs in, outputs out
-    e2e = None
-    if not args.no_e2e:
-        x_host = torch.empty_like(X_all, device="cpu").pin_memory()
-        x_host.copy_(X_all)
-        y_host = torch.empty_like(Y_all, device="cpu").pin_memory()
-
-        def e2e_step():
-            X_all.copy_(x_host, non_blocking=True)
-            graph.replay()
-            y_host.copy_(Y_all, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        barrier()
-        e2e = {"ms_per_step": e0.elapsed_time(e1) / args.steps,
-               "h2d": sum(2 * batch * m["k"] for m in mats), "d2h": sum(2 * batch * m["n"] for m in mats)}
+    e2e = None if args.no_e2e else ps.time_e2e(args.steps, barrier)
 
     # ---- max over ranks
     ms_per_step, e2e_ms = max_over_ranks([elapsed_ms / args.steps, e2e["ms_per_step"] if e2e else 0.0], dist, dev)
@@ -507,20 +627,23 @@ def main():
         e2e["ms_per_step"] = e2e_ms
 
     peak, peak_src = measured_peaks()
+    weight_bytes, algo_bytes = ps.weight_bytes, ps.algo_bytes
     value = job_value(weight_bytes, world, ms_per_step)
     achieved = algo_bytes / (ms_per_step / 1000.0) / 1e9
     traffic = recorded_traffic(args.model, fmt, batch, args.layers)
+    launches_per_step = ps.launches
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(fmt, mats, batch)
-    prefill = None
+    del hg
+    ps.free()
+    legs, prefill = [], None
+    if rank == 0 and not args.no_legs:
+        for i, (model, lf, lb, mode) in enumerate(LEGS):
+            legs.append(leg(model, lf, lb, mode, dev, args.leg_steps, 3, peak, synth_seed(rank) + 100 + i))
     if rank == 0 and not args.no_gemm:
-        del graph, hg
-        graph = hg = None
-        mats.clear()
-        torch.cuda.empty_cache()
-        prefill = gemm_leg(fmt, dev, 5)
+        prefill = {lf: gemm_leg(lf, dev, 5) for lf in (["q1g128", "t2g128", "t5p8"] if not args.no_legs else [fmt])}
 
     if rank == 0:
         line = {
@@ -529,7 +652,9 @@ def main():
             "warmup": max(args.warmup, 3), "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": path_dtype, "data": "synthetic",
-            "config": {"workload": workload_name(args.model, fmt, batch, args.layers), "fmt": fmt, "batch": batch,
+            "config": {"workload": workload_name(args.model, fmt, batch, args.layers)
+                       + ("" if args.mode == "calls" else ", one chain per layer"),
+                       "fmt": fmt, "batch": batch, "mode": args.mode,
                        "weight_bytes_per_step": weight_bytes, "gemv_calls_per_step": calls_per_step,
                        "l2": f"inputs larger than L2 ({weight_bytes / 1e9:.2f} GB of weights per step, L2 126 MB), no flush",
                        "parallelism": f"replicas x{world}"},
@@ -552,15 +677,21 @@ def main():
                            "d2h_bytes_per_step": e2e["d2h"]}
         if cpu:
             line["cpu_baseline"] = cpu
+        if legs:
+            line["configs"] = legs
         if prefill:
             line["prefill_gemm"] = prefill
         print(json.dumps(line), flush=True)
 
-    del graph, hg
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def synth_seed(rank):
+    import synth
+    return synth.SEED_BASE + 1 + 1000 * rank
 
 
 if __name__ == "__main__":

@@ -175,6 +175,19 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
 bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                           const uint16_t* x, int batch, void* y, int y_dtype, void* stream);
 
+/* -------------------------------------------------------------- embedding */
+/* Embedding lookup on a low-bit table ("1-bit Bonsai 8B" notes, section 3 and
+ * Table 1: the embedding layer is low-bit too):
+ *   out[i][k] = BF16_RNE(s[ids[i]][k/128] * q[ids[i]][k]),   i < count,
+ * exact up to the one rounding of the FP16 scale to BF16.  codes/scales: the
+ * N x K table as above (16-byte aligned); ids: device int32 [count] (4-byte
+ * aligned); out: device BF16 [count][K] (16-byte aligned).  An id outside
+ * [0, N) gives a zero row and makes bq_check() report BQ_ERR_SHAPE (the ids
+ * live on the device, so the host cannot check them).  Asynchronous on
+ * `stream`. */
+bq_status bq_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                        const int32_t* ids, int64_t count, uint16_t* out, void* stream);
+
 /* --------------------------------------------------------- layer chains */
 /* One product of a chain (see bq_gemv_chain).  All pointers are device
  * pointers; codes/scales/x 16-byte aligned as for bq_gemv. */

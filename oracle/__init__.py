@@ -79,6 +79,9 @@ def lib():
         L.bqo_matmul_rows.restype = ctypes.c_int
         L.bqo_swiglu.argtypes = [f64p, ctypes.c_int64, ctypes.c_int64, u16p, f64p]
         L.bqo_swiglu.restype = ctypes.c_int
+        L.bqo_embed_rows.argtypes = [ctypes.c_int, u8p, u16p, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.c_int64, u16p]
+        L.bqo_embed_rows.restype = ctypes.c_int
         L.bqo_max_threads.argtypes = []
         L.bqo_max_threads.restype = ctypes.c_int
         _lib = L
@@ -240,6 +243,19 @@ def mlp_swiglu(fmt, gu_codes, gu_scales, d_codes, d_scales, hidden: int, inter: 
     act, _ = swiglu(h)
     y, bound = matmul(fmt, d_codes, d_scales, hidden, inter, act)
     return y, bound, act
+
+
+def embed_rows(fmt, codes, scales, n: int, k: int, ids) -> np.ndarray:
+    """BF16 bits [count][k] of the dequantised rows ids of an n x k table."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    out = np.zeros((ids.size, k), dtype=np.uint16)
+    st = lib().bqo_embed_rows(_fmt(fmt), _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_uint16), n, k,
+                              _ptr(ids, ctypes.c_int32), ids.size, _ptr(out, ctypes.c_uint16))
+    if st != OK:
+        raise OracleError(st, "embed_rows")
+    return out
 
 
 def max_threads() -> int:

@@ -369,3 +369,28 @@ int bqo_swiglu(const double* h, int64_t batch, int64_t inter, uint16_t* act_bf16
     }
     return BQO_OK;
 }
+
+/* ------------------------------------------------------------ embedding rows */
+/* Embedding lookup on a low-bit table ("1-bit Bonsai 8B" notes, section 3 and
+ * Table 1: the embedding layer is low-bit too): row ids[i] of the table,
+ * dequantised as s * q in FP64 (exact) and rounded once to BF16. */
+int bqo_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                   const int32_t* ids, int64_t count, uint16_t* out_bf16) {
+    if (fmt != BQO_Q1G128 && fmt != BQO_T2G128 && fmt != BQO_T5P8G128) return BQO_ERR_FORMAT;
+    if (n < 0 || k < 0 || k % GROUP || count < 0) return BQO_ERR_SHAPE;
+    if (count == 0 || k == 0) return BQO_OK;
+    if (!codes || !scales || !ids || !out_bf16) return BQO_ERR_NULL;
+    const int64_t row_bytes = bqo_codes_bytes(fmt, 1, k);
+    const int64_t G = k / GROUP;
+    for (int64_t i = 0; i < count; ++i) {
+        const int64_t r = ids[i];
+        if (r < 0 || r >= n) return BQO_ERR_SHAPE;
+        const uint8_t* row = codes + r * row_bytes;
+        for (int64_t kk = 0; kk < k; ++kk) {
+            const double s = bqo_half_to_double(scales[r * G + kk / GROUP]);
+            const int q = bqo_weight_code(fmt, row, kk);
+            out_bf16[i * k + kk] = bqo_double_to_bf16(s * (double)q);
+        }
+    }
+    return BQO_OK;
+}

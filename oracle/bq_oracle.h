@@ -77,6 +77,12 @@ int bqo_matmul_rows(int fmt, const uint8_t* codes, const uint16_t* scales,
  * computed in FP64; act_f64 (may be NULL) receives the unrounded values. */
 int bqo_swiglu(const double* h, int64_t batch, int64_t inter, uint16_t* act_bf16, double* act_f64);
 
+/* Embedding lookup: out[i][k] = BF16_RNE(s[ids[i]][k/128] * q[ids[i]][k])
+ * (the product in FP64 is exact), for i < count.  An id outside [0, n) is
+ * BQO_ERR_SHAPE. */
+int bqo_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                   const int32_t* ids, int64_t count, uint16_t* out_bf16);
+
 /* Number of OpenMP threads a call with nthreads <= 0 would use. */
 int bqo_max_threads(void);
 

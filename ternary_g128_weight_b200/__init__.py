@@ -29,7 +29,7 @@ EXPORTED = [
     "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8",
     "bq_gemv_workspace_bytes", "bq_gemv_launches", "bq_gemv", "bq_gemv_noalloc",
     "bq_gemm_workspace_bytes", "bq_gemm_launches", "bq_gemm",
-    "bq_gemv_chain_workspace_bytes", "bq_gemv_chain",
+    "bq_gemv_chain_workspace_bytes", "bq_gemv_chain", "bq_embed_rows",
     "bq_check", "bq_debug_wait_timeout", "bq_status_string", "bq_version",
 ]
 
@@ -74,6 +74,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.bq_gemm_workspace_bytes.argtypes = [i32, i64, i64, i64]; L.bq_gemm_workspace_bytes.restype = i64
     L.bq_gemm_launches.argtypes = [i32, i64, i64, i64]; L.bq_gemm_launches.restype = i32
     L.bq_gemm.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]; L.bq_gemm.restype = i32
+    L.bq_embed_rows.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp]; L.bq_embed_rows.restype = i32
     L.bq_gemv_chain_workspace_bytes.argtypes = []; L.bq_gemv_chain_workspace_bytes.restype = i64
     L.bq_gemv_chain.argtypes = [i32, ctypes.POINTER(ChainStep), i32, i32, vp, sz, vp]
     L.bq_gemv_chain.restype = i32
@@ -234,6 +235,19 @@ def bq_gemm(fmt, codes, scales, n: int, k: int, x, y=None, workspace=None, strea
                         _ptr(workspace), wsb, _stream(stream))
     _check(st, "bq_gemm")
     return y
+
+
+# --------------------------------------------------------------- embedding
+def bq_embed_rows(fmt, codes, scales, n: int, k: int, ids, out=None, stream=None):
+    """BF16 rows ids (int32 CUDA tensor) of the n x k low-bit table, [count][k]."""
+    import torch
+    ids = ids.reshape(-1)
+    if out is None:
+        out = torch.empty((ids.numel(), k), dtype=torch.bfloat16, device=ids.device)
+    st = load().bq_embed_rows(_fmt(fmt), _ptr(codes), _ptr(scales), n, k, _ptr(ids), ids.numel(), _ptr(out),
+                              _stream(stream))
+    _check(st, "bq_embed_rows")
+    return out
 
 
 # ------------------------------------------------------------------ chains

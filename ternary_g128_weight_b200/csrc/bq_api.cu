@@ -231,6 +231,18 @@ bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
+bq_status bq_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                        const int32_t* ids, int64_t count, uint16_t* out, void* stream) {
+    bq_status st = validate_matrix(fmt, codes, scales, n, k);
+    if (st != BQ_OK) return st;
+    if (count < 0 || count > (int64_t)INT32_MAX * 8) return BQ_ERR_SHAPE;
+    if (count == 0 || k == 0) return BQ_OK;
+    if (!ids || !out) return BQ_ERR_NULL;
+    if (!aligned(ids, 4) || !aligned(out, 16)) return BQ_ERR_ALIGN;
+    const cudaError_t e = launch_embed_rows(fmt, codes, scales, n, k, ids, count, out, as_stream(stream));
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 int64_t bq_gemv_chain_workspace_bytes(void) { return 256; }
 
 bq_status bq_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch,

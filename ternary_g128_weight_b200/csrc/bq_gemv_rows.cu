@@ -198,29 +198,32 @@ __device__ __forceinline__ int prep_class_shift(int P, int m) {
 // (value 4j + m of raw); 2-bit: the pairs k = 32t + 4j + 2P + {0,1} and
 // 32t + 16 + 4j + 2P + {0,1} (words 2j and 2j + 1 of raw); 5-trit: all 32
 // activations of thread t (value r of raw, both pairs).  xg is the group's
-// first activation (16-byte aligned).  The loads go through L2 (not the
-// non-coherent path): in the chain kernel x may have been written by other
-// CTAs of the same launch.
-template <int FMT>
+// first activation (16-byte aligned).  COHERENT: the loads go through L2 (the
+// chain kernel, where x may have been written by other CTAs of the same
+// launch); otherwise through the non-coherent cached path.
+template <bool COHERENT, typename T>
+__device__ __forceinline__ T ld_x(const T* p) { return COHERENT ? __ldcg(p) : __ldg(p); }
+
+template <int FMT, bool COHERENT>
 __device__ __forceinline__ void load_task_x(const uint16_t* xg, int t, int P, uint32_t (&raw)[16]) {
     if (FMT == BQ_Q1G128) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint2 v = __ldcg(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
+            const uint2 v = ld_x<COHERENT>(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
             raw[2 * j] = v.x;
             raw[2 * j + 1] = v.y;
         }
     } else if (FMT == BQ_T2G128) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            raw[2 * j] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 4 * j + 2 * P));
-            raw[2 * j + 1] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 32 * t + 16 + 4 * j + 2 * P));
+            raw[2 * j] = ld_x<COHERENT>(reinterpret_cast<const uint32_t*>(xg + 32 * t + 4 * j + 2 * P));
+            raw[2 * j + 1] = ld_x<COHERENT>(reinterpret_cast<const uint32_t*>(xg + 32 * t + 16 + 4 * j + 2 * P));
         }
     } else {
         const uint32_t* src = reinterpret_cast<const uint32_t*>(xg + 30 * t);  // 60 t bytes: 4-byte aligned
 #pragma unroll
-        for (int i = 0; i < 15; ++i) raw[i] = __ldcg(src + i);
-        raw[15] = __ldcg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
+        for (int i = 0; i < 15; ++i) raw[i] = ld_x<COHERENT>(src + i);
+        raw[15] = ld_x<COHERENT>(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
     }
 }
 
@@ -654,7 +657,7 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
 // it (copies issued) carry over from one call to the next.  False if a slot
 // wait timed out.
 template <int FMT>
-__device__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0,
+__device__ __forceinline__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0,
                         int rt1, Ring& rp, int& it, int lane) {
     constexpr int TCB = tile_code_bytes<FMT>();
     const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
@@ -684,8 +687,8 @@ __device__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t
 // of all of K).  Warp items (stage, batch row, half h of the stage's groups),
 // item i on warp i % NW; lane 8 gq + 2 t + P takes group 4 h + gq.  Rows go up
 // to the n-tiles' width (zero past the batch; one row at 16 lanes).
-template <int FMT, int NT, int LANES, int NW>
-__device__ void prep_x(const Params& p, uint8_t* smem, int warp, int lane) {
+template <int FMT, int NT, int LANES, int NW, bool COHERENT>
+__device__ __forceinline__ void prep_x(const Params& p, uint8_t* smem, int warp, int lane) {
     constexpr int kPrepBatch = 2;
     uint8_t* xres = smem + p.x_off;
     const int rows = LANES == 16 ? 1 : 2 * NT;
@@ -699,7 +702,7 @@ __device__ void prep_x(const Params& p, uint8_t* smem, int warp, int lane) {
             const int sr = i >> 1, G = 4 * (i & 1) + gq;
             const int st = sr / rows, bb = sr - st * rows;
             if (i < items && bb < p.batch) {
-                load_task_x<FMT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, P, raw[j]);
+                load_task_x<FMT, COHERENT>(p.x + (int64_t)bb * p.k + (int64_t)st * 1024 + G * 128, t, P, raw[j]);
             } else {
 #pragma unroll
                 for (int w = 0; w < 16; ++w) raw[j][w] = 0u;
@@ -722,7 +725,7 @@ __device__ void prep_x(const Params& p, uint8_t* smem, int warp, int lane) {
 // step, whose chunks hold c gate and c up tiles and end with the SwiGLU
 // epilogue).  False if a wait timed out.
 template <int FMT, int NT, int LANES, int NW>
-__device__ bool run_chunks(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0, int rt1,
+__device__ __forceinline__ bool run_chunks(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0, int rt1,
                            Ring& rp, int warp, int lane) {
     const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
     for (int r = rt0; r < rt1;) {
@@ -817,7 +820,7 @@ __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
         }
     }
     ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
-    prep_x<FMT, NT, LANES, NW>(p, smem, warp, lane);
+    prep_x<FMT, NT, LANES, NW, false>(p, smem, warp, lane);
     bar_compute<NW>();
     Ring rp;
     rp.depth = p.slots;
@@ -953,7 +956,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
         const Params& p = cp.step[s];
         if (s > 0) ok = grid_wait<NW>(cp.bar, (unsigned int)(s * C), p0.status, flag);
         if (!ok) break;
-        prep_x<FMT, NT, LANES, NW>(p, smem, warp, lane);
+        prep_x<FMT, NT, LANES, NW, true>(p, smem, warp, lane);
         bar_compute<NW>();
         const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
         const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);

@@ -76,6 +76,10 @@ bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
 
+// Embedding lookup (bq_embed_rows).
+cudaError_t launch_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                              const int32_t* ids, int64_t count, uint16_t* out, cudaStream_t s);
+
 // Persistent layer chain (bq_gemv_chain): eligibility of the step list and
 // its launch; bar = the two zeroed barrier counters.
 bool gemv_chain_eligible(int fmt, const bq_chain_step* steps, int nsteps, int batch);

@@ -419,3 +419,36 @@ def test_swiglu_pins():
     assert np.all(act == 0x3F3B)
     assert np.all(y == inter * 0.73046875)
     assert np.all(bound == inter * 0.73046875)
+
+
+def test_embed_rows_pins():
+    """Embedding lookup (8B notes, section 3 and Table 1: the embedding layer is
+    low-bit too), pinned to values the definition fixes: bit 1 -> +s and bit 0
+    -> -s; a ternary zero is +0; the FP16 scale rounded once to BF16, ties to
+    even (1 + 2^-8 is a tie -> 1.0; 1 + 3 2^-8 -> 1 + 2^-6); the rows are the
+    ones asked for, in the order asked for; an id past the table is an error."""
+    n, k = 4, 256
+    codes = np.zeros(oracle.codes_bytes("q1g128", n, k), dtype=np.uint8).reshape(n, k // 8)
+    codes[1] = 0xFF                                 # row 1: every weight +s
+    codes[2, 0] = 0x01                              # row 2: weight 0 +s, the rest -s
+    scales = np.array([[0x3C00, 0x3C00], [0x3C04, 0x3C0C], [0x4000, 0x3800], [0x0001, 0x7BFF]],
+                      dtype=np.uint16)              # 1, 1; 1+2^-8, 1+3*2^-8; 2, 0.5; 2^-24, 65504
+    out = oracle.embed_rows("q1g128", codes.reshape(-1), scales.reshape(-1), n, k, [1, 0, 2, 3, 1])
+    assert out.shape == (5, k)
+    assert np.all(out[0, :128] == 0x3F80) and np.all(out[0, 128:] == 0x3F82)   # +1.0 (tie), +1.015625
+    assert np.array_equal(out[4], out[0])
+    assert np.all(out[1] == 0xBF80)                                              # row 0: all -1.0
+    assert out[2, 0] == 0x4000 and np.all(out[2, 1:128] == 0xC000) and np.all(out[2, 128:] == 0xBF00)
+    assert np.all(out[3, :128] == 0xB380)           # -2^-24 in BF16 (exactly representable)
+    assert np.all(out[3, 128:] == 0xC780)           # -65504 -> BF16 RNE -65536
+    # ternary: zero trits give +0, t = +-1 gives +-s
+    t = np.array([[0, 1, -1, 0] * 32], dtype=np.float32)
+    tc, ts = oracle.pack("t2g128", t * 0.5, scales_in=np.array([0x3800], dtype=np.uint16))
+    o2 = oracle.embed_rows("t2g128", tc, ts, 1, 128, [0])
+    assert list(o2[0, :4]) == [0x0000, 0x3F00, 0xBF00, 0x0000]
+    t5c, t5s = oracle.pack("t5p8", t * 0.5, scales_in=np.array([0x3800], dtype=np.uint16))
+    assert np.array_equal(oracle.embed_rows("t5p8", t5c, t5s, 1, 128, [0]), o2)
+    with pytest.raises(oracle.OracleError):
+        oracle.embed_rows("q1g128", codes.reshape(-1), scales.reshape(-1), n, k, [4])
+    with pytest.raises(oracle.OracleError):
+        oracle.embed_rows("q1g128", codes.reshape(-1), scales.reshape(-1), n, k, [-1])
