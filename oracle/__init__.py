@@ -32,8 +32,8 @@ import numpy as np
 
 from . import build as _build
 
-Q1G128, T2G128, T5P8G128 = 1, 2, 3
-FORMATS = {"q1g128": Q1G128, "t2g128": T2G128, "t5p8": T5P8G128}
+Q1G128, T2G128, T5P8G128, A1G128 = 1, 2, 3, 4
+FORMATS = {"q1g128": Q1G128, "t2g128": T2G128, "t5p8": T5P8G128, "a1g128": A1G128}
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_NONFINITE, ERR_SCALE_RANGE, ERR_FORMAT = range(7)
 GROUP = 128
 
@@ -82,6 +82,14 @@ def lib():
         L.bqo_embed_rows.argtypes = [ctypes.c_int, u8p, u16p, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int64, u16p]
         L.bqo_embed_rows.restype = ctypes.c_int
+        L.bqo_pack_affine.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int64, ctypes.c_int64, u16p, u8p, u16p]
+        L.bqo_pack_affine.restype = ctypes.c_int
+        L.bqo_matmul_affine.argtypes = [u8p, u16p, ctypes.c_int64, ctypes.c_int64, u16p, ctypes.c_int64, i64p,
+                                        ctypes.c_int64, f64p, f64p, ctypes.c_int]
+        L.bqo_matmul_affine.restype = ctypes.c_int
+        L.bqo_embed_rows_affine.argtypes = [u8p, u16p, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.POINTER(ctypes.c_int32), ctypes.c_int64, u16p]
+        L.bqo_embed_rows_affine.restype = ctypes.c_int
         L.bqo_max_threads.argtypes = []
         L.bqo_max_threads.restype = ctypes.c_int
         _lib = L
@@ -255,6 +263,52 @@ def embed_rows(fmt, codes, scales, n: int, k: int, ids) -> np.ndarray:
                               _ptr(ids, ctypes.c_int32), ids.size, _ptr(out, ctypes.c_uint16))
     if st != OK:
         raise OracleError(st, "embed_rows")
+    return out
+
+
+def pack_affine(w: np.ndarray, params_in: np.ndarray | None = None):
+    """Affine 1-bit g128 (w' = s b + z): codes (as the binary format) and the
+    FP16 (s, z) pairs [N][G][2] (uint16 bits, flattened)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    codes = np.zeros(n * (k // 8), dtype=np.uint8)
+    params = np.zeros(n * (k // GROUP) * 2, dtype=np.uint16)
+    pin = None if params_in is None else np.ascontiguousarray(params_in, dtype=np.uint16).reshape(-1)
+    st = lib().bqo_pack_affine(w.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), n, k,
+                               None if pin is None else _ptr(pin, ctypes.c_uint16),
+                               _ptr(codes, ctypes.c_uint8), _ptr(params, ctypes.c_uint16))
+    if st != OK:
+        raise OracleError(st, "pack_affine")
+    return codes, params
+
+
+def matmul_affine(codes, params, n: int, k: int, x_bf16: np.ndarray, rows=None, nthreads: int = 0):
+    """y[b][rows] and bound[b][rows] of the affine product (all rows if rows is None)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16).reshape(-1, k)
+    batch = x.shape[0]
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    params = np.ascontiguousarray(params, dtype=np.uint16)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    R = n if r is None else r.size
+    y = np.zeros((batch, R), dtype=np.float64)
+    bound = np.zeros((batch, R), dtype=np.float64)
+    st = lib().bqo_matmul_affine(_ptr(codes, ctypes.c_uint8), _ptr(params, ctypes.c_uint16), n, k,
+                                 _ptr(x, ctypes.c_uint16), batch, None if r is None else _ptr(r, ctypes.c_int64),
+                                 R, _ptr(y, ctypes.c_double), _ptr(bound, ctypes.c_double), int(nthreads))
+    if st != OK:
+        raise OracleError(st, "matmul_affine")
+    return y, bound
+
+
+def embed_rows_affine(codes, params, n: int, k: int, ids) -> np.ndarray:
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    params = np.ascontiguousarray(params, dtype=np.uint16)
+    out = np.zeros((ids.size, k), dtype=np.uint16)
+    st = lib().bqo_embed_rows_affine(_ptr(codes, ctypes.c_uint8), _ptr(params, ctypes.c_uint16), n, k,
+                                     _ptr(ids, ctypes.c_int32), ids.size, _ptr(out, ctypes.c_uint16))
+    if st != OK:
+        raise OracleError(st, "embed_rows_affine")
     return out
 
 

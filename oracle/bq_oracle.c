@@ -121,8 +121,8 @@ static int fmt_ok(int fmt) {
 }
 
 int64_t bqo_codes_bytes(int fmt, int64_t n, int64_t k) {
-    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % GROUP) return -1;
-    if (fmt == BQO_Q1G128) return n * (k / 8);
+    if ((!fmt_ok(fmt) && fmt != BQO_A1G128) || n < 0 || k < 0 || k % GROUP) return -1;
+    if (fmt == BQO_Q1G128 || fmt == BQO_A1G128) return n * (k / 8);
     if (fmt == BQO_T2G128) return n * (k / 4);
     return n * (k / GROUP) * 26;
 }
@@ -133,6 +133,8 @@ int64_t bqo_scales_bytes(int64_t n, int64_t k) {
 }
 
 double bqo_effective_bits(int fmt) {
+    if (fmt == BQO_A1G128) /* one bit plus an FP16 (scale, bias) pair per 128 */
+        return 8.0 * (double)(bqo_codes_bytes(fmt, 1, GROUP) + 4) / (double)GROUP;
     if (!fmt_ok(fmt)) return -1.0;
     /* bytes for one 128-weight group: codes + 2-byte scale, in bits / 128 */
     return 8.0 * (double)(bqo_codes_bytes(fmt, 1, GROUP) + 2) / (double)GROUP;
@@ -390,6 +392,110 @@ int bqo_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_
             const double s = bqo_half_to_double(scales[r * G + kk / GROUP]);
             const int q = bqo_weight_code(fmt, row, kk);
             out_bf16[i * k + kk] = bqo_double_to_bf16(s * (double)q);
+        }
+    }
+    return BQO_OK;
+}
+
+/* ------------------------------------------------------------ affine 1-bit */
+static int affine_bit(const uint8_t* row, int64_t k) { return (row[k >> 3] >> (k & 7)) & 1; }
+
+int bqo_pack_affine(const float* w, int64_t n, int64_t k, const uint16_t* params_in,
+                    uint8_t* codes, uint16_t* params) {
+    if (n < 0 || k < 0 || k % GROUP) return BQO_ERR_SHAPE;
+    if (n == 0 || k == 0) return BQO_OK;
+    if (!w || !codes || !params) return BQO_ERR_NULL;
+    const int64_t G = k / GROUP;
+    memset(codes, 0, (size_t)(n * (k / 8)));
+    for (int64_t r = 0; r < n; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            const float* wg = w + r * k + g * GROUP;
+            for (int i = 0; i < GROUP; ++i)
+                if (!isfinite(wg[i])) return BQO_ERR_NONFINITE;
+            uint16_t sh, zh;
+            if (params_in) {
+                sh = params_in[(r * G + g) * 2];
+                zh = params_in[(r * G + g) * 2 + 1];
+                if ((sh & 0x8000) || (sh & 0x7C00) == 0x7C00 || (zh & 0x7C00) == 0x7C00) return BQO_ERR_SCALE_RANGE;
+            } else {
+                double lo = wg[0], hi = wg[0];
+                for (int i = 1; i < GROUP; ++i) {
+                    if (wg[i] < lo) lo = wg[i];
+                    if (wg[i] > hi) hi = wg[i];
+                }
+                zh = bqo_double_to_half(lo);
+                sh = bqo_double_to_half(hi - lo); /* exact in FP64 for two floats */
+                if ((sh & 0x7C00) == 0x7C00 || (zh & 0x7C00) == 0x7C00) return BQO_ERR_SCALE_RANGE;
+            }
+            params[(r * G + g) * 2] = sh;
+            params[(r * G + g) * 2 + 1] = zh;
+            const double sv = bqo_half_to_double(sh), zv = bqo_half_to_double(zh);
+            uint8_t* row = codes + r * (k / 8);
+            for (int i = 0; i < GROUP; ++i) {
+                const int64_t kk = g * GROUP + i;
+                if ((double)wg[i] - zv > sv / 2.0) row[kk >> 3] |= (uint8_t)(1u << (kk & 7));
+            }
+        }
+    }
+    return BQO_OK;
+}
+
+int bqo_matmul_affine(const uint8_t* codes, const uint16_t* params, int64_t n, int64_t k,
+                      const uint16_t* x, int64_t batch, const int64_t* rows, int64_t nrows,
+                      double* y, double* bound, int nthreads) {
+    if (n < 0 || k < 0 || k % GROUP || batch < 0) return BQO_ERR_SHAPE;
+    const int64_t R = rows ? nrows : n;
+    if (R < 0) return BQO_ERR_SHAPE;
+    if (R == 0 || batch == 0) return BQO_OK;
+    if (!codes || !params || !x || !y || !bound) return BQO_ERR_NULL;
+    if (rows)
+        for (int64_t i = 0; i < R; ++i)
+            if (rows[i] < 0 || rows[i] >= n) return BQO_ERR_SHAPE;
+    const int64_t G = k / GROUP;
+#ifdef _OPENMP
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel for num_threads(nt) schedule(dynamic, 16)
+#endif
+    for (int64_t i = 0; i < R; ++i) {
+        const int64_t r = rows ? rows[i] : i;
+        const uint8_t* row = codes + r * (k / 8);
+        for (int64_t b = 0; b < batch; ++b) {
+            const uint16_t* xb = x + b * k;
+            double acc = 0.0, bnd = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                const double sv = bqo_half_to_double(params[(r * G + g) * 2]);
+                const double zv = bqo_half_to_double(params[(r * G + g) * 2 + 1]);
+                double ax = 0.0;
+                for (int j = 0; j < GROUP; ++j) {
+                    const int64_t kk = g * GROUP + j;
+                    const double xv = bqo_bf16_to_double(xb[kk]);
+                    acc += (sv * (double)affine_bit(row, kk) + zv) * xv;
+                    ax += fabs(xv);
+                }
+                bnd += (fabs(sv) + fabs(zv)) * ax;
+            }
+            y[b * R + i] = acc;
+            bound[b * R + i] = bnd;
+        }
+    }
+    (void)nthreads;
+    return BQO_OK;
+}
+
+int bqo_embed_rows_affine(const uint8_t* codes, const uint16_t* params, int64_t n, int64_t k,
+                          const int32_t* ids, int64_t count, uint16_t* out_bf16) {
+    if (n < 0 || k < 0 || k % GROUP || count < 0) return BQO_ERR_SHAPE;
+    if (count == 0 || k == 0) return BQO_OK;
+    if (!codes || !params || !ids || !out_bf16) return BQO_ERR_NULL;
+    const int64_t G = k / GROUP;
+    for (int64_t i = 0; i < count; ++i) {
+        const int64_t r = ids[i];
+        if (r < 0 || r >= n) return BQO_ERR_SHAPE;
+        for (int64_t kk = 0; kk < k; ++kk) {
+            const int64_t g = kk / GROUP;
+            const double sv = bqo_half_to_double(params[(r * G + g) * 2]);
+            const double zv = bqo_half_to_double(params[(r * G + g) * 2 + 1]);
+            out_bf16[i * k + kk] = bqo_double_to_bf16(sv * (double)affine_bit(codes + r * (k / 8), kk) + zv);
         }
     }
     return BQO_OK;

@@ -32,7 +32,7 @@ extern "C" {
 
 enum { BQO_OK = 0, BQO_ERR_NULL = 1, BQO_ERR_SHAPE = 2, BQO_ERR_ALIGN = 3,
        BQO_ERR_NONFINITE = 4, BQO_ERR_SCALE_RANGE = 5, BQO_ERR_FORMAT = 6 };
-enum { BQO_Q1G128 = 1, BQO_T2G128 = 2, BQO_T5P8G128 = 3 };
+enum { BQO_Q1G128 = 1, BQO_T2G128 = 2, BQO_T5P8G128 = 3, BQO_A1G128 = 4 };
 
 /* IEEE-754 binary16 and bfloat16, written from the encoding definitions. */
 double   bqo_half_to_double(uint16_t h);
@@ -82,6 +82,29 @@ int bqo_swiglu(const double* h, int64_t batch, int64_t inter, uint16_t* act_bf16
  * BQO_ERR_SHAPE. */
 int bqo_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                    const int32_t* ids, int64_t count, uint16_t* out_bf16);
+
+/* Affine 1-bit g128, the MLX-style variant ("Bonsai-27B-mlx-1bit ... Binary
+ * g128", section "MLX打包优化": MLX's grouped low-bit format stores a scale and a
+ * bias per group; "1-bit Bonsai 8B" notes, Table 2: the MLX 1-bit (g128)
+ * package): w' = s * b + z, b in {0, 1} stored as the binary format stores its
+ * bits, one FP16 pair (s, z) per 128 weights in params [N][G][2].
+ * Packing (a reading; the pages give no rule): z = FP16_RNE(min w),
+ * s = FP16_RNE(max w - min w), b = 1 iff w - z > s/2 (FP64, a tie gives 0),
+ * i.e. round_half_even((w - z) / s) in {0, 1}.  params_in (or NULL): given
+ * pairs, s finite without its sign bit, z finite.
+ * Product: y = sum_g sum_{k in g} (s_g b_k + z_g) x_k (FP64) for the rows listed
+ * (rows == NULL: every row, output [batch][n]); bound = sum_g (|s_g| + |z_g|)
+ * sum_{k in g} |x_k|, the scale of the tolerance (over every k, as for the
+ * ternary formats).
+ * Embedding: out[i][k] = BF16_RNE(s b + z) of row ids[i] (FP64 exact before the
+ * rounding). */
+int bqo_pack_affine(const float* w, int64_t n, int64_t k, const uint16_t* params_in,
+                    uint8_t* codes, uint16_t* params);
+int bqo_matmul_affine(const uint8_t* codes, const uint16_t* params, int64_t n, int64_t k,
+                      const uint16_t* x, int64_t batch, const int64_t* rows, int64_t nrows,
+                      double* y, double* bound, int nthreads);
+int bqo_embed_rows_affine(const uint8_t* codes, const uint16_t* params, int64_t n, int64_t k,
+                          const int32_t* ids, int64_t count, uint16_t* out_bf16);
 
 /* Number of OpenMP threads a call with nthreads <= 0 would use. */
 int bqo_max_threads(void);

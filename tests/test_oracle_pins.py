@@ -452,3 +452,79 @@ def test_embed_rows_pins():
         oracle.embed_rows("q1g128", codes.reshape(-1), scales.reshape(-1), n, k, [4])
     with pytest.raises(oracle.OracleError):
         oracle.embed_rows("q1g128", codes.reshape(-1), scales.reshape(-1), n, k, [-1])
+
+
+def test_affine_storage_pins(golden_dir):
+    """Affine 1-bit g128 (MLX-style): one bit plus an FP16 (scale, bias) pair per
+    128 weights is 1 + 32/128 = 1.25 bits/weight (page 1, 'MLX打包优化': a scale
+    and a bias per group).  For the weight count behind Table 2's GGUF figure
+    (1,151,820,864 B at 18 B per 128 weights) that is GGUF x 20/18 =
+    1,279,800,960 B, 0.026% under Table 2's MLX 1-bit (g128) package
+    (1,280,131,424 B, which also holds the tensors kept unquantised)."""
+    facts = json.load(open(os.path.join(golden_dir, "page_facts.json")))
+    t2 = facts["table2_bytes"]
+    assert oracle.effective_bits("a1g128") == 1.25
+    assert oracle.codes_bytes("a1g128", 3, 256) == 3 * 32
+    weights = t2["gguf_q1_0_g128"] * 128 // 18
+    affine_bytes = weights * (16 + 4) // 128
+    assert affine_bytes * 18 == t2["gguf_q1_0_g128"] * 20
+    assert 0 < t2["mlx_1bit_g128"] - affine_bytes < 0.0003 * t2["mlx_1bit_g128"]
+    assert facts["mlx_scale_and_bias"]["params_per_group"] == ["scale", "bias"]
+
+
+def test_affine_oracle_pins():
+    """The affine product pinned to the native binary product: a native group
+    (bits, s) written as affine pairs (2s, -s) gives the same y (w' = 2 s b - s);
+    two-level groups reconstruct exactly; a weight exactly half a step above the
+    bias takes bit 0 (round half to even), just above it bit 1; one-hot x returns
+    the dequantised column; brute force against numpy on a tiny matrix."""
+    g = synth.rng(71)
+    n, k = 24, 512
+    w = synth.weights_normal(g, n, k)
+    qc, qs = oracle.pack("q1g128", w)
+    x = synth.x_bf16(g, 3, k)
+    y_native, _ = oracle.matmul("q1g128", qc, qs, n, k, x)
+    s = np.array([oracle.half_to_double(h) for h in qs], dtype=np.float64)
+    pairs = np.stack([np.array([oracle.double_to_half(2 * v) for v in s], dtype=np.uint16),
+                      np.array([oracle.double_to_half(-v) for v in s], dtype=np.uint16)], axis=1)
+    ac, ap = oracle.pack_affine(oracle.dequant("q1g128", qc, qs, n, k).astype(np.float32), params_in=pairs)
+    assert np.array_equal(ac, qc)                 # the same bits
+    y_aff, bound = oracle.matmul_affine(ac, ap, n, k, x)
+    np.testing.assert_allclose(y_aff, y_native, rtol=1e-12, atol=1e-300)
+    assert np.all(bound > 0)
+    # two levels a < b (FP16-exact, b - a FP16-exact): exact reconstruction
+    a, b = -0.375, 0.625
+    lv = np.where(g.random((2, 256)) < 0.5, a, b).astype(np.float32)
+    lv[:, 0], lv[:, 1] = a, b
+    c2, p2 = oracle.pack_affine(lv)
+    assert list(p2[:2]) == [oracle.double_to_half(1.0), oracle.double_to_half(a)]
+    one = np.zeros((1, 256), dtype=np.uint16)
+    for kk in (0, 1, 130, 255):
+        xh = one.copy()
+        xh[0, kk] = 0x3F80                         # BF16 1.0
+        yy, _ = oracle.matmul_affine(c2, p2, 2, 256, xh)
+        assert list(yy[0]) == list(lv[:, kk].astype(np.float64))
+    # tie: min 0, max 1 -> s = 1, z = 0; w = 0.5 -> bit 0, w = 0.5 + 2^-20 -> bit 1
+    tw = np.zeros((1, 128), dtype=np.float32)
+    tw[0, 1] = 1.0
+    tw[0, 2] = 0.5
+    tw[0, 3] = 0.5 + 2.0 ** -20
+    tc, tp = oracle.pack_affine(tw)
+    assert (tc[0] >> 1) & 1 == 1 and (tc[0] >> 2) & 1 == 0 and (tc[0] >> 3) & 1 == 1
+    # brute force against numpy: bits from the pinned binary decoder, (s, z) from the pairs
+    wt = synth.weights_normal(g, 5, 256)
+    cc, pp = oracle.pack_affine(wt)
+    bits = (oracle.unpack("q1g128", cc, 5, 256).astype(np.float64) + 1) / 2
+    sz = np.array([oracle.half_to_double(h) for h in pp], dtype=np.float64).reshape(5, 2, 2)
+    wd = bits * np.repeat(sz[:, :, 0], 128, axis=1) + np.repeat(sz[:, :, 1], 128, axis=1)
+    xt = synth.x_bf16(g, 2, 256)
+    xf = np.array([[oracle.bf16_to_double(v) for v in row] for row in xt])
+    yb, _ = oracle.matmul_affine(cc, pp, 5, 256, xt)
+    np.testing.assert_allclose(yb, xf @ wd.T, rtol=1e-12, atol=1e-15)
+    # every reconstruction within half a step of its weight (plus the FP16 roundings)
+    err = np.abs(wd - wt.astype(np.float64))
+    step = np.repeat(sz[:, :, 0], 128, axis=1)
+    assert np.all(err <= step / 2 + 2.0 ** -10 * (np.abs(wt) + step))
+    # embedding: the dequantised row rounded once to BF16
+    e = oracle.embed_rows_affine(cc, pp, 5, 256, [4, 0])
+    assert e[0, 0] == oracle.double_to_bf16(wd[4, 0]) and e[1, 255] == oracle.double_to_bf16(wd[0, 255])
