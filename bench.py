@@ -31,7 +31,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-FMT_NAMES = {"q1g128": 1, "t2g128": 2, "t5p8": 3}
+FMT_NAMES = {"q1g128": 1, "t2g128": 2, "t5p8": 3, "a1g128": 4}
 
 
 def parse():
@@ -352,10 +352,10 @@ def make_weights(fmt, n, k, gen, dev, direct_codes):
     import torch
     import synth
     import ternary_g128_weight_b200 as bq
-    if fmt == "q1g128":
-        if direct_codes:
-            return (synth.device_code_bytes(gen, bq.bq_codes_bytes(fmt, n, k), device=dev),
-                    synth.device_scales_uniform(gen, n, k // 128, device=dev).view(-1))
+    if fmt == "q1g128" and direct_codes:
+        return (synth.device_code_bytes(gen, bq.bq_codes_bytes(fmt, n, k), device=dev),
+                synth.device_scales_uniform(gen, n, k // 128, device=dev).view(-1))
+    if fmt in ("q1g128", "a1g128"):
         return bq.bq_pack(fmt, synth.device_weights_normal(gen, n, k, device=dev))
     t = synth.device_trits(gen, n, k, device=dev)
     s = synth.device_scales_uniform(gen, n, k // 128, device=dev)
@@ -529,12 +529,13 @@ def leg(model, fmt, batch, mode, dev, steps, warmup, peak, seed):
 
 # The secondary configurations: the Qwen3-8B shapes in both ternary formats
 # at batch 1 and 16 and in binary at batch 8, the 27B class in all three
-# formats at batch 1 and 16, and the binary Qwen3-8B pass as per-layer chains.
+# formats at batch 1 and 16, the binary Qwen3-8B pass as per-layer chains, and
+# the affine 1-bit variant (scale and bias per group) at batch 1.
 LEGS = [("qwen3-8b", "t2g128", 1, "calls"), ("qwen3-8b", "t5p8", 1, "calls"), ("qwen3-8b", "q1g128", 8, "calls"),
         ("qwen3-8b", "t2g128", 16, "calls"), ("qwen3-8b", "t5p8", 16, "calls"),
         ("27b", "q1g128", 1, "calls"), ("27b", "t2g128", 1, "calls"), ("27b", "t5p8", 1, "calls"),
         ("27b", "q1g128", 16, "calls"), ("27b", "t2g128", 16, "calls"), ("27b", "t5p8", 16, "calls"),
-        ("qwen3-8b", "q1g128", 1, "chain")]
+        ("qwen3-8b", "q1g128", 1, "chain"), ("qwen3-8b", "a1g128", 1, "calls")]
 
 
 # ----------------------------------------------------------------------- ours

@@ -24,6 +24,16 @@
  *            BQ_T5P8G128: [N][26*G] bytes; in group g, byte j < 25 holds
  *                         v = sum_{i<5} (q_{128g+5j+i}+1) 3^i, byte 25 holds the
  *                         last three codes the same way.      1.75 bits/weight
+ *            BQ_A1G128  : the BQ_Q1G128 bit layout, but bit b means s*b + z: the
+ *                         affine variant MLX packs ("Bonsai-27B-mlx-1bit ... Binary
+ *                         g128", section "MLX打包优化": a scale and a bias per
+ *                         group).  Its `scales` array holds FP16 (s, z) pairs
+ *                         [N][G][2].                          1.25 bits/weight
+ *                         Supported by the packer, bq_gemv / bq_gemv_noalloc on
+ *                         the row-owning path (batch <= 8, K % 1024 == 0) and
+ *                         bq_embed_rows; bq_gemm and bq_gemv_chain return
+ *                         BQ_ERR_FORMAT.  Tolerance scale for this format:
+ *                         sum_k (|s| + |z|) |x_k| over every k.
  *   x        BF16 bit patterns [B][K] (GEMV) or [T][K] (GEMM), contiguous.
  *   y        [B][N] (GEMV, BF16 or F32) or [T][N] (GEMM, BF16).
  *
@@ -72,7 +82,7 @@ typedef enum {
     BQ_ERR_WORKSPACE = 9    /* workspace NULL or smaller than *_workspace_bytes */
 } bq_status;
 
-typedef enum { BQ_Q1G128 = 1, BQ_T2G128 = 2, BQ_T5P8G128 = 3 } bq_format;
+typedef enum { BQ_Q1G128 = 1, BQ_T2G128 = 2, BQ_T5P8G128 = 3, BQ_A1G128 = 4 } bq_format;
 typedef enum { BQ_BF16 = 0, BQ_F32 = 1 } bq_dtype;
 
 #define BQ_GROUP 128
@@ -86,6 +96,9 @@ typedef enum { BQ_BF16 = 0, BQ_F32 = 1 } bq_dtype;
  * 3^5 = 243 <= 256 ("把 27B 模型压到 4GB" section 2.4 on both ternary
  * storages). */
 int64_t bq_codes_bytes(int fmt, int64_t n, int64_t k);
+/* Bytes of the group parameters of a format: N * (K/128) * 2 (one FP16 scale per
+ * group), or N * (K/128) * 4 for BQ_A1G128 ((scale, bias) pairs); -1 if invalid. */
+int64_t bq_group_params_bytes(int fmt, int64_t n, int64_t k);
 /* Bytes of the FP16 scale array, N * (K/128) * 2; -1 for an invalid shape.
  * One FP16 scale per 128 consecutive weights ("Bonsai-27B-mlx-1bit ...
  * Binary g128", section "Binary g128权重表示原理"). */
@@ -121,6 +134,14 @@ bq_status bq_pack_t2g128(const float* w, int64_t n, int64_t k, const uint16_t* s
                          uint8_t* codes, uint16_t* scales, void* stream);
 bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
                        uint8_t* codes, uint16_t* scales, void* stream);
+/* Affine 1-bit packer (BQ_A1G128).  Reading of the pages, which give no rule:
+ *   z = FP16_RNE(min w), s = FP16_RNE(max w - min w) (the difference exact in
+ *   FP64), b = 1 iff w - z > s/2 (FP64; a tie gives 0), unless params_in gives
+ *   the (s, z) pairs ([N][G][2] FP16: s finite with its sign bit clear, z
+ *   finite).  params: device FP16 [N][G][2].  Errors and synchronisation as the
+ *   other packers; the result is bit-exact with the reference definition. */
+bq_status bq_pack_a1g128(const float* w, int64_t n, int64_t k, const uint16_t* params_in,
+                         uint8_t* codes, uint16_t* params, void* stream);
 
 /* ------------------------------------------------------------------- GEMV */
 /* Workspace bytes bq_gemv needs for this call shape (0 when none is needed);

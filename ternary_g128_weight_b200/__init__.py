@@ -19,14 +19,14 @@ LIB_PATH = os.path.join(PKG_DIR, "libbq.so")
 
 BQ_OK, BQ_ERR_NULL, BQ_ERR_SHAPE, BQ_ERR_ALIGN, BQ_ERR_NONFINITE = 0, 1, 2, 3, 4
 BQ_ERR_SCALE_RANGE, BQ_ERR_FORMAT, BQ_ERR_CUDA, BQ_ERR_TIMEOUT, BQ_ERR_WORKSPACE = 5, 6, 7, 8, 9
-BQ_Q1G128, BQ_T2G128, BQ_T5P8G128 = 1, 2, 3
+BQ_Q1G128, BQ_T2G128, BQ_T5P8G128, BQ_A1G128 = 1, 2, 3, 4
 BQ_BF16, BQ_F32 = 0, 1
 BQ_GROUP, BQ_MAX_BATCH = 128, 16
-FORMATS = {"q1g128": BQ_Q1G128, "t2g128": BQ_T2G128, "t5p8": BQ_T5P8G128}
+FORMATS = {"q1g128": BQ_Q1G128, "t2g128": BQ_T2G128, "t5p8": BQ_T5P8G128, "a1g128": BQ_A1G128}
 
 EXPORTED = [
-    "bq_codes_bytes", "bq_scales_bytes", "bq_effective_bits",
-    "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8",
+    "bq_codes_bytes", "bq_scales_bytes", "bq_group_params_bytes", "bq_effective_bits",
+    "bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8", "bq_pack_a1g128",
     "bq_gemv_workspace_bytes", "bq_gemv_launches", "bq_gemv", "bq_gemv_noalloc",
     "bq_gemm_workspace_bytes", "bq_gemm_launches", "bq_gemm",
     "bq_gemv_chain_workspace_bytes", "bq_gemv_chain", "bq_embed_rows",
@@ -62,8 +62,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
     L.bq_codes_bytes.argtypes = [i32, i64, i64]; L.bq_codes_bytes.restype = i64
     L.bq_scales_bytes.argtypes = [i64, i64]; L.bq_scales_bytes.restype = i64
+    L.bq_group_params_bytes.argtypes = [i32, i64, i64]; L.bq_group_params_bytes.restype = i64
     L.bq_effective_bits.argtypes = [i32]; L.bq_effective_bits.restype = ctypes.c_double
-    for name in ("bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8"):
+    for name in ("bq_pack_q1g128", "bq_pack_t2g128", "bq_pack_t5p8", "bq_pack_a1g128"):
         f = getattr(L, name)
         f.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         f.restype = i32
@@ -119,6 +120,10 @@ def bq_scales_bytes(n: int, k: int) -> int:
     return int(load().bq_scales_bytes(n, k))
 
 
+def bq_group_params_bytes(fmt, n: int, k: int) -> int:
+    return int(load().bq_group_params_bytes(_fmt(fmt), n, k))
+
+
 def bq_effective_bits(fmt) -> float:
     return float(load().bq_effective_bits(_fmt(fmt)))
 
@@ -131,7 +136,7 @@ def bq_version() -> int:
 def _pack(name: str, fmt: int, w, scales_in=None, codes=None, scales=None, stream=None):
     import torch
     n, k = w.shape
-    cb, sb = bq_codes_bytes(fmt, n, k), bq_scales_bytes(n, k)
+    cb, sb = bq_codes_bytes(fmt, n, k), bq_group_params_bytes(fmt, n, k)
     if cb < 0 or sb < 0:
         raise BQError(BQ_ERR_SHAPE, name)
     if codes is None:
@@ -156,7 +161,13 @@ def bq_pack_t5p8(w, scales_in=None, codes=None, scales=None, stream=None):
     return _pack("bq_pack_t5p8", BQ_T5P8G128, w, scales_in, codes, scales, stream)
 
 
-PACKERS = {BQ_Q1G128: bq_pack_q1g128, BQ_T2G128: bq_pack_t2g128, BQ_T5P8G128: bq_pack_t5p8}
+def bq_pack_a1g128(w, params_in=None, codes=None, params=None, stream=None):
+    """Affine 1-bit: (codes uint8, params int16 holding FP16 (scale, bias) pairs [N][G][2])."""
+    return _pack("bq_pack_a1g128", BQ_A1G128, w, params_in, codes, params, stream)
+
+
+PACKERS = {BQ_Q1G128: bq_pack_q1g128, BQ_T2G128: bq_pack_t2g128, BQ_T5P8G128: bq_pack_t5p8,
+           BQ_A1G128: bq_pack_a1g128}
 
 
 def bq_pack(fmt, w, scales_in=None, codes=None, scales=None, stream=None):

@@ -14,7 +14,9 @@ __device__ unsigned long long g_pack_first_error = ~0ull;
 
 std::mutex g_pack_mutex;
 
-inline bool fmt_ok(int fmt) { return fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128; }
+inline bool fmt_ok(int fmt) {
+    return fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128 || fmt == BQ_A1G128;
+}
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
@@ -111,7 +113,7 @@ extern "C" {
 
 int64_t bq_codes_bytes(int fmt, int64_t n, int64_t k) {
     if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup) return -1;
-    if (fmt == BQ_Q1G128) return n * (k / 8);
+    if (fmt == BQ_Q1G128 || fmt == BQ_A1G128) return n * (k / 8);
     if (fmt == BQ_T2G128) return n * (k / 4);
     return n * (k / kGroup) * 26;
 }
@@ -121,9 +123,14 @@ int64_t bq_scales_bytes(int64_t n, int64_t k) {
     return n * (k / kGroup) * 2;
 }
 
+int64_t bq_group_params_bytes(int fmt, int64_t n, int64_t k) {
+    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup) return -1;
+    return n * (k / kGroup) * (fmt == BQ_A1G128 ? 4 : 2);
+}
+
 double bq_effective_bits(int fmt) {
     if (!fmt_ok(fmt)) return -1.0;
-    return 8.0 * (double)(bq_codes_bytes(fmt, 1, kGroup) + 2) / (double)kGroup;
+    return 8.0 * (double)(bq_codes_bytes(fmt, 1, kGroup) + bq_group_params_bytes(fmt, 1, kGroup)) / (double)kGroup;
 }
 
 bq_status bq_pack_q1g128(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
@@ -137,6 +144,10 @@ bq_status bq_pack_t2g128(const float* w, int64_t n, int64_t k, const uint16_t* s
 bq_status bq_pack_t5p8(const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
                        uint8_t* codes, uint16_t* scales, void* stream) {
     return pack_common(BQ_T5P8G128, w, n, k, scales_in, codes, scales, stream);
+}
+bq_status bq_pack_a1g128(const float* w, int64_t n, int64_t k, const uint16_t* params_in,
+                         uint8_t* codes, uint16_t* params, void* stream) {
+    return pack_common(BQ_A1G128, w, n, k, params_in, codes, params, stream);
 }
 
 
@@ -192,7 +203,7 @@ static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
-    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
+    if (!fmt_ok(fmt) || fmt == BQ_A1G128 || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
     if (t == 0 || n == 0 || k == 0) return 0;
     if (gemm_uses_gemv(fmt, n, k, t)) return gemv_workspace_bytes(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_workspace_bytes(n, k, t);
@@ -200,7 +211,7 @@ int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {
 }
 
 int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t) {
-    if (!fmt_ok(fmt) || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
+    if (!fmt_ok(fmt) || fmt == BQ_A1G128 || n < 0 || k < 0 || k % kGroup || t < 0) return -1;
     if (t == 0 || n == 0 || k == 0) return 0;
     if (gemm_uses_gemv(fmt, n, k, t)) return bq_gemv_launches(fmt, n, k, (int)t);
     if (gemm_tc_eligible(fmt, n, k, t)) return gemm_tc_launches(n, k, t);
@@ -210,6 +221,7 @@ int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t) {
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                   const uint16_t* x, int64_t t, uint16_t* y, void* workspace, size_t workspace_bytes,
                   void* stream) {
+    if (fmt == BQ_A1G128) return BQ_ERR_FORMAT;  // the prefill GEMM does not take the affine variant
     bq_status st = validate_matrix(fmt, codes, scales, n, k);
     if (st != BQ_OK) return st;
     if (t < 0) return BQ_ERR_SHAPE;
@@ -247,7 +259,7 @@ int64_t bq_gemv_chain_workspace_bytes(void) { return 256; }
 
 bq_status bq_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch,
                         void* workspace, size_t workspace_bytes, void* stream) {
-    if (!fmt_ok(fmt)) return BQ_ERR_FORMAT;
+    if (!fmt_ok(fmt) || fmt == BQ_A1G128) return BQ_ERR_FORMAT;
     if (!steps) return BQ_ERR_NULL;
     if (nsteps < 1 || nsteps > BQ_MAX_CHAIN_STEPS || batch < 1 || batch > BQ_MAX_BATCH) return BQ_ERR_SHAPE;
     for (int i = 0; i < nsteps; ++i) {

@@ -17,7 +17,7 @@ constexpr int kWarpsPerBlock = 8;
 // Code of weight i of a group (0..127): +1 / -1 (binary), or the trit c - 1.
 template <int FMT>
 __device__ __forceinline__ void group_codes(const uint8_t* g, int lane, int (&q)[4]) {
-    if (FMT == BQ_Q1G128) {
+    if (FMT == BQ_Q1G128 || FMT == BQ_A1G128) {
         const uint32_t nib = (g[lane >> 1] >> (4 * (lane & 1))) & 0xFu;  // weights 4l .. 4l+3
 #pragma unroll
         for (int j = 0; j < 4; ++j) q[j] = ((nib >> j) & 1u) ? 1 : -1;
@@ -36,6 +36,19 @@ __device__ __forceinline__ void group_codes(const uint8_t* g, int lane, int (&q)
     }
 }
 
+// BF16 round-to-nearest-even of an FP64 value v whose magnitude is within the
+// FP32 range: truncate to FP32 (toward zero), then round the 16 discarded bits
+// with a sticky bit for what the truncation dropped (one rounding in all).
+__device__ __forceinline__ uint16_t f64_to_bf16_rn(double v) {
+    float t;
+    asm("cvt.rz.f32.f64 %0, %1;" : "=f"(t) : "d"(v));
+    const bool sticky = (double)t != v;
+    const uint32_t u = __float_as_uint(t), mag = u & 0x7FFFFFFFu, low = mag & 0xFFFFu;
+    uint32_t hi = mag >> 16;
+    if (low > 0x8000u || (low == 0x8000u && (sticky || (hi & 1u)))) ++hi;
+    return (uint16_t)(((u >> 16) & 0x8000u) | hi);
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     embed_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t n, int64_t k,
@@ -46,8 +59,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int lane = threadIdx.x & 31;
     if (i >= count) return;
     const int64_t G = k / 128;
-    const int64_t row_bytes = FMT == BQ_Q1G128 ? k / 8 : FMT == BQ_T2G128 ? k / 4 : G * 26;
-    constexpr int kGroupBytes = FMT == BQ_Q1G128 ? 16 : FMT == BQ_T2G128 ? 32 : 26;
+    constexpr bool kBits = FMT == BQ_Q1G128 || FMT == BQ_A1G128;
+    const int64_t row_bytes = kBits ? k / 8 : FMT == BQ_T2G128 ? k / 4 : G * 26;
+    constexpr int kGroupBytes = kBits ? 16 : FMT == BQ_T2G128 ? 32 : 26;
     const int32_t id = __ldg(ids + i);
     uint2* orow = reinterpret_cast<uint2*>(out + i * k);
     if (id < 0 || (int64_t)id >= n) {
@@ -57,6 +71,20 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         return;
     }
     const uint8_t* row = codes + (int64_t)id * row_bytes;
+    if (FMT == BQ_A1G128) {
+        // s b + z (exact in FP64), rounded once to BF16
+        const uint32_t* prow = reinterpret_cast<const uint32_t*>(scales) + (int64_t)id * G;
+        for (int64_t g = 0; g < G; ++g) {
+            const uint32_t pz = __ldg(prow + g);
+            const double sv = half_bits_to_float((uint16_t)(pz & 0xFFFFu)), zv = half_bits_to_float((uint16_t)(pz >> 16));
+            const uint32_t nib = (row[g * 16 + (lane >> 1)] >> (4 * (lane & 1))) & 0xFu;
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = f64_to_bf16_rn(((nib >> j) & 1u) ? sv + zv : zv);
+            orow[g * 32 + lane] = make_uint2(o[0] | (o[1] << 16), o[2] | (o[3] << 16));
+        }
+        return;
+    }
     const uint16_t* srow = scales + (int64_t)id * G;
     for (int64_t g = 0; g < G; ++g) {
         const float s = half_bits_to_float(__ldg(srow + g));
@@ -87,7 +115,9 @@ cudaError_t launch_embed_rows(int fmt, const uint8_t* codes, const uint16_t* sca
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (fmt == BQ_Q1G128)
+    if (fmt == BQ_A1G128)
+        e = cudaLaunchKernelEx(&cfg, embed_rows_kernel<BQ_A1G128>, codes, scales, n, k, ids, count, out, status);
+    else if (fmt == BQ_Q1G128)
         e = cudaLaunchKernelEx(&cfg, embed_rows_kernel<BQ_Q1G128>, codes, scales, n, k, ids, count, out, status);
     else if (fmt == BQ_T2G128)
         e = cudaLaunchKernelEx(&cfg, embed_rows_kernel<BQ_T2G128>, codes, scales, n, k, ids, count, out, status);

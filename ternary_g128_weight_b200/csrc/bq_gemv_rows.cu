@@ -8,6 +8,8 @@
 // operands of the warp MMA m16n8k32,
 //   binary : byte j of (w & (0x01010101 << p)) = 2^p * bit(8j+p),
 //   2-bit  : byte j of (w & (0x03030303 << 2i)) = 4^i * c(4j+i), c = q+1,
+//   affine : the binary bits, w = s b + z ("Bonsai-27B ... Binary g128", section
+//            "MLX打包优化": a scale and a bias per group),
 //   5-trit : a byte v = sum c_i 3^i ("把 27B 模型压到 4GB" section 2.4: 3^5 <= 256)
 //            gives c0..c3 as the four bytes of a 256-entry table word (one
 //            copy per lane in shared memory, so lookups never conflict) and
@@ -21,6 +23,7 @@
 // int32 column sums are recombined in FP32:
 //   binary : y += s * (2 * 2^-E * sum bit B 2^p - z)
 //   ternary: y += s * (    2^-E * sum c   B 4^i - z)
+//   affine : y += s * 2^-E * sum bit B 2^p + zb * z   (zb the group's bias)
 // with z the group's activation sum in FP32 ("Bonsai-27B ... Binary g128":
 // 0 -> -scale, 1 -> +scale; "1-bit Bonsai 8B" notes, section 4.1: one FP16
 // scale per 128 weights).
@@ -54,7 +57,16 @@ namespace rows {
 
 constexpr int kGroupsPerStage = 8;  // 1024 K per stage
 constexpr int kMaxChunkTiles = 8;   // chunk bound of the 2-bit and 5-trit formats
-constexpr int kTileScaleBytes = 16 * kGroupsPerStage * 2;  // 256
+constexpr int kTileScaleBytes = 16 * kGroupsPerStage * 2;  // 256: one FP16 scale per group
+// The bit formats: binary and affine share the code layout and its decode.
+template <int FMT>
+constexpr bool bits_fmt() { return FMT == BQ_Q1G128 || FMT == BQ_A1G128; }
+// FP16 values per group in the scale plane: the scale, or the (scale, bias)
+// pair of the affine format.
+template <int FMT>
+constexpr int spg() { return FMT == BQ_A1G128 ? 2 : 1; }
+template <int FMT>
+constexpr int tile_scale_bytes() { return kTileScaleBytes * spg<FMT>(); }
 constexpr int kMaxSlots = 8;
 constexpr int kSmemFull = 232448;  // opt-in shared memory per block on sm_100 (one CTA per SM)
 constexpr int kSmemHalf = 115712;  // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2
@@ -69,6 +81,11 @@ template <>
 struct Fmt<BQ_Q1G128> {
     static constexpr int kBoxes = 1;      // 128-byte columns per row tile and stage
     static constexpr int kCoefShift = 1;  // 2 * sum(bit * x) - sum(x)
+};
+template <>
+struct Fmt<BQ_A1G128> {
+    static constexpr int kBoxes = 1;
+    static constexpr int kCoefShift = 0;  // sum(bit * x), the bias term added apart
 };
 template <>
 struct Fmt<BQ_T2G128> {
@@ -92,7 +109,7 @@ constexpr int kBoxColumnBytes = kMaxChunkTiles * 16 * 128;  // 16 KB
 // Largest chunk (row tiles) a kernel is built for: 16 for the binary format
 // up to batch 4 (two row tiles per warp at NW = 8, one at NW = 16), else 8.
 template <int FMT, int NT>
-constexpr int mct() { return (FMT == BQ_Q1G128 && NT <= 2) ? 16 : kMaxChunkTiles; }
+constexpr int mct() { return (bits_fmt<FMT>() && NT <= 2) ? 16 : kMaxChunkTiles; }
 
 struct Params {
     const uint16_t* x;  // [batch][K] BF16
@@ -177,7 +194,7 @@ __device__ __forceinline__ int ilog2f(float m) {
 // through shuffles.
 template <int FMT>
 __device__ __forceinline__ constexpr int prep_src(int P, int m, int j) {
-    if (FMT == BQ_Q1G128) return 8 * j + 4 * P + m;                        // k = 32t + 8j + 2q + h
+    if (bits_fmt<FMT>()) return 8 * j + 4 * P + m;                        // k = 32t + 8j + 2q + h
     if (FMT == BQ_T2G128) return 16 * (m & 1) + 4 * j + 2 * P + (m >> 1);  // k = 32t + 16h + 4j + q
     if (P == 0) return 5 * m + j;                 // digits 0..3 of bytes 6t .. 6t+3
     if (m < 2) return 20 + 5 * m + j;             // digits 0..3 of bytes 6t+4, 6t+5
@@ -189,7 +206,7 @@ __device__ __forceinline__ constexpr int prep_src(int P, int m, int j) {
 // (binary: the bit's weight 2^class; 2-bit: 4^class).
 template <int FMT>
 __device__ __forceinline__ int prep_class_shift(int P, int m) {
-    if (FMT == BQ_Q1G128) return 4 * P + m;               // (8j + 4P + m) mod 8
+    if (bits_fmt<FMT>()) return 4 * P + m;               // (8j + 4P + m) mod 8
     if (FMT == BQ_T2G128) return 2 * (2 * P + (m >> 1));  // 2 * ((16(m&1) + 4j + 2P + (m>>1)) mod 4)
     return 0;
 }
@@ -206,7 +223,7 @@ __device__ __forceinline__ T ld_x(const T* p) { return COHERENT ? __ldcg(p) : __
 
 template <int FMT, bool COHERENT>
 __device__ __forceinline__ void load_task_x(const uint16_t* xg, int t, int P, uint32_t (&raw)[16]) {
-    if (FMT == BQ_Q1G128) {
+    if (bits_fmt<FMT>()) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint2 v = ld_x<COHERENT>(reinterpret_cast<const uint2*>(xg + 32 * t + 8 * j + 4 * P));
@@ -234,7 +251,7 @@ __device__ __forceinline__ float raw_value(const uint32_t (&raw)[16], int r) {
 // Activation (P, m, j) of the task (see load_task_x).
 template <int FMT>
 __device__ __forceinline__ float task_value(const uint32_t (&raw)[16], int P, int m, int j) {
-    if (FMT == BQ_Q1G128) return raw_value(raw, 4 * j + m);
+    if (bits_fmt<FMT>()) return raw_value(raw, 4 * j + m);
     if (FMT == BQ_T2G128) return raw_value(raw, 2 * (2 * j + (m & 1)) + (m >> 1));
     const float v0 = raw_value(raw, prep_src<FMT>(0, m, j)), v1 = raw_value(raw, prep_src<FMT>(1, m, j));
     return P ? v1 : v0;
@@ -342,16 +359,21 @@ __device__ __forceinline__ void t5_row(const uint8_t* p, const uint32_t* lut, in
 }
 
 // GPW consecutive FP16 scales (the warp's groups of one row and stage) as
-// packed pairs.
-template <int GPW>
-__device__ __forceinline__ void load_scales(const uint8_t* p, uint32_t (&s)[(GPW + 1) / 2]) {
-    if constexpr (GPW == 8) {
+// packed pairs; N = 2 * GPW values for the (scale, bias) pairs of the affine
+// format.
+template <int N>
+__device__ __forceinline__ void load_scales(const uint8_t* p, uint32_t (&s)[(N + 1) / 2]) {
+    if constexpr (N == 16) {
+        const uint4 v0 = *reinterpret_cast<const uint4*>(p), v1 = *reinterpret_cast<const uint4*>(p + 16);
+        s[0] = v0.x; s[1] = v0.y; s[2] = v0.z; s[3] = v0.w;
+        s[4] = v1.x; s[5] = v1.y; s[6] = v1.z; s[7] = v1.w;
+    } else if constexpr (N == 8) {
         const uint4 v = *reinterpret_cast<const uint4*>(p);
         s[0] = v.x; s[1] = v.y; s[2] = v.z; s[3] = v.w;
-    } else if constexpr (GPW == 4) {
+    } else if constexpr (N == 4) {
         const uint2 v = *reinterpret_cast<const uint2*>(p);
         s[0] = v.x; s[1] = v.y;
-    } else if constexpr (GPW == 2) {
+    } else if constexpr (N == 2) {
         s[0] = *reinterpret_cast<const uint32_t*>(p);
     } else {
         s[0] = *reinterpret_cast<const uint16_t*>(p);
@@ -396,12 +418,14 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     auto stage = [&](int st, int slot) {
         const uint8_t* sb = smem + slot * p.slot_bytes;
         const uint8_t* xs = xres + (size_t)st * NT * X_NT;
-        uint32_t sc[TPW][2][(GPW + 1) / 2];
+        constexpr int SN = GPW * spg<FMT>();  // FP16 values of the warp's groups per row
+        uint32_t sc[TPW][2][(SN + 1) / 2];
 #pragma unroll
         for (int tp = 0; tp < TPW; ++tp) {
-            const uint8_t* srow = sb + p.scales_off + (my_rt + NW * tp) * kTileScaleBytes + gsub * GPW * 2;
-            load_scales<GPW>(srow + g * 16, sc[tp][0]);
-            load_scales<GPW>(srow + (g + 8) * 16, sc[tp][1]);
+            const uint8_t* srow =
+                sb + p.scales_off + (my_rt + NW * tp) * tile_scale_bytes<FMT>() + gsub * GPW * 2 * spg<FMT>();
+            load_scales<SN>(srow + g * 16 * spg<FMT>(), sc[tp][0]);
+            load_scales<SN>(srow + (g + 8) * 16 * spg<FMT>(), sc[tp][1]);
         }
 #pragma unroll
         for (int gi = 0; gi < GPW; ++gi) {
@@ -419,7 +443,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
             for (int tp = 0; tp < TPW; ++tp) {
                 const uint8_t* codes_t = sb + (my_rt + NW * tp) * TSTRIDE;  // column box 0 of this row tile
                 int acc[NT][4];
-                if (FMT == BQ_Q1G128) {
+                if (bits_fmt<FMT>()) {
                     const int off = ((G ^ g) << 4) + 4 * t;
                     const uint32_t w0 = *reinterpret_cast<const uint32_t*>(codes_t + g * 128 + off);
                     const uint32_t w1 = *reinterpret_cast<const uint32_t*>(codes_t + (g + 8) * 128 + off);
@@ -474,17 +498,24 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                         }
                     }
                 }
-                const float s0 = scale_of(sc[tp][0], gi), s1 = scale_of(sc[tp][1], gi);
+                const float s0 = scale_of(sc[tp][0], spg<FMT>() * gi), s1 = scale_of(sc[tp][1], spg<FMT>() * gi);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     // D0 + 256 D1 is exact in int32 (|D0|, |D1| <= 2^21)
                     const float v0 = (float)(acc[nt][0] + (acc[nt][1] << 8));
                     const float v1 = (float)(acc[nt][2] + (acc[nt][3] << 8));
-                    // (with one factor tab.y = 1: the same rounding as fmaf(v, 2^e, -z))
-                    const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                    const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
-                    yacc[tp][nt][0] = fmaf(s0, u0, yacc[tp][nt][0]);
-                    yacc[tp][nt][1] = fmaf(s1, u1, yacc[tp][nt][1]);
+                    if constexpr (FMT == BQ_A1G128) {
+                        // s * sum(bit x) + zb * sum(x) (the sum on digit pair 0 only)
+                        const float z0 = scale_of(sc[tp][0], 2 * gi + 1), z1 = scale_of(sc[tp][1], 2 * gi + 1);
+                        yacc[tp][nt][0] = fmaf(s0, v0 * tab[nt].x * tab[nt].y, fmaf(z0, tab[nt].z, yacc[tp][nt][0]));
+                        yacc[tp][nt][1] = fmaf(s1, v1 * tab[nt].x * tab[nt].y, fmaf(z1, tab[nt].z, yacc[tp][nt][1]));
+                    } else {
+                        // (with one factor tab.y = 1: the same rounding as fmaf(v, 2^e, -z))
+                        const float u0 = fmaf(v0 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                        const float u1 = fmaf(v1 * tab[nt].x, tab[nt].y, -tab[nt].z);
+                        yacc[tp][nt][0] = fmaf(s0, u0, yacc[tp][nt][0]);
+                        yacc[tp][nt][1] = fmaf(s1, u1, yacc[tp][nt][1]);
+                    }
                 }
             }
         }
@@ -493,7 +524,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     // stage, stages are taken U at a time, so that U independent MMA chains run
     // between two barrier waits, if the ring holds 2 U slots.  (The longer
     // 2-bit and 5-trit stage bodies measured slower this way.)
-    constexpr int U = (FMT != BQ_Q1G128 || GPW * NT * TPW >= 4) ? 1 : 4 / (GPW * NT * TPW);
+    constexpr int U = (!bits_fmt<FMT>() || GPW * NT * TPW >= 4) ? 1 : 4 / (GPW * NT * TPW);
     const int ustep = (U > 1 && p.slots >= 2 * U) ? U : 1;  // (the producer keeps U slots ahead)
     bool alive = true;
     for (int st = 0; st < p.stages; st += ustep) {
@@ -638,8 +669,8 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
                              st * (KB * 128) + b * 128, chunk_row_tile(p, r, ct, 8 * h8) * 16, &full[slot]);
         } else if (lane >= 16 && lane < 16 + nbox) {
             const int h8 = lane - 16;
-            ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * kTileScaleBytes, &tm.scales128,
-                             st * kGroupsPerStage, chunk_row_tile(p, r, ct, 8 * h8) * 16, &full[slot]);
+            ptx::tma_load_2d(sb + p.scales_off + h8 * kMaxChunkTiles * tile_scale_bytes<FMT>(), &tm.scales128,
+                             st * kGroupsPerStage * spg<FMT>(), chunk_row_tile(p, r, ct, 8 * h8) * 16, &full[slot]);
         }
     } else if (lane < ct) {
         const int rt = chunk_row_tile(p, r, ct, lane);
@@ -647,8 +678,8 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
         for (int b = 0; b < KB; ++b)
             ptx::tma_load_2d(sb + b * (p.chunk_cap * 2048) + lane * 2048, &tm.codes16, st * (KB * 128) + b * 128,
                              rt * 16, &full[slot]);
-        ptx::tma_load_2d(sb + p.scales_off + lane * kTileScaleBytes, &tm.scales16, st * kGroupsPerStage, rt * 16,
-                         &full[slot]);
+        ptx::tma_load_2d(sb + p.scales_off + lane * tile_scale_bytes<FMT>(), &tm.scales16,
+                         st * kGroupsPerStage * spg<FMT>(), rt * 16, &full[slot]);
     }
 }
 
@@ -672,7 +703,7 @@ __device__ __forceinline__ bool produce(const Maps& tm, const Params& p, uint8_t
                     record_status(p.status, BQ_ERR_TIMEOUT);
                     ok = 0;
                 } else {
-                    ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + kTileScaleBytes)));
+                    ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)(ct * (TCB + tile_scale_bytes<FMT>())));
                 }
             }
             if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
@@ -995,13 +1026,15 @@ bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
     // than the most tiles a CTA owns (rounded down to a power of two), so
     // slots are sized for that; a slot is a multiple of 1 KB (the swizzled
     // copies land on 1 KB boundaries).
-    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + kTileScaleBytes;
-    pl.chunk_cap = (fmt == BQ_Q1G128 && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
+    const int64_t tsb = kTileScaleBytes * (fmt == BQ_A1G128 ? 2 : 1);
+    const bool bits = fmt == BQ_Q1G128 || fmt == BQ_A1G128;
+    const int64_t tile_bytes = (bits ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + tsb;
+    pl.chunk_cap = (bits && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
     const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
     while (pl.chunk_cap > 1 && pl.chunk_cap > most) pl.chunk_cap >>= 1;
     const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
     pl.slot_bytes = (int)slot;
-    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - tsb);
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
     const int64_t red = (int64_t)nw * 32 * pl.nt * 2 * 4;
@@ -1020,7 +1053,8 @@ bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
 
 Plan make_plan(int fmt, int64_t n, int64_t k, int batch) {
     Plan pl;
-    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 1 && batch <= 8 && k > 0 &&
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128 || fmt == BQ_A1G128) && batch >= 1 &&
+          batch <= 8 && k > 0 &&
           k % 1024 == 0 && n > 0 &&
           n <= (int64_t)INT32_MAX - 16 && k / 4 <= (int64_t)INT32_MAX / 4 && k <= (int64_t)1 << 20))
         return pl;
@@ -1054,7 +1088,7 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
                                                   NW == 8 ? kSmemHalf : kSmemFull);
         if (e != cudaSuccess) return e;
     }
-    const int64_t row_bytes = (FMT == BQ_Q1G128) ? k / 8 : (FMT == BQ_T2G128) ? k / 4 : (k / 128) * 26;
+    const int64_t row_bytes = bits_fmt<FMT>() ? k / 8 : (FMT == BQ_T2G128) ? k / 4 : (k / 128) * 26;
     const int64_t G = k / 128;
     Maps tm;
     for (int v = 0; v < 2; ++v) {
@@ -1072,9 +1106,10 @@ cudaError_t launch_typed(const uint8_t* codes, const uint16_t* scales, int64_t n
                 return cudaErrorInvalidValue;
         }
         {
-            cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)n};
-            cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
-            cuuint32_t box[2] = {(cuuint32_t)kGroupsPerStage, rows};
+            // the scale plane: [N][G] FP16, or [N][G][2] (scale, bias) pairs
+            cuuint64_t dims[2] = {(cuuint64_t)(G * spg<FMT>()), (cuuint64_t)n};
+            cuuint64_t strides[1] = {(cuuint64_t)(G * 2 * spg<FMT>())};
+            cuuint32_t box[2] = {(cuuint32_t)(kGroupsPerStage * spg<FMT>()), rows};
             cuuint32_t es[2] = {1, 1};
             if (enc(v == 0 ? &tm.scales16 : &tm.scales128, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
                     const_cast<uint16_t*>(scales), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1267,6 +1302,7 @@ cudaError_t launch_chain_fmt(const bq_chain_step* steps, int nsteps, int batch, 
 }  // namespace rows
 
 bool gemv_chain_eligible(int fmt, const bq_chain_step* steps, int nsteps, int batch) {
+    if (fmt != BQ_Q1G128 && fmt != BQ_T2G128 && fmt != BQ_T5P8G128) return false;
     if (nsteps < 1 || nsteps > rows::kMaxChainSteps || batch < 1 || batch > 8) return false;
     for (int i = 0; i < nsteps; ++i) {
         const bq_chain_step& st = steps[i];
@@ -1293,6 +1329,7 @@ cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scal
     const rows::Plan pl = rows::make_plan(fmt, n, k, batch);
     if (!pl.ok) return cudaErrorInvalidValue;
     if (fmt == BQ_Q1G128) return rows::launch_fmt<BQ_Q1G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (fmt == BQ_A1G128) return rows::launch_fmt<BQ_A1G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     if (fmt == BQ_T2G128) return rows::launch_fmt<BQ_T2G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     return rows::launch_fmt<BQ_T5P8G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }

@@ -53,7 +53,7 @@ using namespace bq;
 
 extern "C" bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                                      const uint16_t* x, int batch, void* y, int y_dtype, void* stream) {
-    if (fmt != BQ_Q1G128 && fmt != BQ_T2G128 && fmt != BQ_T5P8G128) return BQ_ERR_FORMAT;
+    if (fmt != BQ_Q1G128 && fmt != BQ_T2G128 && fmt != BQ_T5P8G128 && fmt != BQ_A1G128) return BQ_ERR_FORMAT;
     if (n < 0 || k < 0 || k % kGroup != 0 || batch < 1 || batch > BQ_MAX_BATCH) return BQ_ERR_SHAPE;
     if (y_dtype != BQ_BF16 && y_dtype != BQ_F32) return BQ_ERR_FORMAT;
     if (n == 0) return BQ_OK;

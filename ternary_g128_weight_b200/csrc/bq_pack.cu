@@ -98,6 +98,62 @@ __global__ void __launch_bounds__(128) pack_kernel(const float* __restrict__ w, 
     }
 }
 
+// Affine 1-bit variant (the layout MLX packs: a scale and a bias per group,
+// "Bonsai-27B-mlx-1bit ... Binary g128", section "MLX打包优化").  Reading of
+// the rule: z = FP16_RNE(min w), s = FP16_RNE(max w - min w) (exact in FP64),
+// bit = 1 iff w - z > s/2 in FP64 (ties give 0); params [N][G][2] = (s, z).
+__global__ void __launch_bounds__(128) pack_affine_kernel(const float* __restrict__ w, int64_t n, int64_t k,
+                                                          const uint16_t* __restrict__ params_in,
+                                                          uint8_t* __restrict__ codes, uint16_t* __restrict__ params,
+                                                          unsigned long long* first_error) {
+    const int64_t G = k / kGroup;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= n * G) return;
+    const int64_t r = gid / G, g = gid - r * G;
+    const float4* src = reinterpret_cast<const float4*>(w + r * k + g * kGroup);
+    float v[kGroup];
+#pragma unroll
+    for (int i = 0; i < kGroup / 4; ++i) {
+        float4 f = __ldg(src + i);
+        v[4 * i + 0] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+    }
+    bool finite = true;
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) finite &= isfinite(v[i]);
+    if (!finite) { record_pack_error(first_error, gid, BQ_ERR_NONFINITE); return; }
+    uint16_t sh, zh;
+    if (params_in) {
+        sh = params_in[2 * gid];
+        zh = params_in[2 * gid + 1];
+        if ((sh & 0x8000u) || (sh & 0x7C00u) == 0x7C00u || (zh & 0x7C00u) == 0x7C00u) {
+            record_pack_error(first_error, gid, BQ_ERR_SCALE_RANGE);
+            return;
+        }
+    } else {
+        float lo = v[0], hi = v[0];
+#pragma unroll
+        for (int i = 1; i < kGroup; ++i) {
+            lo = fminf(lo, v[i]);
+            hi = fmaxf(hi, v[i]);
+        }
+        zh = f64_to_f16_rn((double)lo);
+        sh = f64_to_f16_rn((double)hi - (double)lo);
+        if ((sh & 0x7C00u) == 0x7C00u || (zh & 0x7C00u) == 0x7C00u) {
+            record_pack_error(first_error, gid, BQ_ERR_SCALE_RANGE);
+            return;
+        }
+    }
+    params[2 * gid] = sh;
+    params[2 * gid + 1] = zh;
+    const double zv = f16_bits_to_f64(zh), half_s = f16_bits_to_f64(sh) / 2.0;
+    uint32_t word[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i)
+        if ((double)v[i] - zv > half_s) word[i >> 5] |= 1u << (i & 31);
+    uint4* dst = reinterpret_cast<uint4*>(codes + r * (k / 8) + g * 16);
+    *dst = make_uint4(word[0], word[1], word[2], word[3]);
+}
+
 }  // namespace
 
 cudaError_t launch_pack(int fmt, const float* w, int64_t n, int64_t k, const uint16_t* scales_in,
@@ -107,7 +163,9 @@ cudaError_t launch_pack(int fmt, const float* w, int64_t n, int64_t k, const uin
     if (groups == 0) return cudaSuccess;
     const int threads = 128;
     const int64_t blocks = (groups + threads - 1) / threads;
-    if (fmt == BQ_Q1G128)
+    if (fmt == BQ_A1G128)
+        pack_affine_kernel<<<(unsigned)blocks, threads, 0, s>>>(w, n, k, scales_in, codes, scales, first_error);
+    else if (fmt == BQ_Q1G128)
         pack_kernel<BQ_Q1G128><<<(unsigned)blocks, threads, 0, s>>>(w, n, k, scales_in, codes, scales, first_error);
     else if (fmt == BQ_T2G128)
         pack_kernel<BQ_T2G128><<<(unsigned)blocks, threads, 0, s>>>(w, n, k, scales_in, codes, scales, first_error);

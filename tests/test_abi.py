@@ -175,3 +175,12 @@ def test_chain_argument_errors_without_device(lib):
     assert call([ok], ws=0) == bq.BQ_ERR_WORKSPACE
     assert call([ok], wsb=16) == bq.BQ_ERR_WORKSPACE
     assert lib.bq_gemv_chain(bq.BQ_Q1G128, None, 1, 1, ctypes.c_void_p(A), 256, None) == bq.BQ_ERR_NULL
+
+
+def test_affine_sizes_match_oracle(lib):
+    for n, k in [(0, 128), (7, 1024), (151936, 4096)]:
+        assert bq.bq_codes_bytes("a1g128", n, k) == oracle.codes_bytes("a1g128", n, k) == n * k // 8
+        assert bq.bq_group_params_bytes("a1g128", n, k) == n * (k // 128) * 4
+        assert bq.bq_group_params_bytes("q1g128", n, k) == bq.bq_scales_bytes(n, k)
+    assert bq.bq_effective_bits("a1g128") == oracle.effective_bits("a1g128") == 1.25
+    assert bq.bq_gemm_workspace_bytes("a1g128", 64, 1024, 64) == -1
