@@ -18,6 +18,10 @@ pages it cites:
   (SwiGLU feed-forward: ``swiglu`` / ``mlp_swiglu``, with the BF16 rounding of
   the activation a reading, not a page fact).
 
+The 4-bit KV cache and its decode attention live in ``oracle.kv4`` (numpy
+FP64; "Bonsai-27B-mlx-1bit ... Binary g128", sections "峰值内存管理" and
+"KV压缩潜力"; "Ternary Bonsai", hybrid attention with a 4-bit KV cache).
+
 Parity status: the packing rules (mean-|w| scale, zero maps to +1, ternary
 threshold s/2, bit order, base-3 digit order) are readings of pages that do not
 state them; they are pinned to closed forms and invariants, not to any
@@ -31,6 +35,7 @@ import os
 import numpy as np
 
 from . import build as _build
+from . import kv4  # noqa: F401  (4-bit KV cache oracle)
 
 Q1G128, T2G128, T5P8G128, A1G128 = 1, 2, 3, 4
 FORMATS = {"q1g128": Q1G128, "t2g128": T2G128, "t5p8": T5P8G128, "a1g128": A1G128}
