@@ -112,8 +112,9 @@ def attention_decode(q_bf16, k_codes, k_params, v_codes, v_params, lens, hkv: in
     [B][Hkv][l_cap][d/128]; lens: [B].  heads: optional list of (b, h) pairs to
     compute (others are left NaN).
     Returns (out [B][Hq][d] FP64, mag [B][Hq][d] FP64) where
-    mag[b][h][j] = sum_t p_t (|V_tj| + |z_t| + 8 |s_t|) / sum_t p_t, the size
-    of the terms the output sums (s_t, z_t the group parameters of V_tj)."""
+    mag[b][h][j] = sum_t p_t (|V_tj| + 8 |s_t|) / sum_t p_t, the size of the
+    terms the output averages (s_t the scale of V_tj's group; 8 |s_t| bounds the
+    centred code part |s_t (c - 8)| of V_tj = s_t (c - 8) + (z_t + 8 s_t))."""
     q = _bf16_to_f64(q_bf16)
     B, hq = q.shape[0], q.shape[1]
     G = hq // hkv
@@ -136,8 +137,7 @@ def attention_decode(q_bf16, k_codes, k_params, v_codes, v_params, lens, hkv: in
             K = dequant(kc[b, kv, :n], kp[b, kv, :n], d)
             V = dequant(vc[b, kv, :n], vp[b, kv, :n], d)
             p = vp[b, kv, :n]
-            sz = (np.abs(_f16_bits_to_f64((p >> 16).astype(np.uint16))) +
-                  8.0 * np.abs(_f16_bits_to_f64((p & 0xFFFF).astype(np.uint16))))
+            sz = 8.0 * np.abs(_f16_bits_to_f64((p & 0xFFFF).astype(np.uint16)))
             cache[(b, kv)] = (K, V, np.abs(V) + np.repeat(sz, KV_GROUP, axis=1))
         K, V, A = cache[(b, kv)]
         a = scale * (K @ q[b, h])
