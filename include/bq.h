@@ -164,12 +164,19 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
  * when that is 0), 256-byte aligned; its contents on entry do not matter.
  * Asynchronous on `stream`.
  * Kernel choice (the same for bq_gemv_noalloc and for bq_gemm with T <= 4):
- * batch <= 8 and K % 1024 == 0 run the row-owning tensor-core GEMV (all three
- * formats, one launch, no workspace) when its activation operand and a ring
- * of at least two weight slots fit in shared memory; otherwise binary and
- * 2-bit ternary at batch <= 4 run the split-K tensor-core GEMV (workspace),
- * and the rest (the 5-trit format there, batch 9..16, K % 1024 != 0) the
- * tcgen05 GEMM with T = batch (workspace for the FP16 activations).  A shape
+ * K % 1024 == 0 with binary or 2-bit ternary codes at batch 5..16 runs the
+ * wide-batch GEMV (FP16 effective weights +-s / {-s,0,+s} built in registers,
+ * x pre-scaled per row to FP16, one launch, no workspace) where it measured
+ * fastest -- at batch 5..8 binary W of >= 64 Mi weights or K >= 8192, at batch
+ * 9..16 W of >= 64 Mi weights -- and its FP16 activations (2 K bytes per row,
+ * rows padded to 8 or 16) fit in shared memory; batch <= 8 and K % 1024 == 0
+ * otherwise run the row-owning
+ * tensor-core GEMV (all three formats, one launch, no workspace) when its
+ * activation operand and a ring of at least two weight slots fit in shared
+ * memory; otherwise binary and 2-bit ternary at batch <= 4 run the split-K
+ * tensor-core GEMV (workspace), and the rest (the 5-trit format at batch
+ * 9..16, K % 1024 != 0, operands too large) the tcgen05 GEMM with T = batch
+ * (workspace for the FP16 activations).  A shape
  * no kernel takes (K > 2^28, or N >= 2^31) returns BQ_ERR_SHAPE.
  * bq_gemv_workspace_bytes and bq_gemv_launches report the chosen path (-1 for
  * such a shape). */
@@ -273,6 +280,81 @@ int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t);
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                   const uint16_t* x, int64_t t, uint16_t* y,
                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------- 4-bit KV cache */
+/* A 4-bit KV cache for decode attention ("Bonsai-27B-mlx-1bit ... Binary
+ * g128", sections "峰值内存管理" and "KV压缩潜力": the KV cache is quantised to
+ * 4 bits for long contexts; "Ternary Bonsai", hybrid-attention section: 4-bit
+ * KV-cache quantisation; "1-bit Bonsai 8B" notes, Table 1: grouped-query
+ * attention, 32 query / 8 KV heads).  The pages fix the bit width only; the
+ * format is this library's reading:
+ *   every cached K or V vector of head dimension D (128 or 256) is cut into
+ *   groups of 128 values, each stored as 64 bytes of 4-bit codes (value 2i in
+ *   the low nibble of byte i) and one 32-bit word (FP16 scale s in bits 0..15,
+ *   FP16 bias z in bits 16..31), min-max affine with 16 levels:
+ *     s = FP16_RNE((max - min) / 15), z = FP16_RNE(min)  (the quotient in FP64),
+ *     c = clamp(rint((x - z) / s), 0, 15)  (in FP64; c = 0 when s == 0),
+ *     value = s c + z.                                  4.25 bits per value
+ * A group holding NaN / Inf is stored as zeros (s = z = 0, codes 0) and
+ * bq_check() reports BQ_ERR_NONFINITE; one whose s or z overflows FP16 the
+ * same, with BQ_ERR_SCALE_RANGE.
+ * Cache layout of one layer (all device memory, caller-owned, 16-byte aligned):
+ *   codes  uint8  [B][Hkv][L_cap][D/2]
+ *   params uint32 [B][Hkv][L_cap][D/128]
+ * with L_cap % 64 == 0 (the capacity in tokens); K and V have one of each. */
+#define BQ_KV4_CAP_MULTIPLE 64
+
+/* Bytes of the codes / params of `rows` cached vectors; -1 if d is not 128 or
+ * 256 or rows < 0. */
+int64_t bq_kv4_codes_bytes(int64_t rows, int d);
+int64_t bq_kv4_params_bytes(int64_t rows, int d);
+
+/* Quantise `rows` contiguous BF16 vectors x [rows][d] into codes [rows][d/2]
+ * and params [rows][d/128] (for example one sequence's and KV head's prompt
+ * keys, written straight into its cache rows).  All pointers device, 16-byte
+ * aligned.  Bit-exact to the definition above.  Asynchronous on `stream`;
+ * group errors surface through bq_check(). */
+bq_status bq_kv4_quantize(const uint16_t* x, int64_t rows, int d, uint8_t* codes, uint32_t* params,
+                          void* stream);
+
+/* Append one decode step: the new key and value of every sequence b and KV
+ * head h (k, v BF16 [B][Hkv][d]) are quantised into row pos[b] of their caches
+ * (codes / params laid out as above).  pos: device int32 [B]; a position
+ * outside [0, L_cap) writes nothing for that sequence and makes bq_check()
+ * report BQ_ERR_SHAPE.  Asynchronous on `stream`. */
+bq_status bq_kv4_append(const uint16_t* k, const uint16_t* v, int batch, int hkv, int d, const int32_t* pos,
+                        int64_t l_cap, uint8_t* k_codes, uint32_t* k_params, uint8_t* v_codes,
+                        uint32_t* v_params, void* stream);
+
+/* Workspace bytes bq_kv4_attention_decode needs (0 when the context is not
+ * split across CTAs); -1 for an invalid shape. */
+int64_t bq_kv4_attention_workspace_bytes(int batch, int hq, int hkv, int d, int64_t l_cap, int64_t max_len);
+
+/* Decode attention over the 4-bit cache, one query token per sequence:
+ *   for query head h of sequence b (KV head kv = h / G, G = hq / hkv <= 8) and
+ *   its first lens[b] cached tokens t:
+ *     a_t = scale <q[b][h], K_t>,  p_t = exp(a_t - max a),
+ *     out[b][h] = sum_t p_t V_t / sum_t p_t     (zeros when lens[b] == 0),
+ * with K_t, V_t the dequantised cache rows (s c + z).
+ * q BF16 [B][hq][d]; out [B][hq][d] BF16 or F32 (out_dtype); lens device int32
+ * [B] with 0 <= lens[b] <= max_len <= L_cap (a length outside that range is
+ * clamped into it and bq_check() reports BQ_ERR_SHAPE); d 128 or 256;
+ * B * hkv <= 65535.  The kernel reads whole stages of 64 (d = 128) or 32
+ * tokens, so cache rows up to the next multiple of that past lens[b] are read
+ * (never past L_cap) but do not enter the result.
+ * Precision: |out - exact| <= 2e-3 * sum_t p_t (|V_tj| + 8 |s_t|) / sum_t p_t
+ * (s_t the scale of V_tj's group) plus the output rounding (2^-8 |out| for
+ * BF16), while every token's scale * sum_j |q_j K_tj| stays below 256.
+ * workspace: >= bq_kv4_attention_workspace_bytes() device bytes, 256-byte
+ * aligned, ZERO-FILLED before its first use; every call leaves its counters
+ * zero (calls sharing a workspace must not overlap on the GPU; after a
+ * BQ_ERR_TIMEOUT zero it again).  The result does not depend on timing (the
+ * context splits are merged in a fixed order).  Asynchronous on `stream`. */
+bq_status bq_kv4_attention_decode(const uint16_t* q, const uint8_t* k_codes, const uint32_t* k_params,
+                                  const uint8_t* v_codes, const uint32_t* v_params, const int32_t* lens,
+                                  int batch, int hq, int hkv, int d, int64_t l_cap, int64_t max_len,
+                                  float scale, void* out, int out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ errors */
 /* Synchronises `stream`, then reports a pending CUDA error (BQ_ERR_CUDA) or a

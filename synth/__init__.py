@@ -38,6 +38,23 @@ CLASS27B_BLOCKS = 64
 PREFILL_SHAPES = [(17408, 5120), (5120, 17408)]
 PREFILL_TOKENS = [1, 8, 64, 512, 4096]
 
+# Decode attention of Qwen3-8B ("1-bit Bonsai 8B" notes, Table 1: 32 query /
+# 8 KV heads, hidden 4096, so head dimension 128; 65,536-token context).
+QWEN3_8B_ATTN = {"hq": 32, "hkv": 8, "d": 128, "max_ctx": 65536}
+
+
+def kv4_cache_bytes(g: np.random.Generator, b: int, hkv: int, l_cap: int, d: int, s_lo=0.02, s_hi=0.2):
+    """Random 4-bit cache contents: uniform code bytes, FP16 scales uniform in
+    [s_lo, s_hi], FP16 biases -7.5 s (1 + u), u uniform in [-0.1, 0.1], packed
+    as (s | z << 16).  Returns (codes uint8 [b][hkv][l_cap][d/2], params uint32
+    [b][hkv][l_cap][d/128])."""
+    codes = g.integers(0, 256, size=(b, hkv, l_cap, d // 2), dtype=np.uint8)
+    s = g.uniform(s_lo, s_hi, size=(b, hkv, l_cap, d // 128))
+    z = -7.5 * s * (1.0 + g.uniform(-0.1, 0.1, size=s.shape))
+    sb = s.astype(np.float16).view(np.uint16).astype(np.uint32)
+    zb = z.astype(np.float16).view(np.uint16).astype(np.uint32)
+    return codes, (sb | (zb << 16)).astype(np.uint32)
+
 
 def rng(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(seed))

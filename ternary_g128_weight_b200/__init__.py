@@ -30,6 +30,8 @@ EXPORTED = [
     "bq_gemv_workspace_bytes", "bq_gemv_launches", "bq_gemv", "bq_gemv_noalloc",
     "bq_gemm_workspace_bytes", "bq_gemm_launches", "bq_gemm",
     "bq_gemv_chain_workspace_bytes", "bq_gemv_chain", "bq_embed_rows",
+    "bq_kv4_codes_bytes", "bq_kv4_params_bytes", "bq_kv4_quantize", "bq_kv4_append",
+    "bq_kv4_attention_workspace_bytes", "bq_kv4_attention_decode",
     "bq_check", "bq_debug_wait_timeout", "bq_status_string", "bq_version",
 ]
 
@@ -76,6 +78,15 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.bq_gemm_launches.argtypes = [i32, i64, i64, i64]; L.bq_gemm_launches.restype = i32
     L.bq_gemm.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp, sz, vp]; L.bq_gemm.restype = i32
     L.bq_embed_rows.argtypes = [i32, vp, vp, i64, i64, vp, i64, vp, vp]; L.bq_embed_rows.restype = i32
+    L.bq_kv4_codes_bytes.argtypes = [i64, i32]; L.bq_kv4_codes_bytes.restype = i64
+    L.bq_kv4_params_bytes.argtypes = [i64, i32]; L.bq_kv4_params_bytes.restype = i64
+    L.bq_kv4_quantize.argtypes = [vp, i64, i32, vp, vp, vp]; L.bq_kv4_quantize.restype = i32
+    L.bq_kv4_append.argtypes = [vp, vp, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp]; L.bq_kv4_append.restype = i32
+    L.bq_kv4_attention_workspace_bytes.argtypes = [i32, i32, i32, i32, i64, i64]
+    L.bq_kv4_attention_workspace_bytes.restype = i64
+    L.bq_kv4_attention_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, i64, ctypes.c_float,
+                                          vp, i32, vp, sz, vp]
+    L.bq_kv4_attention_decode.restype = i32
     L.bq_gemv_chain_workspace_bytes.argtypes = []; L.bq_gemv_chain_workspace_bytes.restype = i64
     L.bq_gemv_chain.argtypes = [i32, ctypes.POINTER(ChainStep), i32, i32, vp, sz, vp]
     L.bq_gemv_chain.restype = i32
@@ -303,3 +314,67 @@ def bq_debug_wait_timeout(spin_limit: int, stream=None) -> int:
 
 def bq_status_string(status: int) -> str:
     return status_string(status)
+
+
+# ---------------------------------------------------------- 4-bit KV cache
+def bq_kv4_codes_bytes(rows: int, d: int) -> int:
+    return int(load().bq_kv4_codes_bytes(rows, d))
+
+
+def bq_kv4_params_bytes(rows: int, d: int) -> int:
+    return int(load().bq_kv4_params_bytes(rows, d))
+
+
+def bq_kv4_quantize(x, codes=None, params=None, stream=None):
+    """Quantise BF16 vectors x [..., d] (CUDA) to the 4-bit g128 cache format:
+    returns (codes uint8 [..., d/2], params int32 [..., d/128]) (the given
+    buffers if passed)."""
+    import torch
+    d = x.shape[-1]
+    lead = tuple(x.shape[:-1])
+    rows = x.numel() // d if d else 0
+    if codes is None:
+        codes = torch.empty(lead + (d // 2,), dtype=torch.uint8, device=x.device)
+    if params is None:
+        params = torch.empty(lead + (d // 128,), dtype=torch.int32, device=x.device)
+    st = load().bq_kv4_quantize(_ptr(x), rows, d, _ptr(codes), _ptr(params), _stream(stream))
+    _check(st, "bq_kv4_quantize")
+    return codes, params
+
+
+def bq_kv4_append(k, v, pos, k_codes, k_params, v_codes, v_params, stream=None):
+    """Write the new K and V (BF16 [B][Hkv][d]) into row pos[b] (int32 CUDA
+    tensor [B]) of the caches (codes uint8 [B][Hkv][L_cap][d/2], params int32
+    [B][Hkv][L_cap][d/128])."""
+    B, hkv, d = k.shape
+    l_cap = k_codes.shape[2]
+    st = load().bq_kv4_append(_ptr(k), _ptr(v), B, hkv, d, _ptr(pos), l_cap, _ptr(k_codes), _ptr(k_params),
+                              _ptr(v_codes), _ptr(v_params), _stream(stream))
+    _check(st, "bq_kv4_append")
+
+
+def bq_kv4_attention_workspace_bytes(batch: int, hq: int, hkv: int, d: int, l_cap: int, max_len: int) -> int:
+    return int(load().bq_kv4_attention_workspace_bytes(batch, hq, hkv, d, l_cap, max_len))
+
+
+def bq_kv4_attention_decode(q, k_codes, k_params, v_codes, v_params, lens, max_len: int, scale: float,
+                            out=None, out_dtype=None, workspace=None, stream=None):
+    """Decode attention of q (BF16 [B][Hq][d]) over the 4-bit caches (see bq.h);
+    lens int32 CUDA [B].  Returns (out, workspace); pass the workspace back to
+    reuse it (a zero-filled one is made when None)."""
+    import torch
+    B, hq, d = q.shape
+    hkv, l_cap = k_codes.shape[1], k_codes.shape[2]
+    if out is None:
+        dt = torch.float32 if out_dtype == BQ_F32 else torch.bfloat16
+        out = torch.empty((B, hq, d), dtype=dt, device=q.device)
+    odt = BQ_F32 if out.dtype == torch.float32 else BQ_BF16
+    need = bq_kv4_attention_workspace_bytes(B, hq, hkv, d, l_cap, max_len)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=q.device)
+    wsb = workspace.numel() * workspace.element_size()
+    st = load().bq_kv4_attention_decode(_ptr(q), _ptr(k_codes), _ptr(k_params), _ptr(v_codes), _ptr(v_params),
+                                        _ptr(lens), B, hq, hkv, d, l_cap, max_len, float(scale), _ptr(out), odt,
+                                        _ptr(workspace), wsb, _stream(stream))
+    _check(st, "bq_kv4_attention_decode")
+    return out, workspace

@@ -81,7 +81,21 @@ int* device_status_ptr() {
 }  // namespace bq
 
 namespace bq {
+// Where the wide-batch kernel beats the alternatives, as measured on B200
+// (one launch per matrix, weights larger than L2): at batch 5..8 against the
+// row-owning kernel for binary matrices of >= 64 Mi weights and for K >= 8192
+// (4096 x 12288: 28 vs 38 us binary, 33 vs 41 us 2-bit; 4096 x 4096: 12.0 vs
+// 9.1 us, so not there); at batch 9..16 against the tcgen05 GEMM for >= 64 Mi
+// weights (24576 x 4096 binary: 35 vs 63 us; 4096 x 4096: 23 vs 19 us).
+static bool prefer_wide(int fmt, int64_t n, int64_t k, int batch) {
+    const int64_t weights = n * k;
+    constexpr int64_t kLarge = 64LL << 20;
+    if (batch <= 8) return (fmt == BQ_Q1G128 && weights >= kLarge) || k >= 8192;
+    return weights >= kLarge;
+}
+
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
+    if (batch >= 5 && prefer_wide(fmt, n, k, batch) && gemv_wide_eligible(fmt, n, k, batch)) return GemvPath::Wide;
     if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
     if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
     if (gemm_tc_eligible(fmt, n, k, batch)) return GemvPath::Gemm;
@@ -100,6 +114,7 @@ cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, i
                         const uint16_t* x, int batch, void* y, int y_dtype, void* workspace, cudaStream_t s) {
     switch (gemv_path(fmt, n, k, batch)) {
         case GemvPath::Rows: return launch_gemv_rows(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
+        case GemvPath::Wide: return launch_gemv_wide(fmt, codes, scales, n, k, x, batch, y, y_dtype, s);
         case GemvPath::SplitK: return launch_gemv_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
         case GemvPath::Gemm: return launch_gemm_tc(fmt, codes, scales, n, k, x, batch, y, y_dtype, workspace, s);
         default: return cudaErrorInvalidValue;
@@ -157,6 +172,7 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch) {
     if (k == 0) return 0;  // the output is cleared with a memset, no kernel
     switch (gemv_path(fmt, n, k, batch)) {
         case GemvPath::Rows: return 1;
+        case GemvPath::Wide: return 1;
         case GemvPath::SplitK: return 2;  // activation prep + split-K kernel
         case GemvPath::Gemm: return gemm_tc_launches(n, k, batch);
         default: return -1;  // no kernel takes the shape (bq_gemv returns BQ_ERR_SHAPE)
@@ -192,14 +208,15 @@ bq_status bq_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-// Prefill dispatch: up to 4 tokens run the tensor-core GEMV paths (the weight
-// stream dominates and the result is bit-identical with bq_gemv); more tokens
-// run the tcgen05 GEMM.  A shape neither takes (K > 2^28, N >= 2^31) is
+// Prefill dispatch: up to 4 tokens run the tensor-core GEMV paths, and 5..16
+// tokens the wide-batch GEMV where it takes the shape (the weight stream
+// dominates; the result is bit-identical with bq_gemv); more tokens run the
+// tcgen05 GEMM.  A shape neither takes (K > 2^28, N >= 2^31) is
 // rejected with BQ_ERR_SHAPE.
 static bool gemm_uses_gemv(int fmt, int64_t n, int64_t k, int64_t t) {
-    if (t > 4) return false;
+    if (t > BQ_MAX_BATCH) return false;
     const GemvPath p = gemv_path(fmt, n, k, (int)t);
-    return p == GemvPath::Rows || p == GemvPath::SplitK;
+    return (t <= 4 && (p == GemvPath::Rows || p == GemvPath::SplitK)) || p == GemvPath::Wide;
 }
 
 int64_t bq_gemm_workspace_bytes(int fmt, int64_t n, int64_t k, int64_t t) {

@@ -1006,6 +1006,316 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
     }
 }
 
+// ------------------------------------------------------- wide-batch decode
+// Batch 5..16, binary and 2-bit ternary.  The weights become exact FP16
+// effective weights s * q inside the A registers of the warp MMA m16n8k16:
+//   binary: ((w << (15 - m)) & 0x80008000) ^ (s | s << 16) ^ 0x80008000 is the
+//           pair (weight m, weight m + 16) of code word w as (+-s, +-s), the
+//           sign the negated bit (bit 1 -> +s);
+//   2-bit : the codes c of weights i and i + 8 of a word placed in the low bits
+//           of the FP16 1024 give 1024 + c; minus 1025 is q = c - 1, times s is
+//           s * q, all exact;
+// and x enters as FP16 x * 2^e_b with one power of two per batch row b (its
+// largest |x| in [2^14, 2^15): exact for every BF16 value within 2^-31 of the
+// row's largest magnitude), so the MMA accumulates s * q * x over all of K in
+// FP32 and y = acc * 2^-e_b -- no per-group recombination and no digit split:
+// one decoded 16 x 16 weight fragment feeds one MMA per 8 batch rows.
+constexpr int kWideAux = 256;  // row maxima, exponents and 2^-e per batch row
+
+// Activation area per stage: [group G][j 0..7][batch row b][thread t][2 words],
+// word p of (G, b, t) the FP16 pair of the two activations register p of a
+// weight row pairs (see wide_lo / wide_hi); MMA j reads words 2j, 2j + 1.
+template <int NTW>
+__host__ __device__ constexpr int wide_stage_bytes() { return kGroupsPerStage * 8 * (NTW * 8) * 4 * 8; }
+
+// The weights (relative to 32 t in the group) of register p (0..15) of a
+// thread's weight row: binary (p, p + 16); 2-bit p < 8: (p, p + 8), else
+// (p + 8, p + 16).
+template <int FMT>
+__device__ __forceinline__ constexpr int wide_lo(int p) { return FMT == BQ_T2G128 ? (p < 8 ? p : p + 8) : p; }
+template <int FMT>
+__device__ __forceinline__ constexpr int wide_hi(int p) { return FMT == BQ_T2G128 ? (p < 8 ? p + 8 : p + 16) : p + 16; }
+
+// x -> the FP16 activation area of all of K, per-row power-of-two pre-scale.
+template <int FMT, int NTW, int NW>
+__device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
+    constexpr int BP = NTW * 8;
+    const int tid = threadIdx.x;
+    uint32_t* rmax = reinterpret_cast<uint32_t*>(smem + p.lut_off);
+    int* es = reinterpret_cast<int*>(smem + p.lut_off + 64);
+    float* inv = reinterpret_cast<float*>(smem + p.lut_off + 128);
+    if (tid < BP) rmax[tid] = 0u;
+    bar_compute<NW>();
+    // largest |x| of every batch row (FP32 bits of the magnitude: monotonic)
+    const int64_t c8 = p.k / 8;
+    for (int b = 0; b < p.batch; ++b) {
+        uint32_t m = 0u;
+        for (int64_t c = tid; c < c8; c += NW * 32) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + b * p.k) + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m = max(m, max((w[q] << 16) & 0x7FFFFFFFu, w[q] & 0x7FFF0000u));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((tid & 31) == 0) atomicMax(&rmax[b], m);
+    }
+    bar_compute<NW>();
+    if (tid < BP) {
+        const float m = __uint_as_float(rmax[tid]);
+        const int e = m > 0.f ? 14 - ilog2f(m) : 0;  // in [-113, 147]
+        es[tid] = e;
+        inv[tid] = ldexpf(1.0f, -e);  // exact (a subnormal below 2^-126)
+    }
+    bar_compute<NW>();
+    // (stage, group, batch row, thread t): 32 activations -> 16 FP16 pairs
+    uint8_t* xres = smem + p.x_off;
+    const int tasks = p.stages * kGroupsPerStage * BP * 4;
+    for (int i = tid; i < tasks; i += NW * 32) {
+        const int t = i & 3, b = (i >> 2) % BP, rest = i / (4 * BP), G = rest & 7, st = rest >> 3;
+        uint32_t words[16];
+        if (b < p.batch) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.x + b * p.k + st * 1024 + G * 128 + 32 * t);
+            uint32_t raw[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 v = __ldg(src + q);
+                raw[4 * q] = v.x; raw[4 * q + 1] = v.y; raw[4 * q + 2] = v.z; raw[4 * q + 3] = v.w;
+            }
+            const int e = es[b];
+            uint16_t h[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const float v = __uint_as_float((r & 1) ? (raw[r >> 1] & 0xFFFF0000u) : (raw[r >> 1] << 16));
+                h[r] = __half_as_ushort(__float2half_rn(ldexpf(v, e)));
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                words[q] = (uint32_t)h[wide_lo<FMT>(q)] | ((uint32_t)h[wide_hi<FMT>(q)] << 16);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) words[q] = 0u;
+        }
+        uint8_t* base = xres + (size_t)st * wide_stage_bytes<NTW>();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint2*>(base + ((((G * 8 + j) * BP + b) * 4 + t) * 8)) =
+                make_uint2(words[2 * j], words[2 * j + 1]);
+    }
+}
+
+__device__ __forceinline__ __half2 u2h2(uint32_t u) {
+    __half2 h;
+    *reinterpret_cast<uint32_t*>(&h) = u;
+    return h;
+}
+__device__ __forceinline__ uint32_t h22u(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
+
+// The four A registers of MMA j for rows g (w: its code words) and g + 8
+// (wb), scales S (binary: (s | s << 16) ^ 0x80008000; 2-bit: s | s << 16).
+template <int FMT>
+__device__ __forceinline__ void wide_a(uint2 w, uint2 wb, uint32_t S, uint32_t Sb, int j, uint32_t (&a)[4]) {
+    if (FMT == BQ_Q1G128) {
+        const int m0 = 2 * j, m1 = 2 * j + 1;
+        a[0] = ((w.x << (15 - m0)) & 0x80008000u) ^ S;
+        a[1] = ((wb.x << (15 - m0)) & 0x80008000u) ^ Sb;
+        a[2] = ((w.x << (15 - m1)) & 0x80008000u) ^ S;
+        a[3] = ((wb.x << (15 - m1)) & 0x80008000u) ^ Sb;
+    } else {
+        const __half2 k1025 = u2h2(0x64016401u);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int pr = 2 * j + h;  // register pair p
+            const uint32_t word = pr < 8 ? w.x : w.y, wordb = pr < 8 ? wb.x : wb.y;
+            const int sh = 2 * (pr & 7);
+            const __half2 qa = __hsub2(u2h2(((word >> sh) & 0x00030003u) | 0x64006400u), k1025);
+            const __half2 qb = __hsub2(u2h2(((wordb >> sh) & 0x00030003u) | 0x64006400u), k1025);
+            a[2 * h] = h22u(__hmul2(qa, u2h2(S)));
+            a[2 * h + 1] = h22u(__hmul2(qb, u2h2(Sb)));
+        }
+    }
+}
+
+// One chunk of CT row tiles, all stages, accumulating in FP32 across K; work
+// split as run_chunk.
+template <int FMT, int NTW, int NW, int CT>
+__device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, Ring& rp,
+                               int warp, int lane) {
+    constexpr int TPW = CT >= NW ? CT / NW : 1;
+    constexpr int WPR = CT >= NW ? 1 : ((NW / CT) < kGroupsPerStage ? (NW / CT) : kGroupsPerStage);
+    constexpr int GPW = kGroupsPerStage / WPR;
+    constexpr int BP = NTW * 8;
+    constexpr int TSTRIDE = 2048;  // code bytes between row tiles of a column box
+    const int my_rt = CT >= NW ? warp : warp / WPR;
+    const int gsub = CT >= NW ? 0 : warp % WPR;
+    const bool active = my_rt < CT;
+    const int g = lane >> 2, t = lane & 3;
+    float acc[TPW][NTW][4];
+#pragma unroll
+    for (int tp = 0; tp < TPW; ++tp)
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[tp][nt][c] = 0.0f;
+    bool alive = true;
+    for (int st = 0; st < p.stages; ++st) {
+        const int slot = rp.slot;
+        if (!ptx::mbar_wait_bounded(&full[slot], rp.round & 1u, kWaitPolls)) {
+            record_status(p.status, BQ_ERR_TIMEOUT);
+            alive = false;
+            break;
+        }
+        rp.next();
+        if (active) {
+            const uint8_t* sb = smem + slot * p.slot_bytes;
+            const uint8_t* xs = smem + p.x_off + (size_t)st * wide_stage_bytes<NTW>();
+            uint32_t sc[TPW][2][(GPW + 1) / 2];
+#pragma unroll
+            for (int tp = 0; tp < TPW; ++tp) {
+                const uint8_t* srow = sb + p.scales_off + (my_rt + NW * tp) * kTileScaleBytes + gsub * GPW * 2;
+                load_scales<GPW>(srow + g * 16, sc[tp][0]);
+                load_scales<GPW>(srow + (g + 8) * 16, sc[tp][1]);
+            }
+#pragma unroll
+            for (int gi = 0; gi < GPW; ++gi) {
+                const int G = gsub * GPW + gi;
+#pragma unroll
+                for (int tp = 0; tp < TPW; ++tp) {
+                    const uint8_t* codes_t = sb + (my_rt + NW * tp) * TSTRIDE;
+                    uint2 w, wb;
+                    if (FMT == BQ_Q1G128) {
+                        const int off = ((G ^ g) << 4) + 4 * t;
+                        w = make_uint2(*reinterpret_cast<const uint32_t*>(codes_t + g * 128 + off), 0u);
+                        wb = make_uint2(*reinterpret_cast<const uint32_t*>(codes_t + (g + 8) * 128 + off), 0u);
+                    } else {
+                        const uint8_t* box = codes_t + (G >> 2) * (p.chunk_cap * 2048);
+                        const int chunk = 2 * (G & 3) + (t >> 1);
+                        const int off = ((chunk ^ g) << 4) + 8 * (t & 1);
+                        w = *reinterpret_cast<const uint2*>(box + g * 128 + off);
+                        wb = *reinterpret_cast<const uint2*>(box + (g + 8) * 128 + off);
+                    }
+                    const uint32_t s0 = (sc[tp][0][gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+                    const uint32_t s1 = (sc[tp][1][gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+                    const uint32_t flip = FMT == BQ_Q1G128 ? 0x80008000u : 0u;
+                    const uint32_t S = (s0 | (s0 << 16)) ^ flip, Sb = (s1 | (s1 << 16)) ^ flip;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        uint32_t a[4];
+                        wide_a<FMT>(w, wb, S, Sb, j, a);
+#pragma unroll
+                        for (int nt = 0; nt < NTW; ++nt) {
+                            const uint2 bv = *reinterpret_cast<const uint2*>(
+                                xs + ((((G * 8 + j) * BP + nt * 8 + g) * 4 + t) * 8));
+                            ptx::mma_f16_16816(acc[tp][nt], a[0], a[1], a[2], a[3], bv.x, bv.y);
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[slot]);
+    }
+    if (WPR > 1) {
+        float* red = reinterpret_cast<float*>(smem + p.red_off);
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) red[((warp * 32 + lane) * NTW + nt) * 4 + c] = acc[0][nt][c];
+        bar_compute<NW>();
+        if (active && gsub == 0) {
+#pragma unroll
+            for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int q = 0; q < WPR; ++q) sum += red[(((warp + q) * 32 + lane) * NTW + nt) * 4 + c];
+                    acc[0][nt][c] = sum;
+                }
+        }
+        bar_compute<NW>();
+    }
+    if (active && gsub == 0) {
+        const float* inv = reinterpret_cast<const float*>(smem + p.lut_off + 128);
+#pragma unroll
+        for (int tp = 0; tp < TPW; ++tp)
+#pragma unroll
+            for (int nt = 0; nt < NTW; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int bb = nt * 8 + 2 * t + (c & 1);
+                    const int64_t row = (int64_t)(rt + my_rt + NW * tp) * 16 + g + 8 * (c >> 1);
+                    if (bb < p.batch && row < p.n) {
+                        const float v = acc[tp][nt][c] * inv[bb];
+                        if (p.y_dtype == BQ_F32)
+                            static_cast<float*>(p.y)[bb * p.n + row] = v;
+                        else
+                            static_cast<uint16_t*>(p.y)[bb * p.n + row] = float_to_bf16_bits(v);
+                    }
+                }
+    }
+    return alive;
+}
+
+template <int FMT, int NTW>
+__global__ void __launch_bounds__(threads_of<16>(), 1)
+    gemv_wide_kernel(const __grid_constant__ Maps tm, const Params p) {
+    constexpr int NW = 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = ptx::align_smem<1024>(smem_raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+    uint64_t* empty = full + kMaxSlots;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = gridDim.x, c = blockIdx.x;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.slots; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], NW);
+        }
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
+    const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
+    ptx::pdl_launch_dependents();
+    if (warp == NW) {
+        if (lane == 0) {
+            ptx::prefetch_tensormap(&tm.codes16);
+            ptx::prefetch_tensormap(&tm.scales16);
+            ptx::prefetch_tensormap(&tm.codes128);
+            ptx::prefetch_tensormap(&tm.scales128);
+        }
+        int it = 0;
+        Ring rp;
+        rp.depth = p.slots;
+        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
+        if (lane == 0)
+            for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
+                if (!ptx::mbar_wait_bounded(&full[j % p.slots], (uint32_t)((j / p.slots) & 1), kWaitPolls))
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+        return;
+    }
+    ptx::pdl_wait();  // x is produced, y may still be read, by the previous kernel
+    prep_wide<FMT, NTW, NW>(p, smem);
+    bar_compute<NW>();
+    Ring rp;
+    rp.depth = p.slots;
+    for (int r = rt0; r < rt1;) {
+        const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
+        bool ok;
+        if (ct == 8)
+            ok = run_chunk_wide<FMT, NTW, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 4)
+            ok = run_chunk_wide<FMT, NTW, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
+        else if (ct == 2)
+            ok = run_chunk_wide<FMT, NTW, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
+        else
+            ok = run_chunk_wide<FMT, NTW, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+        if (!ok) break;
+        r += ct;
+    }
+}
+
 // ----------------------------------------------------------------- host
 struct Plan {
     int nt = 0, lanes = 0, nw = 0, stages = 0, row_tiles = 0, slots = 0, grid = 0, chunk_cap = 8, slot_bytes = 0,
@@ -1170,6 +1480,115 @@ cudaError_t launch_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, 
 }  // namespace rows
 
 bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch) { return rows::make_plan(fmt, n, k, batch).ok; }
+
+namespace rows {
+
+cudaError_t encode_maps(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, Maps& tm);
+
+// Wide-batch plan: one CTA of 16 compute warps per SM, the FP16 activation
+// area of all of K resident, a ring of at least two 8-tile slots.
+bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128) && batch >= 5 && batch <= 16 && k > 0 && k % 1024 == 0 &&
+          n > 0 && n <= (int64_t)INT32_MAX - 16 && k <= (int64_t)1 << 20))
+        return false;
+    pl.nt = batch <= 8 ? 1 : 2;  // n-tiles of eight batch rows
+    pl.lanes = 0;
+    pl.nw = 16;
+    pl.stages = (int)(k / 1024);
+    pl.row_tiles = (int)((n + 15) / 16);
+    const int sms = sm_count();
+    pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
+    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : 4096) + kTileScaleBytes;
+    pl.chunk_cap = kMaxChunkTiles;
+    const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
+    while (pl.chunk_cap > 1 && pl.chunk_cap > most) pl.chunk_cap >>= 1;
+    const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+    pl.slot_bytes = (int)slot;
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
+    const int64_t x_area = (int64_t)pl.stages * (pl.nt == 1 ? wide_stage_bytes<1>() : wide_stage_bytes<2>());
+    const int64_t red = (int64_t)16 * 32 * pl.nt * 4 * 4;
+    const int64_t fixed = 1024 + x_area + red + kWideAux + 2 * kMaxSlots * 8;
+    int64_t slots = (kSmemFull - fixed) / slot;
+    if (slots > kMaxSlots) slots = kMaxSlots;
+    if (slots < 2) return false;
+    pl.slots = (int)slots;
+    pl.x_off = (uint32_t)(slots * slot);
+    pl.red_off = (uint32_t)(pl.x_off + x_area);
+    pl.lut_off = (uint32_t)(pl.red_off + red);  // the per-row pre-scale area
+    pl.bar_off = (uint32_t)(pl.lut_off + kWideAux);
+    pl.smem = (uint32_t)(1024 + pl.bar_off + 2 * kMaxSlots * 8);
+    pl.ok = true;
+    return true;
+}
+
+template <int FMT, int NTW>
+cudaError_t launch_wide_typed(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
+                              int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
+    {
+        const cudaError_t e =
+            ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_wide_kernel<FMT, NTW>), kSmemFull);
+        if (e != cudaSuccess) return e;
+    }
+    Maps tm;
+    {
+        const cudaError_t e = encode_maps(FMT, codes, scales, n, k, tm);
+        if (e != cudaSuccess) return e;
+    }
+    Params prm = {};
+    prm.x = x;
+    prm.y = y;
+    prm.n = n;
+    prm.k = k;
+    prm.batch = batch;
+    prm.y_dtype = y_dtype;
+    prm.stages = pl.stages;
+    prm.row_tiles = pl.row_tiles;
+    prm.slots = pl.slots;
+    prm.slot_bytes = pl.slot_bytes;
+    prm.scales_off = pl.scales_off;
+    prm.chunk_cap = pl.chunk_cap;
+    prm.x_off = pl.x_off;
+    prm.red_off = pl.red_off;
+    prm.lut_off = pl.lut_off;
+    prm.bar_off = pl.bar_off;
+    prm.pair_tiles = 0;
+    prm.stg_off = 0;
+    prm.status = device_status_ptr();
+    if (!prm.status) return cudaErrorUnknown;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid);
+    cfg.blockDim = dim3(threads_of<16>());
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = s;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_wide_kernel<FMT, NTW>, tm, prm);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace rows
+
+bool gemv_wide_eligible(int fmt, int64_t n, int64_t k, int batch) {
+    rows::Plan pl;
+    return rows::wide_plan(pl, fmt, n, k, batch);
+}
+
+cudaError_t launch_gemv_wide(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                             const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s) {
+    rows::Plan pl;
+    if (!rows::wide_plan(pl, fmt, n, k, batch)) return cudaErrorInvalidValue;
+    if (fmt == BQ_Q1G128)
+        return pl.nt == 1 ? rows::launch_wide_typed<BQ_Q1G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
+                          : rows::launch_wide_typed<BQ_Q1G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return pl.nt == 1 ? rows::launch_wide_typed<BQ_T2G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
+                      : rows::launch_wide_typed<BQ_T2G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+}
+
+
 
 namespace rows {
 

@@ -76,6 +76,12 @@ bool gemv_rows_eligible(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                              const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
 
+// Wide-batch decode GEMV (binary and 2-bit ternary, batch 5..16, K % 1024 ==
+// 0, FP16 activations of all of K resident in shared memory): no workspace.
+bool gemv_wide_eligible(int fmt, int64_t n, int64_t k, int batch);
+cudaError_t launch_gemv_wide(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
+                             const uint16_t* x, int batch, void* y, int y_dtype, cudaStream_t s);
+
 // Embedding lookup (bq_embed_rows).
 cudaError_t launch_embed_rows(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                               const int32_t* ids, int64_t count, uint16_t* out, cudaStream_t s);
@@ -86,12 +92,14 @@ bool gemv_chain_eligible(int fmt, const bq_chain_step* steps, int nsteps, int ba
 cudaError_t launch_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, int batch, unsigned int* bar,
                               cudaStream_t s);
 
-// GEMV path choice shared by bq_gemv, bq_gemm (T <= 4) and bq_gemv_noalloc:
-// the row-owning kernel where eligible, else the split-K tensor-core kernel,
+// GEMV path choice shared by bq_gemv, bq_gemm (T <= 16) and bq_gemv_noalloc:
+// batch 5..16 the wide-batch kernel where eligible and measured faster
+// (prefer_wide); the row-owning kernel
+// where eligible, else the split-K tensor-core kernel,
 // else the tcgen05 GEMM with T = batch; None when no kernel takes the shape
 // (K > 2^28 or N >= 2^31).  gemv_workspace_bytes reports the workspace of the
 // choice.
-enum class GemvPath { Rows, SplitK, Gemm, None };
+enum class GemvPath { Rows, Wide, SplitK, Gemm, None };
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch);
 int64_t gemv_workspace_bytes(int fmt, int64_t n, int64_t k, int batch);
 cudaError_t launch_gemv(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,

@@ -64,10 +64,11 @@ extern "C" bq_status bq_gemv_noalloc(int fmt, const uint8_t* codes, const uint16
         const size_t bytes = (size_t)batch * n * (y_dtype == BQ_F32 ? 4 : 2);
         return cudaMemsetAsync(y, 0, bytes, s) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
     }
-    // Same path choice as bq_gemv.  The row-owning kernel needs no scratch;
-    // the split-K kernel keeps its prepared activations, row-block counters
-    // and partial sums there, and the tcgen05 GEMM (T = batch) its FP16
-    // activations, per-token scales and, when K is split, partial tiles.
+    // Same path choice as bq_gemv.  The row-owning and wide-batch kernels
+    // need no scratch; the split-K kernel keeps its prepared activations,
+    // row-block counters and partial sums there, and the tcgen05 GEMM
+    // (T = batch) its FP16 activations, per-token scales and, when K is split,
+    // partial tiles.
     if (gemv_path(fmt, n, k, batch) == GemvPath::None) return BQ_ERR_SHAPE;
     const int64_t need = gemv_workspace_bytes(fmt, n, k, batch);
     uint8_t* scratch = nullptr;

@@ -114,6 +114,19 @@ __device__ __forceinline__ void mma_u8s8_init(int (&d)[4], uint32_t a0, uint32_t
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c));
 }
 
+// D(16x8, f32) += A(16x16, f16) * B(16x8, f16).  Fragments: thread (g, t) =
+// (lane / 4, lane % 4) holds A[g][2t..2t+1], A[g+8][2t..2t+1], A[g][2t+8..2t+9],
+// A[g+8][2t+8..2t+9]; B[2t..2t+1][g], B[2t+8..2t+9][g]; D[g][2t], D[g][2t+1],
+// D[g+8][2t], D[g+8][2t+1].
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Programmatic dependent launch: let the next grid in the stream start its
 // prologue now / wait until the previous grid has completed and its writes are
 // visible.

@@ -104,7 +104,11 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_gemv_launches(2, 4096, 4096, 4) == 1
     assert lib.bq_gemv_launches(3, 4096, 4096, 1) == 1       # 5-trit format, row-owning kernel too
     assert lib.bq_gemv_launches(3, 4096, 17408, 4) in (2, 3)  # operand too large: tcgen05 GEMM
-    assert lib.bq_gemv_launches(1, 4096, 4096, 16) in (2, 3)
+    assert lib.bq_gemv_launches(1, 24576, 4096, 16) == 1      # wide-batch kernel (large W)
+    assert lib.bq_gemv_launches(1, 4096, 4096, 16) in (2, 3)   # small W at batch 16: tcgen05 GEMM
+    assert lib.bq_gemv_launches(3, 4096, 4096, 16) in (2, 3)   # 5-trit format at batch 16: tcgen05 GEMM
+    assert lib.bq_gemv_launches(1, 4096, 12288, 16) in (2, 3)  # FP16 x exceeds shared memory: GEMM
+    assert lib.bq_gemm_launches(2, 24576, 4096, 12) == 1       # T 5..16, large W: the wide-batch GEMV
     assert lib.bq_gemm_launches(1, 17408, 5120, 4096) == 2     # prep + GEMM, no K split
     assert lib.bq_gemm_launches(1, 4096, 4096, 1) == 1         # T <= 4: the GEMV
     assert lib.bq_gemm_launches(1, 4096, 100, 8) == -1
@@ -114,16 +118,24 @@ def test_argument_errors_need_no_device(lib):
 
 def test_gemv_path_choice_host_only(lib):
     """Which kernel a bq_gemv call takes is decided on the host (shared memory
-    plan at 148 SMs when no device is visible): the row-owning kernel needs no
-    workspace and one launch; split-K and the GEMM need workspace."""
+    plan at 148 SMs when no device is visible): the row-owning and wide-batch
+    kernels need no workspace and one launch; split-K and the GEMM need
+    workspace."""
     ws, nl = bq.bq_gemv_workspace_bytes, bq.bq_gemv_launches
     for fmt in ("q1g128", "t2g128", "t5p8"):
         for n, k, b in ((4096, 4096, 1), (151936, 4096, 1), (4096, 12288, 1), (777, 1024, 2)):
             assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)   # row-owning
         assert ws(fmt, 4096, 1152, 1) >= 1152 * 2                                 # K % 1024 != 0: GEMM
-        assert ws(fmt, 4096, 4096, 9) >= 9 * 4096 * 2                             # batch > 8: GEMM
+        assert ws(fmt, 4096, 4096, 9) >= 9 * 4096 * 2                             # small W, batch > 8: GEMM
     for fmt in ("q1g128", "t2g128"):
-        assert ws(fmt, 24576, 4096, 8) == 0 and nl(fmt, 24576, 4096, 8) == 1
+        # batch 5..16: the wide-batch kernel where it measured fastest and its
+        # FP16 x (2 K bytes per row, rows padded to 8 or 16) fits: batch 16 at
+        # K = 4096 (128 KB), batch 8 at K = 12288 (192 KB); batch 16 at K = 12288
+        # (384 KB) goes to the GEMM
+        for n, k, b in ((16385, 4096, 9), (151936, 4096, 16), (4096, 12288, 8), (5, 8192, 5)):
+            assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)
+        assert ws(fmt, 4096, 12288, 16) >= 16 * 12288 * 2
+        assert ws(fmt, 6144, 4096, 6) == 0 and nl(fmt, 6144, 4096, 6) == 1          # row-owning
         assert ws(fmt, 4096, 17408, 4) > 0 and nl(fmt, 4096, 17408, 4) == 2  # operand too large: split-K
     # batch 4 at K = 12288: the operand takes 209 KB; two 5 KB binary slots still fit
     # beside it (row-owning), one 9 KB 2-bit slot does not (split-K)
@@ -184,3 +196,49 @@ def test_affine_sizes_match_oracle(lib):
         assert bq.bq_group_params_bytes("q1g128", n, k) == bq.bq_scales_bytes(n, k)
     assert bq.bq_effective_bits("a1g128") == oracle.effective_bits("a1g128") == 1.25
     assert bq.bq_gemm_workspace_bytes("a1g128", 64, 1024, 64) == -1
+
+
+def test_kv4_argument_errors_need_no_device(lib):
+    """4-bit KV-cache calls: sizes and argument errors are decided on the host
+    before any launch."""
+    vp = ctypes.c_void_p
+    assert lib.bq_kv4_codes_bytes(10, 128) == 640 and lib.bq_kv4_params_bytes(10, 128) == 40
+    assert lib.bq_kv4_codes_bytes(3, 256) == 384 and lib.bq_kv4_params_bytes(3, 256) == 24
+    assert lib.bq_kv4_codes_bytes(1, 64) == -1 and lib.bq_kv4_params_bytes(-1, 128) == -1
+    assert lib.bq_kv4_quantize(vp(16), 4, 64, vp(16), vp(16), None) == bq.BQ_ERR_SHAPE
+    assert lib.bq_kv4_quantize(vp(16), 0, 128, None, None, None) == bq.BQ_OK
+    assert lib.bq_kv4_quantize(None, 4, 128, vp(16), vp(16), None) == bq.BQ_ERR_NULL
+    assert lib.bq_kv4_quantize(vp(24), 4, 128, vp(16), vp(16), None) == bq.BQ_ERR_ALIGN
+    ok_append = dict(batch=2, hkv=2, d=128, l_cap=64)
+
+    def append(**kw):
+        a = dict(ok_append, **kw)
+        return lib.bq_kv4_append(vp(16), vp(16), a["batch"], a["hkv"], a["d"], vp(16), a["l_cap"], vp(16),
+                                 vp(16), vp(16), vp(16), None)
+    assert append(l_cap=100) == bq.BQ_ERR_SHAPE
+    assert append(d=64) == bq.BQ_ERR_SHAPE
+    assert append(batch=0) == bq.BQ_OK
+    ws = lib.bq_kv4_attention_workspace_bytes
+    assert ws(1, 32, 8, 128, 65536, 65536) > 0      # one sequence: the context is split across CTAs
+    assert ws(16, 32, 8, 128, 4096, 4096) == 0      # 128 (sequence, KV head) pairs: one CTA each
+    assert ws(1, 36, 4, 128, 64, 64) == -1          # 9 query heads per KV head
+    assert ws(1, 32, 8, 96, 64, 64) == -1           # head dimension
+    assert ws(1, 32, 8, 128, 100, 64) == -1         # capacity not a multiple of 64
+    assert ws(1, 32, 8, 128, 64, 65) == -1          # max_len above the capacity
+
+    def attn(**kw):
+        a = dict(q=vp(16), lens=vp(16), batch=1, hq=8, hkv=2, d=128, l_cap=64, max_len=64, scale=0.1,
+                 out=vp(16), odt=bq.BQ_BF16)
+        a.update(kw)
+        return lib.bq_kv4_attention_decode(a["q"], vp(16), vp(16), vp(16), vp(16), a["lens"], a["batch"], a["hq"],
+                                           a["hkv"], a["d"], a["l_cap"], a["max_len"], a["scale"], a["out"],
+                                           a["odt"], None, 0, None)
+    assert attn(d=64) == bq.BQ_ERR_SHAPE
+    assert attn(hq=18) == bq.BQ_ERR_SHAPE
+    assert attn(odt=9) == bq.BQ_ERR_FORMAT
+    assert attn(scale=float("inf")) == bq.BQ_ERR_SHAPE
+    assert attn(q=None) == bq.BQ_ERR_NULL
+    assert attn(out=vp(8)) == bq.BQ_ERR_ALIGN
+    assert attn(lens=vp(18)) == bq.BQ_ERR_ALIGN
+    assert attn(batch=0) == bq.BQ_OK
+    assert attn(l_cap=65536, max_len=65536, hq=32, hkv=8) == bq.BQ_ERR_WORKSPACE
