@@ -56,7 +56,58 @@ def parse():
                    help="one bq_gemv per product (calls) or one bq_gemv_chain per layer (chain)")
     p.add_argument("--gemm-only", action="store_true",
                    help="run only the prefill GEMM leg (a diagnostic line, e.g. for a profiler)")
+    p.add_argument("--case", choices=["gemv", "kv4"], default=None,
+                   help="profiler case: each launch once to warm up, then once after an L2 flush, and exit "
+                        "(gemv: --fmt, --batch, --shapes; kv4: --batch, --ctx)")
+    p.add_argument("--shapes", default="6144x4096,4096x4096,24576x4096,4096x12288,151936x4096",
+                   help="NxK list for --case gemv (default: one Qwen3-8B layer's launches and the LM head)")
+    p.add_argument("--ctx", type=int, default=65536, help="context tokens for --case kv4")
     return p.parse_args()
+
+
+def run_case(args):
+    """One launch per shape after a warm-up launch and a 256 MB L2 flush: the
+    small, self-ending workloads profiler captures are taken on."""
+    import math
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+    dev = torch.device("cuda", 0)
+    gen = synth.device_generator(synth.SEED_BASE + 9, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    calls = []
+    if args.case == "gemv":
+        f = FMT_NAMES[args.fmt]
+        for sh in args.shapes.split(","):
+            n, k = (int(v) for v in sh.split("x"))
+            codes, scales = make_weights(f, n, k, gen, dev, False)
+            x = synth.device_x_bf16(gen, args.batch, k, device=dev)
+            y = torch.empty((args.batch, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(bq.bq_gemv_workspace_bytes(f, n, k, args.batch), 256), dtype=torch.uint8, device=dev)
+            calls.append(lambda f=f, c=codes, s=scales, n=n, k=k, x=x, y=y, ws=ws:
+                         bq.bq_gemv(f, c, s, n, k, x, y=y, workspace=ws))
+    else:
+        A = synth.QWEN3_8B_ATTN
+        B, ctx, hq, hkv, d = args.batch, args.ctx, A["hq"], A["hkv"], A["d"]
+        cache = synth.device_kv4_cache(gen, B, hkv, ctx, d, device=dev) + \
+            synth.device_kv4_cache(gen, B, hkv, ctx, d, device=dev)
+        q = synth.device_x_bf16(gen, B * hq, d, device=dev).view(B, hq, d)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        o = torch.empty((B, hq, d), dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(bq.bq_kv4_attention_workspace_bytes(B, hq, hkv, d, ctx, ctx), 256),
+                         dtype=torch.uint8, device=dev)
+        calls.append(lambda: bq.bq_kv4_attention_decode(q, *cache, lens, ctx, 1.0 / math.sqrt(d), out=o,
+                                                        workspace=ws))
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    for c in calls:
+        flush.fill_(1)
+        c()
+    torch.cuda.synchronize()
+    assert bq.bq_check() == bq.BQ_OK
+    print(json.dumps({"case": args.case, "launches": len(calls)}), flush=True)
+    return 0
 
 
 def model_shapes(model):
@@ -246,6 +297,134 @@ def gemm_leg(fmt, dev, reps):
             "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst; FP16 operands at the same rate)",
             "kernel": "xprep_f16_kernel + gemm_tc_kernel (tcgen05 kind::f16, TMEM accumulators); T <= 4: the GEMV",
             "dtype": "f16 operands (exact s*q and pre-scaled x), f32 accumulate", "cases": out}
+
+
+def embed_leg(dev, reps):
+    """The 1-bit embedding lookup (bq_embed_rows) on the Qwen3-8B table
+    (151936 x 4096, binary g128) for 1, 16 and 4096 token ids: 20 lookups of
+    fresh random ids per CUDA graph, bytes = table rows read + BF16 rows written."""
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+    hbm, _ = measured_peaks()
+    n, k = synth.QWEN3_8B_LM_HEAD
+    gen = synth.device_generator(synth.SEED_BASE + 8, device=dev)
+    codes, scales = make_weights("q1g128", n, k, gen, dev, True)
+    out = []
+    for count in (1, 16, 4096):
+        ids = [torch.randint(0, n, (count,), generator=gen, device=dev, dtype=torch.int32) for _ in range(20)]
+        o = torch.empty((count, k), dtype=torch.bfloat16, device=dev)
+        for i in ids[:3]:
+            bq.bq_embed_rows("q1g128", codes, scales, n, k, i, out=o)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in ids:
+                bq.bq_embed_rows("q1g128", codes, scales, n, k, i, out=o)
+        g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / len(ids))
+        assert bq.bq_check() == bq.BQ_OK
+        ms = statistics.median(times)
+        byts = count * (bq.bq_codes_bytes("q1g128", 1, k) + bq.bq_scales_bytes(1, k) + 2 * k + 4)
+        out.append({"tokens": count, "us": round(1000.0 * ms, 2), "bytes": byts,
+                    "GB_s": round(byts / (ms / 1000.0) / 1e9, 1), "frac": round(byts / (ms / 1000.0) / 1e9 / hbm, 4)})
+        del g
+    return {"workload": "qwen3-8b embedding table 151936x4096 q1g128, random token ids, one launch per lookup",
+            "kernel": "embed_rows_kernel", "bound": "hbm", "peak": hbm, "cases": out}
+
+
+def attention_leg(dev, reps):
+    """4-bit KV-cache decode attention of Qwen3-8B (32 query / 8 KV heads, head
+    dimension 128): a step is one decode token through 36 layers, each layer
+    appending the token's K and V to its own cache (bq_kv4_append) and attending
+    over the whole context (bq_kv4_attention_decode), in one CUDA graph.  The
+    36 caches together exceed L2.  Reported as cache GB/s against HBM, plus one
+    attention launch timed alone (L2 flushed before it)."""
+    import math
+    import torch
+    import synth
+    import ternary_g128_weight_b200 as bq
+    A = synth.QWEN3_8B_ATTN
+    hq, hkv, d, layers = A["hq"], A["hkv"], A["d"], synth.QWEN3_8B_BLOCKS
+    hbm, _ = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = []
+    for B, ctx in ((1, 65536), (16, 4096)):
+        gen = synth.device_generator(synth.SEED_BASE + 7, device=dev)
+        caches = [synth.device_kv4_cache(gen, B, hkv, ctx, d, device=dev) +
+                  synth.device_kv4_cache(gen, B, hkv, ctx, d, device=dev) for _ in range(layers)]
+        q = synth.device_x_bf16(gen, B * hq, d, device=dev).view(B, hq, d)
+        kn = synth.device_x_bf16(gen, B * hkv, d, device=dev).view(B, hkv, d)
+        vn = synth.device_x_bf16(gen, B * hkv, d, device=dev).view(B, hkv, d)
+        lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+        pos = lens - 1
+        o = torch.empty((B, hq, d), dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(bq.bq_kv4_attention_workspace_bytes(B, hq, hkv, d, ctx, ctx), 256), dtype=torch.uint8,
+                         device=dev)
+        scale = 1.0 / math.sqrt(d)
+
+        def layer(c):
+            bq.bq_kv4_append(kn, vn, pos, c[0], c[1], c[2], c[3])
+            bq.bq_kv4_attention_decode(q, c[0], c[1], c[2], c[3], lens, ctx, scale, out=o, workspace=ws)
+
+        for c in caches:
+            layer(c)
+        torch.cuda.synchronize()
+        st = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            for c in caches:
+                layer(c)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            # (replay() launches on the current stream: time it there)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        # one attention launch alone, L2 flushed, events on its stream
+        a_times = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            bq.bq_kv4_attention_decode(q, *caches[0], lens, ctx, scale, out=o, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            a_times.append(e0.elapsed_time(e1))
+        assert bq.bq_check() == bq.BQ_OK
+        cache_bytes = B * hkv * ctx * (bq.bq_kv4_codes_bytes(1, d) + bq.bq_kv4_params_bytes(1, d)) * 2
+        algo = cache_bytes + B * hq * d * 2 * 2 + B * 4  # + q in, out, lens
+        a_ms = statistics.median(a_times)
+        out.append({"workload": f"qwen3-8b decode attention, 4-bit g128 KV cache, batch {B} x {ctx} tokens, "
+                                f"{layers} layers (append + attention per layer)",
+                    "batch": B, "context": ctx, "ms_per_step": round(ms, 4),
+                    "value": round(layers * algo / (ms / 1000.0) / 1e9, 1), "unit": "GB/s",
+                    "frac": round(layers * algo / (ms / 1000.0) / 1e9 / hbm, 4),
+                    "us_per_layer": round(1000.0 * ms / layers, 2),
+                    "tokens_per_s": round(1000.0 / ms, 1),
+                    "attention_launch": {"us": round(1000.0 * a_ms, 2), "bytes": algo,
+                                         "GB_s": round(algo / (a_ms / 1000.0) / 1e9, 1),
+                                         "frac": round(algo / (a_ms / 1000.0) / 1e9 / hbm, 4)},
+                    "launches_per_step": 2 * layers})
+        del caches, g
+        torch.cuda.empty_cache()
+    return {"bound": "hbm", "peak": hbm, "kernel": "attn_kernel (bq_kv4_attention_decode) + append_kernel",
+            "dtype": "f16 operands (q pre-scaled, codes c - 8, P s_V 2^sigma), f32 accumulate", "cases": out}
 
 
 # ------------------------------------------------------------------ reference
@@ -545,6 +724,8 @@ def main():
         args.layers = model_shapes(args.model)[2]
     if args.impl == "reference":
         return run_reference(args)
+    if args.case:
+        return run_case(args)
 
     import torch
     import ternary_g128_weight_b200 as bq
@@ -645,6 +826,8 @@ def main():
             legs.append(leg(model, lf, lb, mode, dev, args.leg_steps, 3, peak, synth_seed(rank) + 100 + i))
     if rank == 0 and not args.no_gemm:
         prefill = {lf: gemm_leg(lf, dev, 5) for lf in (["q1g128", "t2g128", "t5p8"] if not args.no_legs else [fmt])}
+    attention = attention_leg(dev, 5) if rank == 0 and not args.no_legs else None
+    embedding = embed_leg(dev, 5) if rank == 0 and not args.no_legs else None
 
     if rank == 0:
         line = {
@@ -682,6 +865,10 @@ def main():
             line["configs"] = legs
         if prefill:
             line["prefill_gemm"] = prefill
+        if attention:
+            line["kv4_attention"] = attention
+        if embedding:
+            line["embedding"] = embedding
         print(json.dumps(line), flush=True)
 
     if dist is not None:

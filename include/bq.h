@@ -166,11 +166,9 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
  * Kernel choice (the same for bq_gemv_noalloc and for bq_gemm with T <= 4):
  * K % 1024 == 0 with binary or 2-bit ternary codes at batch 5..16 runs the
  * wide-batch GEMV (FP16 effective weights +-s / {-s,0,+s} built in registers,
- * x pre-scaled per row to FP16, one launch, no workspace) where it measured
- * fastest -- at batch 5..8 binary W of >= 64 Mi weights or K >= 8192, at batch
- * 9..16 W of >= 64 Mi weights -- and its FP16 activations (2 K bytes per row,
- * rows padded to 8 or 16) fit in shared memory; batch <= 8 and K % 1024 == 0
- * otherwise run the row-owning
+ * x pre-scaled per row to FP16, one launch, no workspace) when its FP16
+ * activations (2 K bytes per row, rows padded to 8 or 16) fit in shared
+ * memory; batch <= 8 and K % 1024 == 0 otherwise run the row-owning
  * tensor-core GEMV (all three formats, one launch, no workspace) when its
  * activation operand and a ring of at least two weight slots fit in shared
  * memory; otherwise binary and 2-bit ternary at batch <= 4 run the split-K

@@ -141,3 +141,17 @@ def device_x_bf16(gen, batch: int, k: int, device="cuda"):
 def device_code_bytes(gen, nbytes: int, device="cuda"):
     import torch
     return torch.randint(0, 256, (nbytes,), generator=gen, device=device, dtype=torch.int16).to(torch.uint8)
+
+
+def device_kv4_cache(gen, b: int, hkv: int, l_cap: int, d: int, s_lo=0.02, s_hi=0.2, device="cuda"):
+    """kv4_cache_bytes drawn on the device (torch's CUDA generator): (codes
+    uint8 [b][hkv][l_cap][d/2], params int32 [b][hkv][l_cap][d/128])."""
+    import torch
+    codes = torch.randint(0, 256, (b, hkv, l_cap, d // 2), generator=gen, device=device,
+                          dtype=torch.int16).to(torch.uint8)
+    shape = (b, hkv, l_cap, d // 128)
+    s = torch.rand(shape, generator=gen, device=device) * (s_hi - s_lo) + s_lo
+    z = -7.5 * s * (1.0 + (torch.rand(shape, generator=gen, device=device) * 0.2 - 0.1))
+    sb = s.to(torch.float16).view(torch.int16).to(torch.int32) & 0xFFFF
+    zb = z.to(torch.float16).view(torch.int16).to(torch.int32) << 16
+    return codes, sb | zb

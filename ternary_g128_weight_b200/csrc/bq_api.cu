@@ -81,21 +81,14 @@ int* device_status_ptr() {
 }  // namespace bq
 
 namespace bq {
-// Where the wide-batch kernel beats the alternatives, as measured on B200
-// (one launch per matrix, weights larger than L2): at batch 5..8 against the
-// row-owning kernel for binary matrices of >= 64 Mi weights and for K >= 8192
-// (4096 x 12288: 28 vs 38 us binary, 33 vs 41 us 2-bit; 4096 x 4096: 12.0 vs
-// 9.1 us, so not there); at batch 9..16 against the tcgen05 GEMM for >= 64 Mi
-// weights (24576 x 4096 binary: 35 vs 63 us; 4096 x 4096: 23 vs 19 us).
-static bool prefer_wide(int fmt, int64_t n, int64_t k, int batch) {
-    const int64_t weights = n * k;
-    constexpr int64_t kLarge = 64LL << 20;
-    if (batch <= 8) return (fmt == BQ_Q1G128 && weights >= kLarge) || k >= 8192;
-    return weights >= kLarge;
-}
-
+// Batch 5..16 takes the wide-batch kernel wherever it is eligible: measured
+// on B200 (one launch per matrix, weights larger than L2) it is as fast as or
+// faster than the row-owning kernel at batch 5..8 (binary 4096 x 4096 batch 5:
+// 7.8 vs 9.1 us; 4096 x 12288: 15.2 vs 37.9 us) and than the tcgen05 GEMM at
+// batch 9..16 (binary 4096 x 4096 batch 16: 15.1 vs 18.8 us; 24576 x 4096:
+// 26.8 vs 62.7 us).
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
-    if (batch >= 5 && prefer_wide(fmt, n, k, batch) && gemv_wide_eligible(fmt, n, k, batch)) return GemvPath::Wide;
+    if (batch >= 5 && gemv_wide_eligible(fmt, n, k, batch)) return GemvPath::Wide;
     if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
     if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
     if (gemm_tc_eligible(fmt, n, k, batch)) return GemvPath::Gemm;

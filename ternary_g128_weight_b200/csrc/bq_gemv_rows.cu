@@ -1020,7 +1020,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
 // row's largest magnitude), so the MMA accumulates s * q * x over all of K in
 // FP32 and y = acc * 2^-e_b -- no per-group recombination and no digit split:
 // one decoded 16 x 16 weight fragment feeds one MMA per 8 batch rows.
-constexpr int kWideAux = 256;  // row maxima, exponents and 2^-e per batch row
+constexpr int kWideAux = 256;  // per batch row: largest |x|, 2^e as two factors, 2^-e
 
 // Activation area per stage: [group G][j 0..7][batch row b][thread t][2 words],
 // word p of (G, b, t) the FP16 pair of the two activations register p of a
@@ -1042,8 +1042,8 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
     constexpr int BP = NTW * 8;
     const int tid = threadIdx.x;
     uint32_t* rmax = reinterpret_cast<uint32_t*>(smem + p.lut_off);
-    int* es = reinterpret_cast<int*>(smem + p.lut_off + 64);
-    float* inv = reinterpret_cast<float*>(smem + p.lut_off + 128);
+    float2* fac = reinterpret_cast<float2*>(smem + p.lut_off + 64);  // 2^e as two exact factors
+    float* inv = reinterpret_cast<float*>(smem + p.lut_off + 192);
     if (tid < BP) rmax[tid] = 0u;
     bar_compute<NW>();
     // largest |x| of every batch row (FP32 bits of the magnitude: monotonic)
@@ -1064,7 +1064,8 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
     if (tid < BP) {
         const float m = __uint_as_float(rmax[tid]);
         const int e = m > 0.f ? 14 - ilog2f(m) : 0;  // in [-113, 147]
-        es[tid] = e;
+        const int e1 = min(e, 127);                   // 2^e = 2^e1 2^(e - e1), both normal
+        fac[tid] = make_float2(__int_as_float((e1 + 127) << 23), __int_as_float((e - e1 + 127) << 23));
         inv[tid] = ldexpf(1.0f, -e);  // exact (a subnormal below 2^-126)
     }
     bar_compute<NW>();
@@ -1082,16 +1083,20 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
                 const uint4 v = __ldg(src + q);
                 raw[4 * q] = v.x; raw[4 * q + 1] = v.y; raw[4 * q + 2] = v.z; raw[4 * q + 3] = v.w;
             }
-            const int e = es[b];
-            uint16_t h[32];
+            // x 2^e rounded once to FP16 (the two power-of-two products are
+            // exact while the value stays in the FP32 normal range; below it
+            // the FP16 result is zero either way)
+            const float2 f = fac[b];
+            float v[32];
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const float v = __uint_as_float((r & 1) ? (raw[r >> 1] & 0xFFFF0000u) : (raw[r >> 1] << 16));
-                h[r] = __half_as_ushort(__float2half_rn(ldexpf(v, e)));
+            for (int r = 0; r < 32; ++r)
+                v[r] = __uint_as_float((r & 1) ? (raw[r >> 1] & 0xFFFF0000u) : (raw[r >> 1] << 16)) * f.x * f.y;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                uint32_t w2;
+                asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w2) : "f"(v[wide_hi<FMT>(q)]), "f"(v[wide_lo<FMT>(q)]));
+                words[q] = w2;
             }
-#pragma unroll
-            for (int q = 0; q < 16; ++q)
-                words[q] = (uint32_t)h[wide_lo<FMT>(q)] | ((uint32_t)h[wide_hi<FMT>(q)] << 16);
         } else {
 #pragma unroll
             for (int q = 0; q < 16; ++q) words[q] = 0u;
@@ -1236,7 +1241,7 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
         bar_compute<NW>();
     }
     if (active && gsub == 0) {
-        const float* inv = reinterpret_cast<const float*>(smem + p.lut_off + 128);
+        const float* inv = reinterpret_cast<const float*>(smem + p.lut_off + 192);
 #pragma unroll
         for (int tp = 0; tp < TPW; ++tp)
 #pragma unroll

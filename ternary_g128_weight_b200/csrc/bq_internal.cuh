@@ -93,8 +93,7 @@ cudaError_t launch_gemv_chain(int fmt, const bq_chain_step* steps, int nsteps, i
                               cudaStream_t s);
 
 // GEMV path choice shared by bq_gemv, bq_gemm (T <= 16) and bq_gemv_noalloc:
-// batch 5..16 the wide-batch kernel where eligible and measured faster
-// (prefer_wide); the row-owning kernel
+// batch 5..16 the wide-batch kernel where eligible; the row-owning kernel
 // where eligible, else the split-K tensor-core kernel,
 // else the tcgen05 GEMM with T = batch; None when no kernel takes the shape
 // (K > 2^28 or N >= 2^31).  gemv_workspace_bytes reports the workspace of the

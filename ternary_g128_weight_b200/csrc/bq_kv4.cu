@@ -78,23 +78,47 @@ struct AttnParams {
     int nsplit, spc;   // CTAs per (sequence, KV head), stages per CTA
     void* out;         // [B][Hq][D], BF16 or F32
     int out_f32;
-    float* part;         // [B*Hkv][nsplit][G][D + 2] (nsplit > 1)
+    float* part_o;       // [B*Hkv][nsplit][G][D]  unnormalised outputs (nsplit > 1)
+    float* part_ml;      // [B*Hkv][nsplit][G][2]  running max (log2 units) and sum
     unsigned* counters;  // [B*Hkv], zero between calls (nsplit > 1)
     int* status;
 };
 
-__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+// f16x2 arithmetic on plain 32-bit registers (no __half2 round trips).
+__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+// (FP16(lo), FP16(hi)) packed, lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// 2^x by the hardware approximation (relative error about 2^-22; -inf -> 0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// 2^e for -126 <= e <= 127, exactly.
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // The codes at bits 0..3 and 16..19 of w as the FP16 pair (c_lo - 8, c_hi - 8):
 // 0x6400 | c is 1024 + c, exact; adding -1032 is exact.
 __device__ __forceinline__ uint32_t dq_lo(uint32_t w) {
-    return h2u(__hadd2(u2h((w & 0x000F000Fu) | 0x64006400u), u2h(0xE408E408u)));
+    return hadd2_u((w & 0x000F000Fu) | 0x64006400u, 0xE408E408u);
 }
 // The codes at bits 4..7 and 20..23: 0x6400 | 16 c is 1024 + 16 c; times 1/16
 // minus 72 gives c - 8, exactly.
 __device__ __forceinline__ uint32_t dq_hi(uint32_t w) {
-    return h2u(__hfma2(u2h((w & 0x00F000F0u) | 0x64006400u), u2h(0x2C002C00u), u2h(0xD480D480u)));
+    return hfma2_u((w & 0x00F000F0u) | 0x64006400u, 0x2C002C00u, 0xD480D480u);
 }
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
@@ -183,8 +207,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
         mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 2));
         // power of two that puts the head's largest |q| in [2^14, 2^15): the
-        // FP16 values are the BF16 ones exactly (up to FP16 underflow)
-        const int ex = mx > 0.f ? 14 - ilogbf(mx) : 0;
+        // FP16 values are the BF16 ones exactly (up to FP16 underflow; a head
+        // whose largest |q| is below 2^-112 keeps the factor 2^126)
+        const int ex = mx > 0.f ? min(14 - ilogbf(mx), 126) : 0;
+        const float fx = pow2i(ex);
         float sum[NG];
 #pragma unroll
         for (int grp = 0; grp < NG; ++grp) {
@@ -192,21 +218,23 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
             sum[grp] = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                h[i] = __float2half_rn(ldexpf(v[grp][i], ex));
+                h[i] = __float2half_rn(v[grp][i] * fx);
                 sum[grp] += __half2float(h[i]);
             }
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const int u = s >> 1, j = 2 * (s & 1);
-                qb[grp][s][0] = h2u(__halves2half2(h[8 * u + j], h[8 * u + j + 4]));
-                qb[grp][s][1] = h2u(__halves2half2(h[8 * u + j + 1], h[8 * u + j + 5]));
+                qb[grp][s][0] = (uint32_t)__half_as_ushort(h[8 * u + j]) |
+                                ((uint32_t)__half_as_ushort(h[8 * u + j + 4]) << 16);
+                qb[grp][s][1] = (uint32_t)__half_as_ushort(h[8 * u + j + 1]) |
+                                ((uint32_t)__half_as_ushort(h[8 * u + j + 5]) << 16);
             }
             sum[grp] += __shfl_xor_sync(~0u, sum[grp], 1);
             sum[grp] += __shfl_xor_sync(~0u, sum[grp], 2);
         }
         // per-head constants of the score epilogue, for the heads 2t, 2t+1 this
         // thread's accumulator columns hold (head g' lives in lanes 4 g')
-        const float cg = ldexpf(p.scale_log2, -ex);
+        const float cg = p.scale_log2 * pow2i(-ex);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             ch[j] = __shfl_sync(~0u, cg, 4 * (2 * t + j));
@@ -307,9 +335,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
         smax = fmaxf(smax, __shfl_xor_sync(~0u, smax, 2));
         const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
         const int sig_new = smax > 0.f ? min(sig, 14 - ilogbf(smax)) : sig;
-        const float fl0 = (mn0 == -INFINITY) ? 1.f : exp2f(m_run[0] - mn0);
-        const float fl1 = (mn1 == -INFINITY) ? 1.f : exp2f(m_run[1] - mn1);
-        const float fs = ldexpf(1.f, sig_new - sig);
+        const float fl0 = (mn0 == -INFINITY) ? 1.f : ex2(m_run[0] - mn0);
+        const float fl1 = (mn1 == -INFINITY) ? 1.f : ex2(m_run[1] - mn1);
+        const float fs = pow2i(sig_new - sig);
         const float fo0 = fl0 * fs, fo1 = fl1 * fs;
         if (__any_sync(~0u, fo0 != 1.f || fo1 != 1.f)) {
 #pragma unroll
@@ -333,13 +361,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
         m_run[1] = mn1;
         sig = sig_new;
         const float mref0 = mn0 == -INFINITY ? 0.f : mn0, mref1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float pscale = ldexpf(1.f, sig);
+        const float pscale = pow2i(sig);
 
         // P V
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            const float p00 = exp2f(sc[mt][0] - mref0), p01 = exp2f(sc[mt][1] - mref1);
-            const float p10 = exp2f(sc[mt][2] - mref0), p11 = exp2f(sc[mt][3] - mref1);
+            const float p00 = ex2(sc[mt][0] - mref0), p01 = ex2(sc[mt][1] - mref1);
+            const float p10 = ex2(sc[mt][2] - mref0), p11 = ex2(sc[mt][3] - mref1);
             l_run[0] += p00 + p10;
             l_run[1] += p01 + p11;
             const uint8_t* vrow = sb + Gm::VC + mt * 16 * Gm::ROWB + 8 * g;
@@ -350,8 +378,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
                 const float f0 = sv[mt][0][grp] * pscale, f1 = sv[mt][1][grp] * pscale;
                 // P'' of rows g / g+8 (tokens) and columns 2t, 2t+1 (heads),
                 // transposed to the B fragment: (tokens 2t, 2t+1 | 2t+8, 2t+9; head g)
-                const uint32_t b0 = movmatrix_t(h2u(__floats2half2_rn(p00 * f0, p01 * f0)));
-                const uint32_t b1 = movmatrix_t(h2u(__floats2half2_rn(p10 * f1, p11 * f1)));
+                const uint32_t b0 = movmatrix_t(pack_half2(p00 * f0, p01 * f0));
+                const uint32_t b1 = movmatrix_t(pack_half2(p10 * f1, p11 * f1));
                 const uint8_t* vg = vrow + 64 * grp;
                 const uint2 va = *reinterpret_cast<const uint2*>(vg + (2 * t) * Gm::ROWB);
                 const uint2 vb = *reinterpret_cast<const uint2*>(vg + (2 * t + 1) * Gm::ROWB);
@@ -401,7 +429,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
     float* mm = mo + kWarps * kMaxHeads * D;              // [kWarps][8]
     float* ml = mm + kWarps * kMaxHeads;                  // [kWarps][8]
     float* wgt = ml + kWarps * kMaxHeads;                 // [nsplit][8], then [8] totals
-    const float inv = ldexpf(1.f, -sig);
+    const float inv = pow2i(-sig);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const int h = 2 * t + j;
@@ -444,11 +472,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
             else
                 static_cast<uint16_t*>(p.out)[oi] = float_to_bf16_bits(r);
         } else {
-            float* pp = p.part + (((int64_t)bh * p.nsplit + c) * p.G + h) * (D + 2);
-            pp[d] = O;
+            const int64_t slot = ((int64_t)bh * p.nsplit + c) * p.G + h;
+            p.part_o[slot * D + d] = O;
             if (d == 0) {
-                pp[D] = M;
-                pp[D + 1] = L;
+                p.part_ml[2 * slot] = M;
+                p.part_ml[2 * slot + 1] = L;
             }
         }
     }
@@ -461,33 +489,58 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const float* base = p.part + (int64_t)bh * p.nsplit * p.G * (D + 2);
+    // every split's (max, sum) into shared memory, all loads in flight at once
+    const int nsg = p.nsplit * p.G;
+    const float* pml = p.part_ml + (int64_t)bh * nsg * 2;
+    float* sw = wgt;                 // [nsplit * G] maxima, then weights
+    float* sl = wgt + nsg;           // [nsplit * G] sums
+    float* tot = sl + nsg;           // [G] totals
+    for (int i = threadIdx.x; i < nsg; i += blockDim.x) {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(pml) + i);
+        sw[i] = v.x;
+        sl[i] = v.y;
+    }
+    __syncthreads();
     if (threadIdx.x < p.G) {
         const int h = threadIdx.x;
         float M = -INFINITY;
-        for (int cc = 0; cc < p.nsplit; ++cc) M = fmaxf(M, __ldcg(base + ((int64_t)cc * p.G + h) * (D + 2) + D));
+        for (int cc = 0; cc < p.nsplit; ++cc) M = fmaxf(M, sw[cc * p.G + h]);
         float L = 0.f;
         for (int cc = 0; cc < p.nsplit; ++cc) {
-            const float* pp = base + ((int64_t)cc * p.G + h) * (D + 2);
-            const float a = M == -INFINITY ? 0.f : exp2f(__ldcg(pp + D) - M);
-            wgt[cc * kMaxHeads + h] = a;
-            L = fmaf(a, __ldcg(pp + D + 1), L);
+            const float a = M == -INFINITY ? 0.f : exp2f(sw[cc * p.G + h] - M);
+            sw[cc * p.G + h] = a;
+            L = fmaf(a, sl[cc * p.G + h], L);
         }
-        wgt[p.nsplit * kMaxHeads + h] = L;
+        tot[h] = L;
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < nout; idx += blockDim.x) {
-        const int h = idx / D, d = idx - h * D;
-        float O = 0.f;
-        for (int cc = 0; cc < p.nsplit; ++cc)
-            O = fmaf(wgt[cc * kMaxHeads + h], __ldcg(base + ((int64_t)cc * p.G + h) * (D + 2) + d), O);
-        const float L = wgt[p.nsplit * kMaxHeads + h];
-        const float r = L > 0.f ? O / L : 0.f;
+    // outputs four at a time; the split loop is unrolled so that its loads are
+    // issued together (the sum is still taken in split order)
+    const float* po = p.part_o + (int64_t)bh * nsg * D;
+    const int nq = p.G * (D / 4);
+    for (int idx = threadIdx.x; idx < nq; idx += blockDim.x) {
+        const int h = idx / (D / 4), d = 4 * (idx - h * (D / 4));
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int cc = 0; cc < p.nsplit; ++cc) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(po + ((int64_t)cc * p.G + h) * D + d));
+            const float a = sw[cc * p.G + h];
+            O.x = fmaf(a, v.x, O.x);
+            O.y = fmaf(a, v.y, O.y);
+            O.z = fmaf(a, v.z, O.z);
+            O.w = fmaf(a, v.w, O.w);
+        }
+        const float L = tot[h];
+        const float r[4] = {L > 0.f ? O.x / L : 0.f, L > 0.f ? O.y / L : 0.f, L > 0.f ? O.z / L : 0.f,
+                            L > 0.f ? O.w / L : 0.f};
         const int64_t oi = ((int64_t)bh * p.G + h) * D + d;
-        if (p.out_f32)
-            static_cast<float*>(p.out)[oi] = r;
-        else
-            static_cast<uint16_t*>(p.out)[oi] = float_to_bf16_bits(r);
+        if (p.out_f32) {
+            *reinterpret_cast<float4*>(static_cast<float*>(p.out) + oi) = make_float4(r[0], r[1], r[2], r[3]);
+        } else {
+            const uint32_t lo = float_to_bf16_bits(r[0]) | ((uint32_t)float_to_bf16_bits(r[1]) << 16);
+            const uint32_t hi = float_to_bf16_bits(r[2]) | ((uint32_t)float_to_bf16_bits(r[3]) << 16);
+            *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.out) + oi) = make_uint2(lo, hi);
+        }
     }
     if (threadIdx.x == 0) p.counters[bh] = 0u;  // left zero for the next call
 }
@@ -600,11 +653,13 @@ Plan make_plan(int batch, int hkv, int d, int64_t max_len) {
     return pl;
 }
 
+int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
+
 int64_t workspace_bytes(const Plan& pl, int batch, int hq, int hkv, int d) {
     if (pl.nsplit <= 1) return 0;
     const int64_t units = (int64_t)batch * hkv;
-    const int64_t part = units * pl.nsplit * (int64_t)(hq / hkv) * (d + 2) * 4;
-    return ((part + 255) / 256) * 256 + ((units * 4 + 255) / 256) * 256;
+    const int64_t slots = units * pl.nsplit * (int64_t)(hq / hkv);
+    return round256(slots * d * 4) + round256(slots * 8) + round256(units * 4);
 }
 
 template <int D>
@@ -737,10 +792,13 @@ extern "C" bq_status bq_kv4_attention_decode(const uint16_t* q, const uint8_t* k
     p.spc = pl.spc;
     p.out = out;
     p.out_f32 = out_dtype == BQ_F32;
-    p.part = static_cast<float*>(workspace);
     const int64_t units = (int64_t)batch * hkv;
-    const int64_t part_bytes = need > 0 ? need - ((units * 4 + 255) / 256) * 256 : 0;
-    p.counters = need > 0 ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(workspace) + part_bytes) : nullptr;
+    const int64_t slots = units * pl.nsplit * (int64_t)p.G;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    p.part_o = need > 0 ? reinterpret_cast<float*>(wsb) : nullptr;
+    p.part_ml = need > 0 ? reinterpret_cast<float*>(wsb + kv4::round256(slots * d * 4)) : nullptr;
+    p.counters = need > 0 ? reinterpret_cast<unsigned*>(wsb + kv4::round256(slots * d * 4) + kv4::round256(slots * 8))
+                          : nullptr;
     p.status = status;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = d == 128 ? kv4::launch_attn<128>(p, (int)units, s) : kv4::launch_attn<256>(p, (int)units, s);

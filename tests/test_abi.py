@@ -104,11 +104,10 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_gemv_launches(2, 4096, 4096, 4) == 1
     assert lib.bq_gemv_launches(3, 4096, 4096, 1) == 1       # 5-trit format, row-owning kernel too
     assert lib.bq_gemv_launches(3, 4096, 17408, 4) in (2, 3)  # operand too large: tcgen05 GEMM
-    assert lib.bq_gemv_launches(1, 24576, 4096, 16) == 1      # wide-batch kernel (large W)
-    assert lib.bq_gemv_launches(1, 4096, 4096, 16) in (2, 3)   # small W at batch 16: tcgen05 GEMM
+    assert lib.bq_gemv_launches(1, 4096, 4096, 16) == 1       # wide-batch kernel
     assert lib.bq_gemv_launches(3, 4096, 4096, 16) in (2, 3)   # 5-trit format at batch 16: tcgen05 GEMM
     assert lib.bq_gemv_launches(1, 4096, 12288, 16) in (2, 3)  # FP16 x exceeds shared memory: GEMM
-    assert lib.bq_gemm_launches(2, 24576, 4096, 12) == 1       # T 5..16, large W: the wide-batch GEMV
+    assert lib.bq_gemm_launches(2, 4096, 4096, 12) == 1        # T 5..16: the wide-batch GEMV
     assert lib.bq_gemm_launches(1, 17408, 5120, 4096) == 2     # prep + GEMM, no K split
     assert lib.bq_gemm_launches(1, 4096, 4096, 1) == 1         # T <= 4: the GEMV
     assert lib.bq_gemm_launches(1, 4096, 100, 8) == -1
@@ -126,16 +125,15 @@ def test_gemv_path_choice_host_only(lib):
         for n, k, b in ((4096, 4096, 1), (151936, 4096, 1), (4096, 12288, 1), (777, 1024, 2)):
             assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)   # row-owning
         assert ws(fmt, 4096, 1152, 1) >= 1152 * 2                                 # K % 1024 != 0: GEMM
-        assert ws(fmt, 4096, 4096, 9) >= 9 * 4096 * 2                             # small W, batch > 8: GEMM
+    assert ws("t5p8", 4096, 4096, 9) >= 9 * 4096 * 2                              # 5-trit, batch > 8: GEMM
     for fmt in ("q1g128", "t2g128"):
-        # batch 5..16: the wide-batch kernel where it measured fastest and its
-        # FP16 x (2 K bytes per row, rows padded to 8 or 16) fits: batch 16 at
-        # K = 4096 (128 KB), batch 8 at K = 12288 (192 KB); batch 16 at K = 12288
-        # (384 KB) goes to the GEMM
-        for n, k, b in ((16385, 4096, 9), (151936, 4096, 16), (4096, 12288, 8), (5, 8192, 5)):
+        # batch 5..16: the wide-batch kernel while its FP16 x (2 K bytes per row,
+        # rows padded to 8 or 16) fits: batch 16 at K = 4096 (128 KB), batch 8 at
+        # K = 12288 (192 KB); batch 16 at K = 12288 (384 KB) goes to the GEMM
+        for n, k, b in ((4096, 4096, 9), (16385, 4096, 9), (151936, 4096, 16), (4096, 12288, 8), (5, 1024, 5),
+                        (6144, 4096, 6)):
             assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)
         assert ws(fmt, 4096, 12288, 16) >= 16 * 12288 * 2
-        assert ws(fmt, 6144, 4096, 6) == 0 and nl(fmt, 6144, 4096, 6) == 1          # row-owning
         assert ws(fmt, 4096, 17408, 4) > 0 and nl(fmt, 4096, 17408, 4) == 2  # operand too large: split-K
     # batch 4 at K = 12288: the operand takes 209 KB; two 5 KB binary slots still fit
     # beside it (row-owning), one 9 KB 2-bit slot does not (split-K)

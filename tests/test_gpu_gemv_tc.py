@@ -26,7 +26,7 @@ def test_path_workspace(fmt):
     # tcgen05 GEMM with T = batch: workspace for the FP16 activations
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 1152, 1) >= 1152 * 2   # K % 1024 != 0
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 8) == 0               # batch 5..8 while x fits
-    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 9) >= 9 * 4096 * 2    # small W, batch 9: GEMM
+    assert bq.bq_gemv_workspace_bytes(fmt, 4096, 4096, 9) == 0               # wide-batch kernel
     assert bq.bq_gemv_workspace_bytes(fmt, 4096, 12288, 16) >= 16 * 12288 * 2  # its FP16 x exceeds shared memory
     assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 4096, 1) == 0       # row-owning kernel
     assert bq.bq_gemv_workspace_bytes("t5p8", 4096, 17408, 4) >= 4 * 17408 * 2   # GEMM

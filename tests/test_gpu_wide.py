@@ -19,10 +19,11 @@ def _bits(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-# Shapes the wide kernel takes (batch 5..8: K >= 8192; batch 9..16: >= 64 Mi
-# weights), with ragged row counts: element by element against the oracle.
-WIDE_CASES = [(b, n, k) for b in (5, 6, 8) for n, k in ((33, 8192), (300, 9216), (1001, 8192))] + \
-             [(b, n, k) for b in (9, 12, 16) for n, k in ((16385, 4096), (13120, 5120))]
+# Shapes on the wide path, with ragged row counts, several K stages and the
+# largest K each batch allows: element by element against the oracle.
+WIDE_CASES = [(b, n, k) for b in (5, 6, 8, 9, 12, 16) for n, k in ((33, 1024), (300, 2048), (1000, 4096))] + \
+             [(b, n, k) for b in (5, 8) for n, k in ((129, 8192), (300, 9216))] + \
+             [(b, n, k) for b in (9, 16) for n, k in ((16385, 4096), (1001, 5120))]
 
 
 @pytest.mark.parametrize("fmt", FMTS)
