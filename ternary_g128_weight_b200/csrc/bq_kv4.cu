@@ -19,10 +19,11 @@
 //  * a CTA owns one (sequence, KV head) and a range of the context; its 8 warps
 //    take interleaved stages of 8192 / D tokens, each warp with its own ring of
 //    three stages fed by 1-D bulk copies (K codes, V codes, K params, V params);
-//  * scores: mma.m16n8k16 with A = the K codes of 16 tokens as FP16 (c - 8)
-//    (built from the nibbles with one LOP3 and one HADD2/HFMA2 per pair) and B =
-//    the group's query heads (up to 8) pre-scaled to FP16 by a power of two;
-//    per token and group the score is s Σ q (c - 8) + (z + 8 s) Σ q;
+//  * scores: mma.m16n8k32 (u8 x s8 -> s32) with A = the K codes of 16 tokens
+//    (even / odd nibbles of a word masked into bytes: 3 instructions per 8
+//    values) and B = the group's query heads (up to 8) as 22-bit fixed point in
+//    three int8 digit planes, so Σ q c is exact in int32; per token and group the
+//    score is s Σ q c + z Σ q;
 //  * online softmax in the log2 domain, per head, once per stage;
 //  * P V: mma.m16n8k16 with A = V^T codes (the nibbles of two tokens paired by
 //    one PRMT) and B = P s_V 2^σ as FP16 (s_V folded into the weights, σ a
@@ -179,11 +180,16 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
     if (lane == 0)
         for (int i = 0; i < min(kRing, nmy); ++i) issue(i);
 
-    // ---- query head g of this KV group, as FP16 B fragments ----------------
-    // Thread (g, t) holds dims 128 grp + 32 t + [0, 32) of head g; k-step s of
-    // group grp pairs dims (j, j + 4) of its word u = s / 2 with j = 2 (s & 1)
-    // (b0) and j + 1 (b1), matching the K-code pairs below.
-    uint32_t qb[NG][8][2];
+    // ---- query head g of this KV group, as int8 digit planes ----------------
+    // Thread (g, t) holds dims 128 grp + 32 t + [0, 32) of head g.  Each value
+    // becomes the integer q22 = rint(q 2^e) (the head's largest |q| in
+    // [2^20, 2^21): exact for BF16 values within 2^-13 of it, else rounded by at
+    // most 2^-21 of it), split into balanced base-256 digits d0, d1 in
+    // [-128, 127] and d2 in [-33, 33] with q22 = 65536 d2 + 256 d1 + d0, one MMA
+    // B operand per digit plane.  K-step u of group grp reads word u of the
+    // thread's K codes: its even nibbles (dims 8u + 0, 2, 4, 6) fill k-slots
+    // 4t .. 4t+3 (b0), its odd nibbles k-slots 4t+16 .. 4t+19 (b1).
+    uint32_t qb[NG][4][3][2];
     float ch[2], dh[2][NG];
     {
         const bool hv = g < p.G;
@@ -206,28 +212,40 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
             }
         mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, 2));
-        // power of two that puts the head's largest |q| in [2^14, 2^15): the
-        // FP16 values are the BF16 ones exactly (up to FP16 underflow; a head
-        // whose largest |q| is below 2^-112 keeps the factor 2^126)
-        const int ex = mx > 0.f ? min(14 - ilogbf(mx), 126) : 0;
+        // (a head whose largest |q| is below 2^-106 keeps the factor 2^126)
+        const int ex = mx > 0.f ? min(20 - ilogbf(mx), 126) : 0;
         const float fx = pow2i(ex);
-        float sum[NG];
+        int sum[NG];
 #pragma unroll
         for (int grp = 0; grp < NG; ++grp) {
-            __half h[32];
-            sum[grp] = 0.f;
+            int qi[32];
+            sum[grp] = 0;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                h[i] = __float2half_rn(v[grp][i] * fx);
-                sum[grp] += __half2float(h[i]);
+                qi[i] = __float2int_rn(v[grp][i] * fx);
+                sum[grp] += qi[i];
             }
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const int u = s >> 1, j = 2 * (s & 1);
-                qb[grp][s][0] = (uint32_t)__half_as_ushort(h[8 * u + j]) |
-                                ((uint32_t)__half_as_ushort(h[8 * u + j + 4]) << 16);
-                qb[grp][s][1] = (uint32_t)__half_as_ushort(h[8 * u + j + 1]) |
-                                ((uint32_t)__half_as_ushort(h[8 * u + j + 5]) << 16);
+            for (int u = 0; u < 4; ++u) {
+                uint32_t b[2][3] = {{0u, 0u, 0u}, {0u, 0u, 0u}};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int odd = 0; odd < 2; ++odd) {
+                        const int a = qi[8 * u + 2 * i + odd];
+                        const int d0 = ((a + 128) & 255) - 128;
+                        const int r = (a - d0) >> 8;
+                        const int d1 = ((r + 128) & 255) - 128;
+                        const int d2 = (r - d1) >> 8;
+                        b[odd][0] |= (uint32_t)(d0 & 255) << (8 * i);
+                        b[odd][1] |= (uint32_t)(d1 & 255) << (8 * i);
+                        b[odd][2] |= (uint32_t)(d2 & 255) << (8 * i);
+                    }
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    qb[grp][u][j][0] = b[0][j];
+                    qb[grp][u][j][1] = b[1][j];
+                }
             }
             sum[grp] += __shfl_xor_sync(~0u, sum[grp], 1);
             sum[grp] += __shfl_xor_sync(~0u, sum[grp], 2);
@@ -239,7 +257,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
         for (int j = 0; j < 2; ++j) {
             ch[j] = __shfl_sync(~0u, cg, 4 * (2 * t + j));
 #pragma unroll
-            for (int grp = 0; grp < NG; ++grp) dh[j][grp] = __shfl_sync(~0u, cg * sum[grp], 4 * (2 * t + j));
+            for (int grp = 0; grp < NG; ++grp)
+                dh[j][grp] = __shfl_sync(~0u, cg * (float)sum[grp], 4 * (2 * t + j));
         }
     }
 
@@ -276,19 +295,31 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
         for (int mt = 0; mt < MT; ++mt) {
             const int r0 = mt * 16 + g, r1 = r0 + 8;
             const bool v0 = tok0 + r0 < len, v1 = tok0 + r1 < len;
-            float acc[NG][4];
+            // S = sum_d q22_d c_d per (token row, head column), exact: three
+            // int8 digit planes, one u8 x s8 MMA each per 32 dims
+            float S[NG][4];
 #pragma unroll
             for (int grp = 0; grp < NG; ++grp) {
-                acc[grp][0] = acc[grp][1] = acc[grp][2] = acc[grp][3] = 0.f;
+                int acc[3][4];
+#pragma unroll
+                for (int j = 0; j < 3; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
                 const uint4 k0 = *reinterpret_cast<const uint4*>(sb + Gm::KC + r0 * Gm::ROWB + 64 * grp + 16 * t);
                 const uint4 k1 = *reinterpret_cast<const uint4*>(sb + Gm::KC + r1 * Gm::ROWB + 64 * grp + 16 * t);
                 const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w}, w1[4] = {k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    ptx::mma_f16_16816(acc[grp], dq_lo(w0[u]), dq_lo(w1[u]), dq_hi(w0[u]), dq_hi(w1[u]),
-                                       qb[grp][2 * u][0], qb[grp][2 * u][1]);
-                    ptx::mma_f16_16816(acc[grp], dq_lo(w0[u] >> 8), dq_lo(w1[u] >> 8), dq_hi(w0[u] >> 8),
-                                       dq_hi(w1[u] >> 8), qb[grp][2 * u + 1][0], qb[grp][2 * u + 1][1]);
+                    const uint32_t l0 = w0[u] & 0x0F0F0F0Fu, h0 = (w0[u] >> 4) & 0x0F0F0F0Fu;
+                    const uint32_t l1 = w1[u] & 0x0F0F0F0Fu, h1 = (w1[u] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                    for (int j = 0; j < 3; ++j)
+                        ptx::mma_u8s8(acc[j], l0, l1, h0, h1, qb[grp][u][j][0], qb[grp][u][j][1]);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // |acc[2]| <= 33 * 15 * 128 < 2^22: to float by the 1.5 * 2^23
+                    // bias; 256 acc[1] + acc[0] fits int32 exactly
+                    const float hi = __int_as_float(acc[2][e] + 0x4B400000) - 12582912.0f;
+                    S[grp][e] = fmaf(hi, 65536.0f, (float)(acc[1][e] * 256 + acc[0][e]));
                 }
             }
             float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
@@ -296,12 +327,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) attn_kernel(const AttnParams p
             for (int grp = 0; grp < NG; ++grp) {
                 const uint32_t pk0 = *reinterpret_cast<const uint32_t*>(sb + Gm::KP + (r0 * NG + grp) * 4);
                 const uint32_t pk1 = *reinterpret_cast<const uint32_t*>(sb + Gm::KP + (r1 * NG + grp) * 4);
-                const float sk0 = f16lo(pk0), wk0 = fmaf(8.f, sk0, f16hi(pk0));
-                const float sk1 = f16lo(pk1), wk1 = fmaf(8.f, sk1, f16hi(pk1));
-                s00 = fmaf(acc[grp][0], sk0 * ch[0], fmaf(wk0, dh[0][grp], s00));
-                s01 = fmaf(acc[grp][1], sk0 * ch[1], fmaf(wk0, dh[1][grp], s01));
-                s10 = fmaf(acc[grp][2], sk1 * ch[0], fmaf(wk1, dh[0][grp], s10));
-                s11 = fmaf(acc[grp][3], sk1 * ch[1], fmaf(wk1, dh[1][grp], s11));
+                // score = s sum q c + z sum q (K = s c + z), in log2 units
+                const float sk0 = f16lo(pk0), zk0 = f16hi(pk0);
+                const float sk1 = f16lo(pk1), zk1 = f16hi(pk1);
+                s00 = fmaf(S[grp][0], sk0 * ch[0], fmaf(zk0, dh[0][grp], s00));
+                s01 = fmaf(S[grp][1], sk0 * ch[1], fmaf(zk0, dh[1][grp], s01));
+                s10 = fmaf(S[grp][2], sk1 * ch[0], fmaf(zk1, dh[0][grp], s10));
+                s11 = fmaf(S[grp][3], sk1 * ch[1], fmaf(zk1, dh[1][grp], s11));
                 const uint32_t pv0 = *reinterpret_cast<const uint32_t*>(sb + Gm::VP + (r0 * NG + grp) * 4);
                 const uint32_t pv1 = *reinterpret_cast<const uint32_t*>(sb + Gm::VP + (r1 * NG + grp) * 4);
                 // tokens past the end: weight 0 and no V parameters (their bytes
