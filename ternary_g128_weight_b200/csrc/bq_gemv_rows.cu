@@ -1046,19 +1046,24 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
     float* inv = reinterpret_cast<float*>(smem + p.lut_off + 192);
     if (tid < BP) rmax[tid] = 0u;
     bar_compute<NW>();
-    // largest |x| of every batch row (FP32 bits of the magnitude: monotonic)
+    // largest |x| of every batch row (FP32 bits of the magnitude: monotonic):
+    // one warp per row, its loads unrolled so that they are in flight together
+    // (a loop over the rows with all threads on one row waited one L2 round
+    // trip per row)
     const int64_t c8 = p.k / 8;
-    for (int b = 0; b < p.batch; ++b) {
+    for (int b = tid >> 5; b < p.batch; b += NW) {
         uint32_t m = 0u;
-        for (int64_t c = tid; c < c8; c += NW * 32) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + b * p.k) + c);
+        const uint4* row = reinterpret_cast<const uint4*>(p.x + b * p.k);
+#pragma unroll 16
+        for (int64_t c = tid & 31; c < c8; c += 32) {
+            const uint4 v = __ldg(row + c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) m = max(m, max((w[q] << 16) & 0x7FFFFFFFu, w[q] & 0x7FFF0000u));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if ((tid & 31) == 0) atomicMax(&rmax[b], m);
+        if ((tid & 31) == 0) rmax[b] = m;
     }
     bar_compute<NW>();
     if (tid < BP) {
@@ -1072,6 +1077,7 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
     // (stage, group, batch row, thread t): 32 activations -> 16 FP16 pairs
     uint8_t* xres = smem + p.x_off;
     const int tasks = p.stages * kGroupsPerStage * BP * 4;
+#pragma unroll 2
     for (int i = tid; i < tasks; i += NW * 32) {
         const int t = i & 3, b = (i >> 2) % BP, rest = i / (4 * BP), G = rest & 7, st = rest >> 3;
         uint32_t words[16];
