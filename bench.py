@@ -56,9 +56,10 @@ def parse():
                    help="one bq_gemv per product (calls) or one bq_gemv_chain per layer (chain)")
     p.add_argument("--gemm-only", action="store_true",
                    help="run only the prefill GEMM leg (a diagnostic line, e.g. for a profiler)")
-    p.add_argument("--case", choices=["gemv", "kv4"], default=None,
+    p.add_argument("--case", choices=["gemv", "gemm", "kv4"], default=None,
                    help="profiler case: each launch once to warm up, then once after an L2 flush, and exit "
-                        "(gemv: --fmt, --batch, --shapes; kv4: --batch, --ctx)")
+                        "(gemv: --fmt, --batch, --shapes; gemm: --fmt, --shapes, --tokens; kv4: --batch, --ctx)")
+    p.add_argument("--tokens", type=int, default=4096, help="tokens T for --case gemm")
     p.add_argument("--shapes", default="6144x4096,4096x4096,24576x4096,4096x12288,151936x4096",
                    help="NxK list for --case gemv (default: one Qwen3-8B layer's launches and the LM head)")
     p.add_argument("--ctx", type=int, default=65536, help="context tokens for --case kv4")
@@ -86,6 +87,17 @@ def run_case(args):
             ws = torch.empty(max(bq.bq_gemv_workspace_bytes(f, n, k, args.batch), 256), dtype=torch.uint8, device=dev)
             calls.append(lambda f=f, c=codes, s=scales, n=n, k=k, x=x, y=y, ws=ws:
                          bq.bq_gemv(f, c, s, n, k, x, y=y, workspace=ws))
+    elif args.case == "gemm":
+        f = FMT_NAMES[args.fmt]
+        for sh in args.shapes.split(","):
+            n, k = (int(v) for v in sh.split("x"))
+            codes, scales = make_weights(f, n, k, gen, dev, False)
+            x = synth.device_x_bf16(gen, args.tokens, k, device=dev)
+            y = torch.empty((args.tokens, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(max(bq.bq_gemm_workspace_bytes(f, n, k, args.tokens), 256), dtype=torch.uint8,
+                             device=dev)
+            calls.append(lambda f=f, c=codes, s=scales, n=n, k=k, x=x, y=y, ws=ws:
+                         bq.bq_gemm(f, c, s, n, k, x, y=y, workspace=ws))
     else:
         A = synth.QWEN3_8B_ATTN
         B, ctx, hq, hkv, d = args.batch, args.ctx, A["hq"], A["hkv"], A["d"]
