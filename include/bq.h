@@ -274,7 +274,9 @@ int bq_gemm_launches(int fmt, int64_t n, int64_t k, int64_t t);
  * power-of-two pre-scale (exact for every BF16 value within 2^-31 of the
  * token's largest magnitude), accumulating in FP32.
  * X BF16 [T][K] 16-byte aligned; Y BF16 [T][N] 16-byte aligned; workspace as
- * bq_gemm_workspace_bytes, 256-byte aligned.  Asynchronous on `stream`. */
+ * bq_gemm_workspace_bytes, 256-byte aligned (FP16 activations and, where K is
+ * split over CTAs, FP32 partial tiles, rewritten by every call: calls that
+ * share a workspace must not overlap on the GPU).  Asynchronous on `stream`. */
 bq_status bq_gemm(int fmt, const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k,
                   const uint16_t* x, int64_t t, uint16_t* y,
                   void* workspace, size_t workspace_bytes, void* stream);

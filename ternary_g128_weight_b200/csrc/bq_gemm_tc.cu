@@ -24,15 +24,17 @@
 // swizzle row of FP16).  When the row tiles alone cannot fill the GPU, each
 // tile's K range is split over several CTAs and a second kernel adds the FP32
 // partial tiles in a fixed order.
-//   warps 0-7  : dequantise the tile's 128 weight rows into the stage's A
-//                buffer (K-major, 128-byte swizzle, the UMMA canonical
-//                layout), two sets of four warps on alternate stages, packed
-//                codes fetched four of their stages ahead;
-//   warp 8     : TMA loads of the FP16 activation tile (same layout) into B;
-//   warp 9     : allocates TMEM (2 x 256 columns) and issues
+//   dequant warps (8 binary, 12 ternary): dequantise the tile's 128 weight
+//                rows into the stage's A buffer (K-major, 128-byte swizzle,
+//                the UMMA canonical layout), two or three sets of four warps
+//                taking the stages in turn, packed codes fetched four of
+//                their stages ahead;
+//   next warp  : TMA loads of the FP16 activation tile (same layout) into B;
+//   next warp  : allocates TMEM (2 x 256 columns) and issues
 //                tcgen05.mma.kind::f16 (M = 128, N = tile_n, K = 16);
-//   warps 10-13: epilogue: TMEM -> registers -> Y (or the partial tile), while
-//                the MMAs of the next work unit accumulate in the other buffer.
+//   last 4     : epilogue: TMEM -> registers -> Y (or the partial tile), while
+//                the MMAs of the next work unit accumulate in the other buffer
+//                (warp w reads TMEM lane quadrant w % 4).
 // Work units are taken token-tile-major so that the activation tile in flight
 // and the packed weights stay resident in L2.
 #include <cuda.h>
@@ -50,10 +52,19 @@ constexpr int kStages = 4;
 constexpr int kABytes = kTileM * kStageK * 2;     // 16 KB
 constexpr int kBBytes = kMaxTileN * kStageK * 2;  // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-// two sets of 4 dequant warps take alternate stages
-constexpr int kDequantSetWarps = 4, kDequantSets = 2, kDequantWarps = kDequantSets * kDequantSetWarps;
-constexpr int kTmaWarp = kDequantWarps, kMmaWarp = kTmaWarp + 1, kEpiWarp0 = kMmaWarp + 1, kEpiWarps = 4;
-constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+// Sets of 4 dequant warps take the stages in turn: two for the binary
+// format, three for the ternary formats, whose decode costs more instructions
+// per weight (measured on B200 at T = 4096: the third set took the 5-trit
+// GEMM from 0.44 to 0.47 of the BF16 peak on 17408 x 5120 and the 2-bit one
+// from 0.59 to 0.60, while it slowed the binary one).
+constexpr int kDequantSetWarps = 4, kEpiWarps = 4;
+template <int FMT>
+struct Roles {
+    static constexpr int kSets = FMT == BQ_Q1G128 ? 2 : 3;
+    static constexpr int kDequantWarps = kSets * kDequantSetWarps;
+    static constexpr int kTmaWarp = kDequantWarps, kMmaWarp = kTmaWarp + 1, kEpiWarp0 = kMmaWarp + 1;
+    static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+};
 constexpr int kTmemCols = 2 * kMaxTileN;
 constexpr int kBarriers = 3 * kStages + 4;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kBarriers * 8 + 16;
@@ -280,8 +291,10 @@ __device__ __forceinline__ Unit unit_of(const Params& p, int64_t mb_count, int s
 
 // ----------------------------------------------------------------- main
 template <int FMT>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                                                              const Params p) {
+__global__ void __launch_bounds__(Roles<FMT>::kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                                         const Params p) {
+    constexpr int kDequantSets = Roles<FMT>::kSets, kDequantWarps = Roles<FMT>::kDequantWarps;
+    constexpr int kTmaWarp = Roles<FMT>::kTmaWarp, kMmaWarp = Roles<FMT>::kMmaWarp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = ptx::align_smem<1024>(smem_raw);
     uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
@@ -585,7 +598,7 @@ cudaError_t launch_typed(Params prm, const Plan& pl, const uint16_t* x, uint16_t
     cudaError_t e = cudaLaunchKernelEx(&cfg, xprep_f16_kernel<FMT>, x, (int64_t)prm.k, xh, inv_scale);
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)pl.grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(Roles<FMT>::kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<FMT>, tm_x, prm);
     if (e != cudaSuccess) return e;

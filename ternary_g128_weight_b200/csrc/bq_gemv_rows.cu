@@ -752,6 +752,22 @@ __device__ __forceinline__ void prep_x(const Params& p, uint8_t* smem, int warp,
     }
 }
 
+// One chunk of ct row tiles, by its compiled shape (only the shapes up to CAP
+// are compiled in).
+template <int FMT, int NT, int LANES, int NW, int CAP>
+__device__ __forceinline__ bool chunk_by_size(int ct, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                                              int r, Ring& rp, int warp, int lane) {
+    if constexpr (CAP >= 16 && mct<FMT, NT>() >= 16) {
+        if (ct == 16) return run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
+    }
+    if constexpr (CAP >= 8) {
+        if (ct == 8) return run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
+        if (ct == 4) return run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
+    }
+    if (ct == 2) return run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
+    return run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+}
+
 // Compute warps: every chunk of row tiles [rt0, rt1) (pair tiles for a SwiGLU
 // step, whose chunks hold c gate and c up tiles and end with the SwiGLU
 // epilogue).  CAP: the largest chunk the launch uses; only the chunk shapes up
@@ -765,28 +781,7 @@ __device__ __forceinline__ bool run_chunks(const Params& p, uint8_t* smem, uint6
     for (int r = rt0; r < rt1;) {
         const int c = chunk_tiles(rt1 - r, cap);
         const int ct = p.pair_tiles > 0 ? 2 * c : c;
-        bool ok;
-        if constexpr (CAP >= 16 && mct<FMT, NT>() >= 16) {
-            if (ct == 16) {
-                ok = run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
-                goto done;
-            }
-        }
-        if constexpr (CAP >= 8) {
-            if (ct == 8) {
-                ok = run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
-                goto done;
-            }
-            if (ct == 4) {
-                ok = run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
-                goto done;
-            }
-        }
-        if (ct == 2)
-            ok = run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
-        else
-            ok = run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
-    done:
+        const bool ok = chunk_by_size<FMT, NT, LANES, NW, CAP>(ct, p, smem, full, empty, r, rp, warp, lane);
         if (!ok) return false;
         if (p.pair_tiles > 0) {
             // act = BF16(silu(gate) * up) of the chunk's c pair tiles
@@ -1282,7 +1277,7 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
     return alive;
 }
 
-template <int FMT, int NTW>
+template <int FMT, int NTW, int CAP>
 __global__ void __launch_bounds__(threads_of<16>(), 1)
     gemv_wide_kernel(const __grid_constant__ Maps tm, const Params p) {
     constexpr int NW = 16;
@@ -1328,11 +1323,16 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
     for (int r = rt0; r < rt1;) {
         const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
         bool ok;
-        if (ct == 8)
-            ok = run_chunk_wide<FMT, NTW, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
-        else if (ct == 4)
-            ok = run_chunk_wide<FMT, NTW, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
-        else if (ct == 2)
+        if constexpr (CAP >= 8) {
+            if (ct == 8 || ct == 4) {
+                ok = ct == 8 ? run_chunk_wide<FMT, NTW, NW, 8>(p, smem, full, empty, r, rp, warp, lane)
+                             : run_chunk_wide<FMT, NTW, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
+                if (!ok) break;
+                r += ct;
+                continue;
+            }
+        }
+        if (ct == 2)
             ok = run_chunk_wide<FMT, NTW, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
         else
             ok = run_chunk_wide<FMT, NTW, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
@@ -1556,12 +1556,12 @@ bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
     return true;
 }
 
-template <int FMT, int NTW>
+template <int FMT, int NTW, int CAP>
 cudaError_t launch_wide_typed(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
                               int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
     {
         const cudaError_t e =
-            ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_wide_kernel<FMT, NTW>), kSmemFull);
+            ensure_dynamic_smem(reinterpret_cast<const void*>(gemv_wide_kernel<FMT, NTW, CAP>), kSmemFull);
         if (e != cudaSuccess) return e;
     }
     Maps tm;
@@ -1600,9 +1600,21 @@ cudaError_t launch_wide_typed(const uint8_t* codes, const uint16_t* scales, int6
     cfg.stream = s;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_wide_kernel<FMT, NTW>, tm, prm);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_wide_kernel<FMT, NTW, CAP>, tm, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// The kernel is built per largest chunk (2: chunks of 2 and 1 tiles; 8: every
+// chunk shape), as the row-owning kernel is.
+template <int FMT>
+cudaError_t launch_wide_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
+                            int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
+    if (pl.chunk_cap <= 2)
+        return pl.nt == 1 ? launch_wide_typed<FMT, 1, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
+                          : launch_wide_typed<FMT, 2, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return pl.nt == 1 ? launch_wide_typed<FMT, 1, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
+                      : launch_wide_typed<FMT, 2, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 }  // namespace rows
@@ -1617,10 +1629,8 @@ cudaError_t launch_gemv_wide(int fmt, const uint8_t* codes, const uint16_t* scal
     rows::Plan pl;
     if (!rows::wide_plan(pl, fmt, n, k, batch)) return cudaErrorInvalidValue;
     if (fmt == BQ_Q1G128)
-        return pl.nt == 1 ? rows::launch_wide_typed<BQ_Q1G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
-                          : rows::launch_wide_typed<BQ_Q1G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    return pl.nt == 1 ? rows::launch_wide_typed<BQ_T2G128, 1>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
-                      : rows::launch_wide_typed<BQ_T2G128, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+        return rows::launch_wide_fmt<BQ_Q1G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return rows::launch_wide_fmt<BQ_T2G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 
