@@ -220,14 +220,18 @@ __device__ __forceinline__ uint32_t ternary_pair(uint32_t c2, uint32_t ss) {
 __device__ __forceinline__ uint32_t div3x2(uint32_t v) { return ((v * 171u) >> 9) & 0x007F007Fu; }
 
 // Five base-3 digits of the two bytes in the halves of v -> pairs h[0..4].
+// The quotients floor(v / 3^i) come from independent multiply-shifts (171 >> 9,
+// 57 >> 9, 19 >> 9, 203 >> 14: exact for every v < 256, and v * m < 2^16, so
+// the halves do not interfere once the bits above each quotient are masked),
+// and digit i is q_i - 3 q_(i+1); no step waits on the one before.
 __device__ __forceinline__ void t5p8_digits(uint32_t v, uint32_t ss, uint32_t* h) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const uint32_t q = div3x2(v);
-        h[e] = ternary_pair(v - 3u * q, ss);
-        v = q;
-    }
-    h[4] = ternary_pair(v, ss);
+    const uint32_t q1 = ((v * 171u) >> 9) & 0x007F007Fu, q2 = ((v * 57u) >> 9) & 0x007F007Fu;
+    const uint32_t q3 = ((v * 19u) >> 9) & 0x007F007Fu, q4 = ((v * 203u) >> 14) & 0x00030003u;
+    h[0] = ternary_pair(v - 3u * q1, ss);
+    h[1] = ternary_pair(q1 - 3u * q2, ss);
+    h[2] = ternary_pair(q2 - 3u * q3, ss);
+    h[3] = ternary_pair(q3 - 3u * q4, ss);
+    h[4] = ternary_pair(q4, ss);
 }
 
 __device__ __forceinline__ uint32_t byte_of(const uint32_t (&w)[4], int i) { return (w[i >> 2] >> (8 * (i & 3))) & 0xFFu; }
@@ -366,6 +370,36 @@ __global__ void __launch_bounds__(Roles<FMT>::kThreads, 1) gemm_tc_kernel(const 
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) pipe[i] = next_chunk();
         bool alive = true;
+        if constexpr (FMT == BQ_T5P8G128) {
+            // the base-3 decode is long: one copy of it in a loop that shifts
+            // the ring of chunks by one entry per stage (the unrolled form below
+            // keeps kAhead copies; for this format the instruction fetch of
+            // those copies measurably stalled the dequant warps)
+#pragma unroll 1
+            for (int64_t j = 0; j < mine; ++j) {
+                const int64_t it = j * kDequantSets + set;  // stage index of the CTA's sequence
+                const int slot = (int)(it % kStages);
+                if (it >= kStages &&
+                    !ptx::mbar_wait_bounded(&empty[slot], (uint32_t)(((it / kStages) - 1) & 1), kWaitPolls)) {
+                    record_status(p.status, BQ_ERR_TIMEOUT);
+                    break;
+                }
+                uint32_t h[32];
+                dequant_chunk<FMT>(pipe[0], h);
+#pragma unroll
+                for (int i = 0; i + 1 < kAhead; ++i) pipe[i] = pipe[i + 1];
+                pipe[kAhead - 1] = next_chunk();
+                uint8_t* a = smem + slot * kStageBytes + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(a + ((c ^ (r & 7)) << 4)) =
+                        make_uint4(h[4 * c], h[4 * c + 1], h[4 * c + 2], h[4 * c + 3]);
+                ptx::fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&full_a[slot]);
+            }
+            alive = false;  // (the loop below is for the other formats)
+        }
         // unrolled by kAhead so that each ring entry is a fixed set of registers:
         // a chunk is consumed kAhead stages after its load was issued
         for (int64_t base = 0; base < mine && alive; base += kAhead) {
