@@ -504,10 +504,32 @@ def cpu_baseline(fmt, mats, batch):
             total_bytes += c.nbytes + s.nbytes
         passes += 1
     dt = time.perf_counter() - t0
+    # the same oracle on one core: the first layer's o matrix, about 3 s
+    n1, k1, c1, s1, x1 = host[2]
+    one_bytes, one_passes, t1 = 0, 0, time.perf_counter()
+    while one_passes < 200 and (one_passes == 0 or time.perf_counter() - t1 < 3.0):
+        oracle.matmul(fmt, c1, s1, n1, k1, x1, nthreads=1)
+        one_bytes += c1.nbytes + s1.nbytes
+        one_passes += 1
+    dt1 = time.perf_counter() - t1
     return {"value": round(total_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"LM head + one layer's q|k|v, o, gate|up, down ({fmt}, batch {batch}) x {passes} passes, "
-                      f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s"}
+                      f"{total_bytes / 1e6:.1f} MB of weights, {dt:.1f} s",
+            "single_core": {"value": round(one_bytes / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"o {n1}x{k1} x {one_passes} passes, {dt1:.1f} s"}}
+
+
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 # ------------------------------------------------------------ ranks (host side)
