@@ -152,6 +152,12 @@ __device__ __forceinline__ int chunk_tiles(int remaining, int cap) {
     return c >= 16 ? 16 : c >= 8 ? 8 : c >= 4 ? 4 : c >= 2 ? 2 : 1;
 }
 
+// Row-owning kernel: a chunk takes as many of the remaining tiles as the cap
+// allows (any count); it runs in the compiled shape of the next power of two,
+// the tiles past its count idle (one pass over K for, e.g., three tiles instead
+// of a pass for two and one for one).
+__device__ __forceinline__ int chunk_count(int remaining, int cap) { return remaining < cap ? remaining : cap; }
+
 // Bytes of the resident activation operand per (stage, n-tile): B fragments
 // [8 groups][2 MMA pairs][LANES][16 B] then the table [8 groups][4][float4].
 __host__ __device__ constexpr int x_nt_bytes(int lanes) { return kGroupsPerStage * 2 * lanes * 16 + kGroupsPerStage * 4 * 16; }
@@ -392,7 +398,7 @@ __device__ __forceinline__ float scale_of(const uint32_t* s, int i) {
 //             going) and the GPW = 8 / WPR groups G = GPW (w % WPR) + i.
 template <int FMT, int NT, int LANES, int NW, int CT>
 __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, Ring& rp,
-                          int warp, int lane) {
+                          int warp, int lane, int ct) {
     constexpr int TPW = CT >= NW ? CT / NW : 1;
     constexpr int WPR = CT >= NW ? 1 : ((NW / CT) < kGroupsPerStage ? (NW / CT) : kGroupsPerStage);
     constexpr int GPW = kGroupsPerStage / WPR;  // groups per warp and stage
@@ -401,7 +407,10 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
     constexpr int X_NT = x_nt_bytes(LANES);
     const int my_rt = CT >= NW ? warp : warp / WPR;
     const int gsub = CT >= NW ? 0 : warp % WPR;
-    const bool active = my_rt < CT;
+    // the chunk holds ct <= CT tiles; a warp whose tiles are all past ct idles
+    // (with several tiles per warp, the ones past ct are computed on stale
+    // slot contents and never stored)
+    const bool active = my_rt < ct;
     const int g = lane >> 2, t = lane & 3;
     // at batch 1 the upper 16 lanes (columns of a second batch row) read the
     // lower lanes' fragments: their sums are never stored
@@ -600,7 +609,8 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int r = 0; r < 2; ++r)
-                    stg[((my_rt + NW * tp) * 16 + g + 8 * r) * 8 + nt * 2 + (t >> 1)] = yacc[tp][nt][r];
+                    if (my_rt + NW * tp < ct)
+                        stg[((my_rt + NW * tp) * 16 + g + 8 * r) * 8 + nt * 2 + (t >> 1)] = yacc[tp][nt][r];
     } else if (active && gsub == 0 && (t & 1) == 0) {
 #pragma unroll
         for (int tp = 0; tp < TPW; ++tp)
@@ -610,7 +620,7 @@ __device__ bool run_chunk(const Params& p, uint8_t* smem, uint64_t* full, uint64
                 for (int r = 0; r < 2; ++r) {
                     const int bb = nt * 2 + (t >> 1);
                     const int64_t row = (int64_t)(rt + my_rt + NW * tp) * 16 + g + 8 * r;
-                    if (bb < p.batch && row < p.n) {
+                    if (bb < p.batch && row < p.n && my_rt + NW * tp < ct) {
                         if (p.y_dtype == BQ_F32)
                             static_cast<float*>(p.y)[bb * p.n + row] = yacc[tp][nt][r];
                         else
@@ -647,8 +657,9 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
     constexpr int TCB = tile_code_bytes<FMT>();
     constexpr int KB = Fmt<FMT>::kBoxes;
     uint8_t* sb = smem + slot * p.slot_bytes;
-    const bool box128 = FMT == BQ_T5P8G128 ? (ct == kMaxChunkTiles && p.pair_tiles == 0)
-                                           : (ct >= kMaxChunkTiles && (p.pair_tiles == 0 || ct >= 2 * kMaxChunkTiles));
+    const bool box128 = FMT == BQ_T5P8G128
+                            ? (ct == kMaxChunkTiles && p.pair_tiles == 0)
+                            : (ct % kMaxChunkTiles == 0 && (p.pair_tiles == 0 || ct >= 2 * kMaxChunkTiles));
     if (FMT == BQ_T5P8G128) {
         if (box128) {
             if (lane == 0) ptx::tma_load_2d(sb, &tm.codes128, st * kT5RowBytes, r * 16, &full[slot]);
@@ -687,13 +698,15 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
 // a SwiGLU step), chunk by chunk and stage by stage, through the ring.  rp and
 // it (copies issued) carry over from one call to the next.  False if a slot
 // wait timed out.
-template <int FMT>
+template <int FMT, bool POW2>
 __device__ __forceinline__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0,
                         int rt1, Ring& rp, int& it, int lane) {
     constexpr int TCB = tile_code_bytes<FMT>();
     const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
     for (int r = rt0; r < rt1;) {
-        const int c = chunk_tiles(rt1 - r, cap);
+        // the same chunks as the consumer: power-of-two chunks for the
+        // wide-batch kernel, any count for the row-owning and chain kernels
+        const int c = POW2 ? chunk_tiles(rt1 - r, cap) : chunk_count(rt1 - r, cap);
         const int ct = p.pair_tiles > 0 ? 2 * c : c;
         for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
             const int slot = rp.slot;
@@ -752,20 +765,22 @@ __device__ __forceinline__ void prep_x(const Params& p, uint8_t* smem, int warp,
     }
 }
 
-// One chunk of ct row tiles, by its compiled shape (only the shapes up to CAP
-// are compiled in).
+// One chunk of ct row tiles in the compiled shape of the next power of two
+// (only the shapes up to CAP are compiled in).
 template <int FMT, int NT, int LANES, int NW, int CAP>
 __device__ __forceinline__ bool chunk_by_size(int ct, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty,
                                               int r, Ring& rp, int warp, int lane) {
     if constexpr (CAP >= 16 && mct<FMT, NT>() >= 16) {
-        if (ct == 16) return run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane);
+        if (ct > 8) return run_chunk<FMT, NT, LANES, NW, mct<FMT, NT>()>(p, smem, full, empty, r, rp, warp, lane, ct);
     }
     if constexpr (CAP >= 8) {
-        if (ct == 8) return run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane);
-        if (ct == 4) return run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
+        if (ct > 4) return run_chunk<FMT, NT, LANES, NW, 8>(p, smem, full, empty, r, rp, warp, lane, ct);
     }
-    if (ct == 2) return run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
-    return run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+    if constexpr (CAP >= 4) {
+        if (ct > 2) return run_chunk<FMT, NT, LANES, NW, 4>(p, smem, full, empty, r, rp, warp, lane, ct);
+    }
+    if (ct == 2) return run_chunk<FMT, NT, LANES, NW, 2>(p, smem, full, empty, r, rp, warp, lane, ct);
+    return run_chunk<FMT, NT, LANES, NW, 1>(p, smem, full, empty, r, rp, warp, lane, ct);
 }
 
 // Compute warps: every chunk of row tiles [rt0, rt1) (pair tiles for a SwiGLU
@@ -779,7 +794,7 @@ __device__ __forceinline__ bool run_chunks(const Params& p, uint8_t* smem, uint6
                            Ring& rp, int warp, int lane) {
     const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
     for (int r = rt0; r < rt1;) {
-        const int c = chunk_tiles(rt1 - r, cap);
+        const int c = chunk_count(rt1 - r, cap);
         const int ct = p.pair_tiles > 0 ? 2 * c : c;
         const bool ok = chunk_by_size<FMT, NT, LANES, NW, CAP>(ct, p, smem, full, empty, r, rp, warp, lane);
         if (!ok) return false;
@@ -841,7 +856,7 @@ __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
         int it = 0;
         Ring rp;
         rp.depth = p.slots;
-        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
+        produce<FMT, false>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
         // every copy this CTA issued must land before it may exit
         if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
@@ -971,7 +986,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
             const Params& p = cp.step[s];
             const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
             const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
-            if (!produce<FMT>(tm.m[s], p, smem, full, empty, rt0, rt1, rp, it, lane)) break;
+            if (!produce<FMT, false>(tm.m[s], p, smem, full, empty, rt0, rt1, rp, it, lane)) break;
         }
         if (lane == 0)
             for (int j = (it > p0.slots ? it - p0.slots : 0); j < it; ++j)
@@ -1308,7 +1323,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
         int it = 0;
         Ring rp;
         rp.depth = p.slots;
-        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
+        produce<FMT, true>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
         if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
                 if (!ptx::mbar_wait_bounded(&full[j % p.slots], (uint32_t)((j / p.slots) & 1), kWaitPolls))
@@ -1357,24 +1372,33 @@ bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
     pl.nw = nw;
     pl.grid = pl.row_tiles < cap_grid ? pl.row_tiles : cap_grid;
     // 16-tile chunks (binary, batch <= 4) only where a CTA owns at least 16
-    // row tiles; otherwise 8-tile slots keep the ring deep.  No chunk is larger
-    // than the most tiles a CTA owns (rounded down to a power of two), so
-    // slots are sized for that; a slot is a multiple of 1 KB (the swizzled
-    // copies land on 1 KB boundaries).
+    // row tiles; otherwise 8-tile slots keep the ring deep.  A chunk is the
+    // smallest power of two that holds the most tiles a CTA owns (e.g. 3 tiles
+    // run as one 4-tile chunk with one tile idle), or, where that leaves the
+    // ring fewer than two slots, the largest power of two within those tiles; a
+    // slot is a multiple of 1 KB (the swizzled copies land on 1 KB boundaries).
     const int64_t tsb = kTileScaleBytes * (fmt == BQ_A1G128 ? 2 : 1);
     const bool bits = fmt == BQ_Q1G128 || fmt == BQ_A1G128;
     const int64_t tile_bytes = (bits ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + tsb;
-    pl.chunk_cap = (bits && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
+    const int top = (bits && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
     const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
-    while (pl.chunk_cap > 1 && pl.chunk_cap > most) pl.chunk_cap >>= 1;
-    const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
-    pl.slot_bytes = (int)slot;
-    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - tsb);
+    int within = top;  // largest power of two <= most
+    while (within > 1 && within > most) within >>= 1;
+    pl.chunk_cap = top;  // smallest power of two >= most
+    while (pl.chunk_cap > 1 && pl.chunk_cap / 2 >= most) pl.chunk_cap >>= 1;
     const int64_t lut = fmt == BQ_T5P8G128 ? kLutBytes : 0;
     const int64_t x_area = ((int64_t)pl.stages * pl.nt * x_nt_bytes(pl.lanes) + 1023) / 1024 * 1024;
     const int64_t red = (int64_t)nw * 32 * pl.nt * 2 * 4;
     const int64_t fixed = 1024 + x_area + red + lut + 2 * kMaxSlots * 8;
-    int64_t slots = (limit - fixed) / slot;
+    int64_t slot = 0, slots = 0;
+    for (;;) {
+        slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+        slots = (limit - fixed) / slot;
+        if (slots >= 2 || pl.chunk_cap == within) break;
+        pl.chunk_cap = within;
+    }
+    pl.slot_bytes = (int)slot;
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - tsb);
     if (slots > kMaxSlots) slots = kMaxSlots;
     if (slots < 2) return false;
     pl.slots = (int)slots;
@@ -1502,12 +1526,13 @@ cudaError_t launch_cap(const uint8_t* codes, const uint16_t* scales, int64_t n, 
     return launch_typed<FMT, 4, 32, 16, CAP>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
-// The kernel is built per largest chunk: 2 (chunks of 2 and 1 tiles), 8
-// (8, 4, 2, 1) or 16 (every chunk shape).
+// The kernel is built per largest chunk: 2 (chunks of 2 and 1 tiles), 4 (4, 2,
+// 1), 8 (8, 4, 2, 1) or 16 (every chunk shape).
 template <int FMT>
 cudaError_t launch_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
                        int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
     if (pl.chunk_cap <= 2) return launch_cap<FMT, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.chunk_cap <= 4) return launch_cap<FMT, 4>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     if (pl.chunk_cap <= 8) return launch_cap<FMT, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     return launch_cap<FMT, 16>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
