@@ -147,15 +147,10 @@ struct Ring {
 template <int NW>
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory"); }
 
-__device__ __forceinline__ int chunk_tiles(int remaining, int cap) {
-    const int c = remaining < cap ? remaining : cap;
-    return c >= 16 ? 16 : c >= 8 ? 8 : c >= 4 ? 4 : c >= 2 ? 2 : 1;
-}
-
-// Row-owning kernel: a chunk takes as many of the remaining tiles as the cap
-// allows (any count); it runs in the compiled shape of the next power of two,
-// the tiles past its count idle (one pass over K for, e.g., three tiles instead
-// of a pass for two and one for one).
+// A chunk takes as many of the remaining tiles as the cap allows (any count);
+// it runs in the compiled shape of the next power of two, the tiles past its
+// count idle (one pass over K for, e.g., three tiles instead of a pass for two
+// and one for one).
 __device__ __forceinline__ int chunk_count(int remaining, int cap) { return remaining < cap ? remaining : cap; }
 
 // Bytes of the resident activation operand per (stage, n-tile): B fragments
@@ -698,15 +693,13 @@ __device__ __forceinline__ void issue_stage(const Maps& tm, const Params& p, uin
 // a SwiGLU step), chunk by chunk and stage by stage, through the ring.  rp and
 // it (copies issued) carry over from one call to the next.  False if a slot
 // wait timed out.
-template <int FMT, bool POW2>
+template <int FMT>
 __device__ __forceinline__ bool produce(const Maps& tm, const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt0,
                         int rt1, Ring& rp, int& it, int lane) {
     constexpr int TCB = tile_code_bytes<FMT>();
     const int cap = p.pair_tiles > 0 ? p.chunk_cap / 2 : p.chunk_cap;
     for (int r = rt0; r < rt1;) {
-        // the same chunks as the consumer: power-of-two chunks for the
-        // wide-batch kernel, any count for the row-owning and chain kernels
-        const int c = POW2 ? chunk_tiles(rt1 - r, cap) : chunk_count(rt1 - r, cap);
+        const int c = chunk_count(rt1 - r, cap);  // the consumer's chunks
         const int ct = p.pair_tiles > 0 ? 2 * c : c;
         for (int st = 0; st < p.stages; ++st, ++it, rp.next()) {
             const int slot = rp.slot;
@@ -856,7 +849,7 @@ __global__ void __launch_bounds__(threads_of<NW>(), NW == 8 ? 2 : 1)
         int it = 0;
         Ring rp;
         rp.depth = p.slots;
-        produce<FMT, false>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
+        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
         // every copy this CTA issued must land before it may exit
         if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
@@ -986,7 +979,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
             const Params& p = cp.step[s];
             const int tq = p.row_tiles / C, trem = p.row_tiles - tq * C;
             const int rt0 = c * tq + min(c, trem), rt1 = rt0 + tq + (c < trem ? 1 : 0);
-            if (!produce<FMT, false>(tm.m[s], p, smem, full, empty, rt0, rt1, rp, it, lane)) break;
+            if (!produce<FMT>(tm.m[s], p, smem, full, empty, rt0, rt1, rp, it, lane)) break;
         }
         if (lane == 0)
             for (int j = (it > p0.slots ? it - p0.slots : 0); j < it; ++j)
@@ -1175,7 +1168,7 @@ __device__ __forceinline__ void wide_a(uint2 w, uint2 wb, uint32_t S, uint32_t S
 // split as run_chunk.
 template <int FMT, int NTW, int NW, int CT>
 __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, uint64_t* empty, int rt, Ring& rp,
-                               int warp, int lane) {
+                               int warp, int lane, int ct) {
     constexpr int TPW = CT >= NW ? CT / NW : 1;
     constexpr int WPR = CT >= NW ? 1 : ((NW / CT) < kGroupsPerStage ? (NW / CT) : kGroupsPerStage);
     constexpr int GPW = kGroupsPerStage / WPR;
@@ -1183,7 +1176,7 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
     constexpr int TSTRIDE = 2048;  // code bytes between row tiles of a column box
     const int my_rt = CT >= NW ? warp : warp / WPR;
     const int gsub = CT >= NW ? 0 : warp % WPR;
-    const bool active = my_rt < CT;
+    const bool active = my_rt < ct;  // (ct <= CT tiles in the chunk; as in run_chunk)
     const int g = lane >> 2, t = lane & 3;
     float acc[TPW][NTW][4];
 #pragma unroll
@@ -1280,7 +1273,7 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
                 for (int c = 0; c < 4; ++c) {
                     const int bb = nt * 8 + 2 * t + (c & 1);
                     const int64_t row = (int64_t)(rt + my_rt + NW * tp) * 16 + g + 8 * (c >> 1);
-                    if (bb < p.batch && row < p.n) {
+                    if (bb < p.batch && row < p.n && my_rt + NW * tp < ct) {
                         const float v = acc[tp][nt][c] * inv[bb];
                         if (p.y_dtype == BQ_F32)
                             static_cast<float*>(p.y)[bb * p.n + row] = v;
@@ -1323,7 +1316,7 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
         int it = 0;
         Ring rp;
         rp.depth = p.slots;
-        produce<FMT, true>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
+        produce<FMT>(tm, p, smem, full, empty, rt0, rt1, rp, it, lane);
         if (lane == 0)
             for (int j = (it > p.slots ? it - p.slots : 0); j < it; ++j)
                 if (!ptx::mbar_wait_bounded(&full[j % p.slots], (uint32_t)((j / p.slots) & 1), kWaitPolls))
@@ -1336,21 +1329,17 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
     Ring rp;
     rp.depth = p.slots;
     for (int r = rt0; r < rt1;) {
-        const int ct = chunk_tiles(rt1 - r, p.chunk_cap);
+        // any tile count, in the compiled shape of the next power of two
+        const int ct = chunk_count(rt1 - r, p.chunk_cap);
         bool ok;
-        if constexpr (CAP >= 8) {
-            if (ct == 8 || ct == 4) {
-                ok = ct == 8 ? run_chunk_wide<FMT, NTW, NW, 8>(p, smem, full, empty, r, rp, warp, lane)
-                             : run_chunk_wide<FMT, NTW, NW, 4>(p, smem, full, empty, r, rp, warp, lane);
-                if (!ok) break;
-                r += ct;
-                continue;
-            }
-        }
-        if (ct == 2)
-            ok = run_chunk_wide<FMT, NTW, NW, 2>(p, smem, full, empty, r, rp, warp, lane);
+        if (CAP >= 8 && ct > 4)
+            ok = run_chunk_wide<FMT, NTW, NW, CAP >= 8 ? 8 : 1>(p, smem, full, empty, r, rp, warp, lane, ct);
+        else if (CAP >= 4 && ct > 2)
+            ok = run_chunk_wide<FMT, NTW, NW, CAP >= 4 ? 4 : 1>(p, smem, full, empty, r, rp, warp, lane, ct);
+        else if (ct == 2)
+            ok = run_chunk_wide<FMT, NTW, NW, 2>(p, smem, full, empty, r, rp, warp, lane, ct);
         else
-            ok = run_chunk_wide<FMT, NTW, NW, 1>(p, smem, full, empty, r, rp, warp, lane);
+            ok = run_chunk_wide<FMT, NTW, NW, 1>(p, smem, full, empty, r, rp, warp, lane, ct);
         if (!ok) break;
         r += ct;
     }
@@ -1559,15 +1548,23 @@ bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
     const int sms = sm_count();
     pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
     const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : 4096) + kTileScaleBytes;
-    pl.chunk_cap = kMaxChunkTiles;
+    // chunks as in the row-owning kernel: the smallest power of two that holds
+    // a CTA's tiles, else (ring of fewer than two slots) the largest within them
     const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
-    while (pl.chunk_cap > 1 && pl.chunk_cap > most) pl.chunk_cap >>= 1;
-    const int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
-    pl.slot_bytes = (int)slot;
-    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
+    int within = kMaxChunkTiles;
+    while (within > 1 && within > most) within >>= 1;
+    pl.chunk_cap = kMaxChunkTiles;
+    while (pl.chunk_cap > 1 && pl.chunk_cap / 2 >= most) pl.chunk_cap >>= 1;
     const int64_t x_area = (int64_t)pl.stages * (pl.nt == 1 ? wide_stage_bytes<1>() : wide_stage_bytes<2>());
     const int64_t red = (int64_t)16 * 32 * pl.nt * 4 * 4;
     const int64_t fixed = 1024 + x_area + red + kWideAux + 2 * kMaxSlots * 8;
+    int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+    if ((kSmemFull - fixed) / slot < 2 && pl.chunk_cap != within) {
+        pl.chunk_cap = within;
+        slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+    }
+    pl.slot_bytes = (int)slot;
+    pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
     int64_t slots = (kSmemFull - fixed) / slot;
     if (slots > kMaxSlots) slots = kMaxSlots;
     if (slots < 2) return false;
@@ -1630,14 +1627,17 @@ cudaError_t launch_wide_typed(const uint8_t* codes, const uint16_t* scales, int6
     return cudaGetLastError();
 }
 
-// The kernel is built per largest chunk (2: chunks of 2 and 1 tiles; 8: every
-// chunk shape), as the row-owning kernel is.
+// The kernel is built per largest chunk (2: chunks of 2 and 1 tiles; 4: 4, 2,
+// 1; 8: every chunk shape), as the row-owning kernel is.
 template <int FMT>
 cudaError_t launch_wide_fmt(const uint8_t* codes, const uint16_t* scales, int64_t n, int64_t k, const uint16_t* x,
                             int batch, void* y, int y_dtype, const Plan& pl, cudaStream_t s) {
     if (pl.chunk_cap <= 2)
         return pl.nt == 1 ? launch_wide_typed<FMT, 1, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
                           : launch_wide_typed<FMT, 2, 2>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (pl.chunk_cap <= 4)
+        return pl.nt == 1 ? launch_wide_typed<FMT, 1, 4>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
+                          : launch_wide_typed<FMT, 2, 4>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
     return pl.nt == 1 ? launch_wide_typed<FMT, 1, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s)
                       : launch_wide_typed<FMT, 2, 8>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
