@@ -1360,8 +1360,9 @@ bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
     const int cap_grid = sms * ctas_per_sm;
     pl.nw = nw;
     pl.grid = pl.row_tiles < cap_grid ? pl.row_tiles : cap_grid;
-    // 16-tile chunks (binary, batch <= 4) only where a CTA owns at least 16
-    // row tiles; otherwise 8-tile slots keep the ring deep.  A chunk is the
+    // 16-tile chunks (binary, batch <= 4) where a CTA owns more than 8 row
+    // tiles (9..15 tiles run as one 16-tile chunk: measured faster than 8 plus
+    // the rest); otherwise 8-tile slots keep the ring deep.  A chunk is the
     // smallest power of two that holds the most tiles a CTA owns (e.g. 3 tiles
     // run as one 4-tile chunk with one tile idle), or, where that leaves the
     // ring fewer than two slots, the largest power of two within those tiles; a
@@ -1369,7 +1370,7 @@ bool layout(Plan& pl, int fmt, int nw, int limit, int sms) {
     const int64_t tsb = kTileScaleBytes * (fmt == BQ_A1G128 ? 2 : 1);
     const bool bits = fmt == BQ_Q1G128 || fmt == BQ_A1G128;
     const int64_t tile_bytes = (bits ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + tsb;
-    const int top = (bits && pl.nt <= 2 && pl.row_tiles / pl.grid >= 16) ? 16 : kMaxChunkTiles;
+    const int top = (bits && pl.nt <= 2 && pl.row_tiles / pl.grid >= 9) ? 16 : kMaxChunkTiles;
     const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
     int within = top;  // largest power of two <= most
     while (within > 1 && within > most) within >>= 1;
