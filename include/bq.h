@@ -164,16 +164,17 @@ int bq_gemv_launches(int fmt, int64_t n, int64_t k, int batch);
  * when that is 0), 256-byte aligned; its contents on entry do not matter.
  * Asynchronous on `stream`.
  * Kernel choice (the same for bq_gemv_noalloc and for bq_gemm with T <= 4):
- * K % 1024 == 0 with binary or 2-bit ternary codes at batch 5..16 runs the
- * wide-batch GEMV (FP16 effective weights +-s / {-s,0,+s} built in registers,
- * x pre-scaled per row to FP16, one launch, no workspace) when its FP16
- * activations (2 K bytes per row, rows padded to 8 or 16) fit in shared
- * memory; batch <= 8 and K % 1024 == 0 otherwise run the row-owning
+ * K % 1024 == 0 with binary or 2-bit ternary codes at batch 5..16, or 5-trit
+ * codes at batch 9..16, runs the wide-batch GEMV (FP16 effective weights
+ * +-s / {-s,0,+s} built in registers, x pre-scaled per row to FP16, one
+ * launch, no workspace) when its FP16 activations (2 K bytes per row, rows
+ * padded to 8 or 16) and a ring of two weight slots fit in shared memory;
+ * batch <= 8 and K % 1024 == 0 otherwise run the row-owning
  * tensor-core GEMV (all three formats, one launch, no workspace) when its
  * activation operand and a ring of at least two weight slots fit in shared
  * memory; otherwise binary and 2-bit ternary at batch <= 4 run the split-K
- * tensor-core GEMV (workspace), and the rest (the 5-trit format at batch
- * 9..16, K % 1024 != 0, operands too large) the tcgen05 GEMM with T = batch
+ * tensor-core GEMV (workspace), and the rest (K % 1024 != 0, operands too
+ * large) the tcgen05 GEMM with T = batch
  * (workspace for the FP16 activations).  A shape
  * no kernel takes (K > 2^28, or N >= 2^31) returns BQ_ERR_SHAPE.
  * bq_gemv_workspace_bytes and bq_gemv_launches report the chosen path (-1 for

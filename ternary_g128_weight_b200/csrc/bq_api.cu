@@ -88,7 +88,9 @@ namespace bq {
 // batch 9..16 (binary 4096 x 4096 batch 16: 15.1 vs 18.8 us; 24576 x 4096:
 // 26.8 vs 62.7 us).
 GemvPath gemv_path(int fmt, int64_t n, int64_t k, int batch) {
-    if (batch >= 5 && gemv_wide_eligible(fmt, n, k, batch)) return GemvPath::Wide;
+    // (the 5-trit format takes it from batch 9, where the alternative is the
+    // GEMM; at batch 5..8 it keeps the row-owning kernel)
+    if (batch >= (fmt == BQ_T5P8G128 ? 9 : 5) && gemv_wide_eligible(fmt, n, k, batch)) return GemvPath::Wide;
     if (gemv_rows_eligible(fmt, n, k, batch)) return GemvPath::Rows;
     if (gemv_tc_eligible(fmt, n, k, batch)) return GemvPath::SplitK;
     if (gemm_tc_eligible(fmt, n, k, batch)) return GemvPath::Gemm;

@@ -1024,7 +1024,8 @@ __global__ void __launch_bounds__(threads_of<16>(), 1)
 }
 
 // ------------------------------------------------------- wide-batch decode
-// Batch 5..16, binary and 2-bit ternary.  The weights become exact FP16
+// Batch 5..16, binary and 2-bit ternary (and 5-trit, whose codes become the
+// same FP16 pairs through base-3 quotient arithmetic).  The weights become exact FP16
 // effective weights s * q inside the A registers of the warp MMA m16n8k16:
 //   binary: ((w << (15 - m)) & 0x80008000) ^ (s | s << 16) ^ 0x80008000 is the
 //           pair (weight m, weight m + 16) of code word w as (+-s, +-s), the
@@ -1045,13 +1046,21 @@ constexpr int kWideAux = 256;  // per batch row: largest |x|, 2^e as two factors
 template <int NTW>
 __host__ __device__ constexpr int wide_stage_bytes() { return kGroupsPerStage * 8 * (NTW * 8) * 4 * 8; }
 
-// The weights (relative to 32 t in the group) of register p (0..15) of a
-// thread's weight row: binary (p, p + 16); 2-bit p < 8: (p, p + 8), else
-// (p + 8, p + 16).
+// The weights of register p (0..15) of a thread's weight row, as indices r
+// into the thread's 32 weights of the group: binary (p, p + 16) and 2-bit
+// p < 8: (p, p + 8), else (p + 8, p + 16), with weight r at k = 32 t + r;
+// 5-trit p < 15: (p, p + 15), digit p % 5 of bytes 6 t + p / 5 and
+// 6 t + p / 5 + 3, and p = 15: (30, 31), the thread's two trits of the group's
+// last eight (weight r < 30 at k = 30 t + r, r = 30, 31 at k = 120 + 2 t + r - 30;
+// the row-owning kernel's split of the 26 bytes).
 template <int FMT>
-__device__ __forceinline__ constexpr int wide_lo(int p) { return FMT == BQ_T2G128 ? (p < 8 ? p : p + 8) : p; }
+__device__ __forceinline__ constexpr int wide_lo(int p) {
+    return FMT == BQ_T2G128 ? (p < 8 ? p : p + 8) : FMT == BQ_T5P8G128 ? (p < 15 ? p : 30) : p;
+}
 template <int FMT>
-__device__ __forceinline__ constexpr int wide_hi(int p) { return FMT == BQ_T2G128 ? (p < 8 ? p + 8 : p + 16) : p + 16; }
+__device__ __forceinline__ constexpr int wide_hi(int p) {
+    return FMT == BQ_T2G128 ? (p < 8 ? p + 8 : p + 16) : FMT == BQ_T5P8G128 ? (p < 15 ? p + 15 : 31) : p + 16;
+}
 
 // x -> the FP16 activation area of all of K, per-row power-of-two pre-scale.
 template <int FMT, int NTW, int NW>
@@ -1099,12 +1108,21 @@ __device__ __forceinline__ void prep_wide(const Params& p, uint8_t* smem) {
         const int t = i & 3, b = (i >> 2) % BP, rest = i / (4 * BP), G = rest & 7, st = rest >> 3;
         uint32_t words[16];
         if (b < p.batch) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x + b * p.k + st * 1024 + G * 128 + 32 * t);
             uint32_t raw[16];
+            if (FMT == BQ_T5P8G128) {
+                // weights 30 t .. 30 t + 29 and 120 + 2 t, 121 + 2 t (4-byte aligned)
+                const uint16_t* xg = p.x + b * p.k + st * 1024 + G * 128;
+                const uint32_t* src = reinterpret_cast<const uint32_t*>(xg + 30 * t);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 v = __ldg(src + q);
-                raw[4 * q] = v.x; raw[4 * q + 1] = v.y; raw[4 * q + 2] = v.z; raw[4 * q + 3] = v.w;
+                for (int q = 0; q < 15; ++q) raw[q] = __ldg(src + q);
+                raw[15] = __ldg(reinterpret_cast<const uint32_t*>(xg + 120 + 2 * t));
+            } else {
+                const uint4* src = reinterpret_cast<const uint4*>(p.x + b * p.k + st * 1024 + G * 128 + 32 * t);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = __ldg(src + q);
+                    raw[4 * q] = v.x; raw[4 * q + 1] = v.y; raw[4 * q + 2] = v.z; raw[4 * q + 3] = v.w;
+                }
             }
             // x 2^e rounded once to FP16 (the two power-of-two products are
             // exact while the value stays in the FP32 normal range; below it
@@ -1164,6 +1182,52 @@ __device__ __forceinline__ void wide_a(uint2 w, uint2 wb, uint32_t S, uint32_t S
     }
 }
 
+// 5-trit format: (c - 1) s of two codes c in {0, 1, 2} held in the halves of
+// c2, as an FP16 pair: (1024 + c) - 1025 = c - 1 exactly, times s exactly.
+__device__ __forceinline__ uint32_t t5_qpair(uint32_t c2, uint32_t S) {
+    const __half2 q = __hsub2(u2h2(c2 | 0x64006400u), u2h2(0x64016401u));
+    return h22u(__hmul2(q, u2h2(S)));
+}
+
+// The five base-3 digits of the two bytes in the halves of v: quotients
+// floor(v / 3^i) by multiply-shift (171 >> 9, 57 >> 9, 19 >> 9, 203 >> 14, exact
+// for every byte; v * m < 2^16, so the halves do not mix once masked), digit i
+// = q_i - 3 q_(i+1) (never negative, so no borrow between the halves).
+__device__ __forceinline__ void t5_digits5(uint32_t v, uint32_t (&d)[5]) {
+    const uint32_t q1 = ((v * 171u) >> 9) & 0x007F007Fu, q2 = ((v * 57u) >> 9) & 0x007F007Fu;
+    const uint32_t q3 = ((v * 19u) >> 9) & 0x007F007Fu, q4 = ((v * 203u) >> 14) & 0x00030003u;
+    d[0] = v - 3u * q1;
+    d[1] = q1 - 3u * q2;
+    d[2] = q2 - 3u * q3;
+    d[3] = q3 - 3u * q4;
+    d[4] = q4;
+}
+
+// The 16 FP16 pairs of one row's group for thread t (pairs as wide_lo /
+// wide_hi): bytes 6t .. 6t+5 paired (j, j + 3) in 16-bit halves, and the
+// thread's two trits of the last eight (bytes 24, 25).  p: the group's 26
+// bytes in shared memory (2-byte aligned); S: the row's FP16 scale in both
+// halves.
+__device__ __forceinline__ void t5_wide_row(const uint8_t* p, int t, uint32_t S, uint32_t (&h)[16]) {
+    const uint32_t u0 = lds_u16(p + 6 * t), u1 = lds_u16(p + 6 * t + 2), u2 = lds_u16(p + 6 * t + 4);
+    const uint32_t ue = lds_u16(p + 24);
+    const uint32_t xs[3] = {(u0 & 0xFFu) | ((u1 >> 8) << 16), (u0 >> 8) | ((u2 & 0xFFu) << 16),
+                            (u1 & 0xFFu) | ((u2 >> 8) << 16)};
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        uint32_t d[5];
+        t5_digits5(xs[j], d);
+#pragma unroll
+        for (int i = 0; i < 5; ++i) h[5 * j + i] = t5_qpair(d[i], S);
+    }
+    // byte 24 (trits 120..124) in the low half, byte 25 (125..127) in the high
+    uint32_t e[5];
+    t5_digits5((ue & 0xFFu) | ((ue >> 8) << 16), e);
+    const uint32_t c0 = (e[0] & 0xFFFFu) | (e[1] << 16), c1 = (e[2] & 0xFFFFu) | (e[3] << 16);
+    const uint32_t c2 = (e[4] & 0xFFFFu) | (e[0] & 0xFFFF0000u), c3 = (e[1] >> 16) | (e[2] & 0xFFFF0000u);
+    h[15] = t5_qpair(t == 0 ? c0 : t == 1 ? c1 : t == 2 ? c2 : c3, S);
+}
+
 // One chunk of CT row tiles, all stages, accumulating in FP32 across K; work
 // split as run_chunk.
 template <int FMT, int NTW, int NW, int CT>
@@ -1173,7 +1237,8 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
     constexpr int WPR = CT >= NW ? 1 : ((NW / CT) < kGroupsPerStage ? (NW / CT) : kGroupsPerStage);
     constexpr int GPW = kGroupsPerStage / WPR;
     constexpr int BP = NTW * 8;
-    constexpr int TSTRIDE = 2048;  // code bytes between row tiles of a column box
+    // code bytes between row tiles (of a column box for the bit formats)
+    constexpr int TSTRIDE = FMT == BQ_T5P8G128 ? tile_code_bytes<FMT>() : 2048;
     const int my_rt = CT >= NW ? warp : warp / WPR;
     const int gsub = CT >= NW ? 0 : warp % WPR;
     const bool active = my_rt < ct;  // (ct <= CT tiles in the chunk; as in run_chunk)
@@ -1210,6 +1275,25 @@ __device__ bool run_chunk_wide(const Params& p, uint8_t* smem, uint64_t* full, u
 #pragma unroll
                 for (int tp = 0; tp < TPW; ++tp) {
                     const uint8_t* codes_t = sb + (my_rt + NW * tp) * TSTRIDE;
+                    if constexpr (FMT == BQ_T5P8G128) {
+                        const uint32_t s0 = (sc[tp][0][gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+                        const uint32_t s1 = (sc[tp][1][gi >> 1] >> (16 * (gi & 1))) & 0xFFFFu;
+                        const uint8_t* r0 = codes_t + g * kT5RowBytes + 26 * G;
+                        uint32_t h0[16], h1[16];
+                        t5_wide_row(r0, t, s0 | (s0 << 16), h0);
+                        t5_wide_row(r0 + 8 * kT5RowBytes, t, s1 | (s1 << 16), h1);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                            for (int nt = 0; nt < NTW; ++nt) {
+                                const uint2 bv = *reinterpret_cast<const uint2*>(
+                                    xs + ((((G * 8 + j) * BP + nt * 8 + g) * 4 + t) * 8));
+                                ptx::mma_f16_16816(acc[tp][nt], h0[2 * j], h1[2 * j], h0[2 * j + 1], h1[2 * j + 1],
+                                                   bv.x, bv.y);
+                            }
+                        }
+                        continue;
+                    }
                     uint2 w, wb;
                     if (FMT == BQ_Q1G128) {
                         const int off = ((G ^ g) << 4) + 4 * t;
@@ -1538,7 +1622,8 @@ cudaError_t encode_maps(int fmt, const uint8_t* codes, const uint16_t* scales, i
 // Wide-batch plan: one CTA of 16 compute warps per SM, the FP16 activation
 // area of all of K resident, a ring of at least two 8-tile slots.
 bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
-    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128) && batch >= 5 && batch <= 16 && k > 0 && k % 1024 == 0 &&
+    if (!((fmt == BQ_Q1G128 || fmt == BQ_T2G128 || fmt == BQ_T5P8G128) && batch >= 5 && batch <= 16 && k > 0 &&
+          k % 1024 == 0 &&
           n > 0 && n <= (int64_t)INT32_MAX - 16 && k <= (int64_t)1 << 20))
         return false;
     pl.nt = batch <= 8 ? 1 : 2;  // n-tiles of eight batch rows
@@ -1548,7 +1633,7 @@ bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
     pl.row_tiles = (int)((n + 15) / 16);
     const int sms = sm_count();
     pl.grid = pl.row_tiles < sms ? pl.row_tiles : sms;
-    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : 4096) + kTileScaleBytes;
+    const int64_t tile_bytes = (fmt == BQ_Q1G128 ? 2048 : fmt == BQ_T2G128 ? 4096 : 16 * kT5RowBytes) + kTileScaleBytes;
     // chunks as in the row-owning kernel: the smallest power of two that holds
     // a CTA's tiles, else (ring of fewer than two slots) the largest within them
     const int most = (pl.row_tiles + pl.grid - 1) / pl.grid;
@@ -1559,10 +1644,15 @@ bool wide_plan(Plan& pl, int fmt, int64_t n, int64_t k, int batch) {
     const int64_t x_area = (int64_t)pl.stages * (pl.nt == 1 ? wide_stage_bytes<1>() : wide_stage_bytes<2>());
     const int64_t red = (int64_t)16 * 32 * pl.nt * 4 * 4;
     const int64_t fixed = 1024 + x_area + red + kWideAux + 2 * kMaxSlots * 8;
+    // (and below that, halved while the activations leave room for fewer than
+    // two slots: a shallow ring of small chunks, e.g. 5-trit codes at K = 5120
+    // and batch 16, rather than the GEMM)
     int64_t slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
-    if ((kSmemFull - fixed) / slot < 2 && pl.chunk_cap != within) {
-        pl.chunk_cap = within;
+    if ((kSmemFull - fixed) / slot < 2 && pl.chunk_cap != within) pl.chunk_cap = within;
+    for (;;) {
         slot = (pl.chunk_cap * tile_bytes + 1023) / 1024 * 1024;
+        if ((kSmemFull - fixed) / slot >= 2 || pl.chunk_cap == 1) break;
+        pl.chunk_cap >>= 1;
     }
     pl.slot_bytes = (int)slot;
     pl.scales_off = pl.chunk_cap * (int)(tile_bytes - kTileScaleBytes);
@@ -1656,7 +1746,8 @@ cudaError_t launch_gemv_wide(int fmt, const uint8_t* codes, const uint16_t* scal
     if (!rows::wide_plan(pl, fmt, n, k, batch)) return cudaErrorInvalidValue;
     if (fmt == BQ_Q1G128)
         return rows::launch_wide_fmt<BQ_Q1G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
-    return rows::launch_wide_fmt<BQ_T2G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    if (fmt == BQ_T2G128) return rows::launch_wide_fmt<BQ_T2G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
+    return rows::launch_wide_fmt<BQ_T5P8G128>(codes, scales, n, k, x, batch, y, y_dtype, pl, s);
 }
 
 

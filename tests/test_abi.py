@@ -105,7 +105,8 @@ def test_argument_errors_need_no_device(lib):
     assert lib.bq_gemv_launches(3, 4096, 4096, 1) == 1       # 5-trit format, row-owning kernel too
     assert lib.bq_gemv_launches(3, 4096, 17408, 4) in (2, 3)  # operand too large: tcgen05 GEMM
     assert lib.bq_gemv_launches(1, 4096, 4096, 16) == 1       # wide-batch kernel
-    assert lib.bq_gemv_launches(3, 4096, 4096, 16) in (2, 3)   # 5-trit format at batch 16: tcgen05 GEMM
+    assert lib.bq_gemv_launches(3, 4096, 4096, 16) == 1        # 5-trit format at batch 16: wide-batch kernel
+    assert lib.bq_gemv_launches(3, 4096, 4096, 8) == 1         # 5-trit format at batch 8: row-owning kernel
     assert lib.bq_gemv_launches(1, 4096, 12288, 16) in (2, 3)  # FP16 x exceeds shared memory: GEMM
     assert lib.bq_gemm_launches(2, 4096, 4096, 12) == 1        # T 5..16: the wide-batch GEMV
     assert lib.bq_gemm_launches(1, 17408, 5120, 4096) == 2     # prep + GEMM, no K split
@@ -125,7 +126,9 @@ def test_gemv_path_choice_host_only(lib):
         for n, k, b in ((4096, 4096, 1), (151936, 4096, 1), (4096, 12288, 1), (777, 1024, 2)):
             assert ws(fmt, n, k, b) == 0 and nl(fmt, n, k, b) == 1, (fmt, n, k, b)   # row-owning
         assert ws(fmt, 4096, 1152, 1) >= 1152 * 2                                 # K % 1024 != 0: GEMM
-    assert ws("t5p8", 4096, 4096, 9) >= 9 * 4096 * 2                              # 5-trit, batch > 8: GEMM
+    # 5-trit at batch 9..16: the wide-batch kernel where its FP16 x fits, else the GEMM
+    assert ws("t5p8", 4096, 4096, 9) == 0 and nl("t5p8", 4096, 4096, 9) == 1
+    assert ws("t5p8", 4096, 12288, 16) >= 16 * 12288 * 2
     for fmt in ("q1g128", "t2g128"):
         # batch 5..16: the wide-batch kernel while its FP16 x (2 K bytes per row,
         # rows padded to 8 or 16) fits: batch 16 at K = 4096 (128 KB), batch 8 at

@@ -41,14 +41,16 @@ def _host_case(fmt, n, k, batch, seed):
     return codes, scales, synth.x_bf16(g, batch, k)
 
 
-# Shapes on every path bq_gemv can take.  The first six need no scratch (the
-# row-owning kernel; the wide-batch kernel at batch 9 and 6); the rest use the
-# fixed array: the split-K kernel (activation operand too large for shared
-# memory at batch 4) and the tcgen05 GEMM with T = batch (the 5-trit format at
-# batch 9, K % 1024 != 0, the 5-trit format at batch 4 and large K).
+# Shapes on every path bq_gemv can take.  The first seven need no scratch (the
+# row-owning kernel; the wide-batch kernel at batch 9 and 6, and for the 5-trit
+# format at batch 9); the rest use the fixed array: the split-K kernel
+# (activation operand too large for shared memory at batch 4) and the tcgen05
+# GEMM with T = batch (the 5-trit format at batch 16 and K = 12288, K % 1024 !=
+# 0, the 5-trit format at batch 4 and large K).
 NO_SCRATCH = [("q1g128", 4096, 4096, 1), ("t2g128", 3000, 2048, 3), ("q1g128", 777, 12288, 2),
-              ("t5p8", 500, 1024, 1), ("q1g128", 16385, 4096, 9), ("t2g128", 129, 8192, 6)]
-SCRATCH = [("t2g128", 4096, 12288, 4), ("q1g128", 4096, 17408, 4), ("t5p8", 4096, 4096, 9),
+              ("t5p8", 500, 1024, 1), ("q1g128", 16385, 4096, 9), ("t2g128", 129, 8192, 6),
+              ("t5p8", 4096, 4096, 9)]
+SCRATCH = [("t2g128", 4096, 12288, 4), ("q1g128", 4096, 17408, 4), ("t5p8", 4096, 12288, 16),
            ("q1g128", 4096, 1152, 1), ("t5p8", 4096, 17408, 4)]
 
 
