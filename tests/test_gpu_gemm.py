@@ -106,8 +106,8 @@ def _edge_tokens(g, t, k):
 @pytest.mark.parametrize("fmt", ["q1g128", "t2g128", "t5p8"])
 @pytest.mark.parametrize("n,k,batch", [(300, 1152, 9), (257, 2176, 16), (200, 1152, 5), (129, 3200, 8)])
 def test_gemm_path_activation_edges_f32(fmt, n, k, batch):
-    """The tcgen05 GEMM (bq_gemv routes K % 1024 != 0 to it with T = batch, and
-    the 5-trit format at batch 9..16) with F32 output on edge-case activations: the per-token
+    """The tcgen05 GEMM (bq_gemv routes K % 1024 != 0 to it with T = batch) with
+    F32 output on edge-case activations: the per-token
     FP16 pre-scale must keep every output within 2e-3 sum|s x| (plus the F32
     rounding of y)."""
     import torch

@@ -1,6 +1,7 @@
-"""The wide-batch decode GEMV (batch 5..16, binary and 2-bit ternary: FP16
-effective weights s * q in the MMA fragments, x pre-scaled per batch row) on
-the GPU against the FP64 oracle at the stated tolerance."""
+"""The wide-batch decode GEMV (batch 5..16 for binary and 2-bit ternary, 9..16
+for 5 trits per byte: FP16 effective weights s * q in the MMA fragments, x
+pre-scaled per batch row) on the GPU against the FP64 oracle at the stated
+tolerance."""
 import numpy as np
 import pytest
 
@@ -26,8 +27,16 @@ WIDE_CASES = [(b, n, k) for b in (5, 6, 8, 9, 12, 16) for n, k in ((33, 1024), (
              [(b, n, k) for b in (9, 16) for n, k in ((16385, 4096), (1001, 5120))]
 
 
-@pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("batch,n,k", WIDE_CASES)
+# 5 trits per byte: batch 9..16 only (batch <= 8 stays on the row-owning
+# kernel); ragged rows, one to six K stages, the 208-byte groups read as pairs
+# of 16-bit halves.
+T5_WIDE_CASES = [(b, n, k) for b in (9, 12, 16) for n, k in ((33, 1024), (300, 2048), (1000, 4096))] + \
+                [(9, 16385, 4096), (16, 16385, 4096), (9, 1001, 5120), (16, 1001, 5120), (10, 777, 3072),
+                 (13, 2047, 6144), (16, 65, 1024)]
+
+
+@pytest.mark.parametrize("fmt,batch,n,k", [(f,) + c for f in FMTS for c in WIDE_CASES] +
+                         [("t5p8",) + c for c in T5_WIDE_CASES])
 def test_wide_shapes(fmt, batch, n, k):
     import torch
     assert bq.bq_gemv_workspace_bytes(fmt, n, k, batch) == 0 and bq.bq_gemv_launches(fmt, n, k, batch) == 1
@@ -42,7 +51,7 @@ def test_wide_shapes(fmt, batch, n, k):
         check_close(y, yref, bound, name, strict=True, what=f"wide {fmt} {n}x{k} b{batch} {name}")
 
 
-@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("fmt", FMTS + ["t5p8"])
 def test_wide_activation_edges(fmt):
     """Per-row pre-scale at the edges: an all-zero row, magnitudes over
     1e-30 .. 1e30, a row with one huge value and the rest at and below 2^-31 of
@@ -77,10 +86,9 @@ def test_wide_activation_edges(fmt):
     assert np.all(y[0].cpu().numpy() == 0.0)
 
 
-@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("fmt,batch", [(f, b) for f in FMTS for b in (8, 16)] + [("t5p8", 16)])
 @pytest.mark.parametrize("shape", [(6144, 4096), (24576, 4096), (151936, 4096), (34816, 5120), (248320, 5120),
                                    (4096, 12288)])
-@pytest.mark.parametrize("batch", [8, 16])
 def test_wide_config_shapes_sampled(fmt, shape, batch):
     """The Qwen3-8B and 27B-class decode shapes at batch 8 and 16 (those the wide
     kernel takes), sampled rows against the oracle."""
@@ -110,16 +118,18 @@ def test_wide_config_shapes_sampled(fmt, shape, batch):
     check_close(y[:, sel], yref, bound, "bf16", strict=True, what=f"wide {fmt} {n}x{k} b{batch}")
 
 
-def test_wide_gemm_tokens_match_gemv():
-    """bq_gemm with 5..16 tokens takes the same kernel as bq_gemv: identical bits."""
+@pytest.mark.parametrize("fmt,tokens", [("q1g128", (5, 9, 16)), ("t5p8", (9, 16))])
+def test_wide_gemm_tokens_match_gemv(fmt, tokens):
+    """bq_gemm with the token counts the wide kernel takes runs the same kernel
+    as bq_gemv: identical bits."""
     import torch
     n, k = 16390, 4096
-    codes, scales = host_weights("q1g128", n, k, synth.SEED_BASE + 830)
+    codes, scales = host_weights(fmt, n, k, synth.SEED_BASE + 830)
     c, s = to_dev(codes), to_dev(scales.astype(np.int16))
-    for t in (5, 9, 16):
+    for t in tokens:
         x = x_to_dev(synth.x_bf16(synth.rng(831 + t), t, k))
-        assert bq.bq_gemm_launches("q1g128", n, k, t) == 1
-        y1 = bq.bq_gemm("q1g128", c, s, n, k, x)
-        y2 = bq.bq_gemv("q1g128", c, s, n, k, x)
+        assert bq.bq_gemm_launches(fmt, n, k, t) == 1
+        y1 = bq.bq_gemm(fmt, c, s, n, k, x)
+        y2 = bq.bq_gemv(fmt, c, s, n, k, x)
         torch.cuda.synchronize()
         assert torch.equal(y1, y2)
