@@ -41,11 +41,6 @@ int sm_count();
 cudaError_t ensure_dynamic_smem(const void* func, int bytes);
 EncodeTiledFn encode_fn();
 
-// BF16 bit pattern -> float (exact).
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
-    return __uint_as_float(b << 16);
-}
-
 // Low / high BF16 of a packed pair -> float.
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
